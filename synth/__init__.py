@@ -1,0 +1,197 @@
+"""Seeded synthetic inputs for the W4A16 weight-only matmul.
+
+This module is shared by both sides of every parity check: the fp64 oracle and
+the CUDA library each take their inputs from here, and nothing here performs
+any of the method's own arithmetic (no dequantisation, no matmul).  It only
+draws random numbers and rounds them to their storage types (BF16, FP8-E4M3).
+
+Generator
+---------
+SplitMix64 (Steele, Lea and Flood, "Fast splittable pseudorandom number
+generators", OOPSLA 2014), used counter-style: element ``i`` of a stream with
+key ``key`` is ``mix64(key + (i + 1) * GAMMA)``, i.e. the (i+1)-th output of a
+SplitMix64 generator seeded with ``key``.  Streams are keyed by
+``(seed, tensor_id)`` through ``stream_key``.  Because every element is a pure
+function of its index, any subset of a tensor (one row of a 248,320-row output
+projection, say) can be regenerated on its own, and the CUDA twin in
+``synth/csrc/synth_gen.cu`` reproduces the same values on the device.
+
+Draws
+-----
+* 4-bit codes: the top 4 bits of the 64-bit output (exactly uniform on 0..15).
+* uniform double in (0, 1): ``((z >> 11) + 0.5) * 2**-53``.
+* standard normal: Box-Muller on the uniforms of counters ``2i`` and ``2i+1``,
+  ``sqrt(-2 ln u1) * cos(2 pi u2)`` (the sine half is not used).
+
+Value recipes (the workload of the 5120-hidden dense model's linears)
+--------------------------------------------------------------------
+* int4 GPTQ weights: q = code - 8, uniform on [-8, 7].
+* int4 group scales (one per 128 K-elements per output column):
+  RNE_bf16(0.01 * exp(0.25 * z)), z ~ N(0, 1); 0.25 is read as the standard
+  deviation of the log-normal exponent.
+* activations: RNE_bf16(z), z ~ N(0, 1).
+* NVFP4 e2m1 codes: uniform on the 16 codes.
+* NVFP4 group scales (one per 16 K-elements per output column):
+  RNE_e4m3(|z| * 0.05), saturating at 448.
+* NVFP4 per-tensor scale: fp32(1/448).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+# Tensor ids: one independent stream per logical tensor of a problem.
+T_Q = 1        # int4 codes
+T_S = 2        # int4 bf16 group scales (normal draws)
+T_X = 3        # activations (normal draws)
+T_C = 4        # nvfp4 e2m1 codes
+T_S8 = 5       # nvfp4 e4m3 group scales (normal draws)
+
+INT4_GROUP = 128
+NVFP4_GROUP = 16
+
+
+def mix64(z: np.ndarray) -> np.ndarray:
+    """SplitMix64 output function (the 'mix' finaliser), on uint64 arrays."""
+    z = np.asarray(z, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z = (z ^ (z >> np.uint64(30))) * _M1
+        z = (z ^ (z >> np.uint64(27))) * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def stream_key(seed: int, tensor_id: int) -> np.uint64:
+    """Key of the stream for one tensor of one seeded problem."""
+    with np.errstate(over="ignore"):
+        a = mix64(np.uint64(seed & 0xFFFFFFFFFFFFFFFF) + GAMMA)
+        b = mix64(a + np.uint64(tensor_id) * GAMMA)
+    return np.uint64(b)
+
+
+def raw64(seed: int, tensor_id: int, index: np.ndarray) -> np.ndarray:
+    """64-bit outputs for the given element indices of one stream."""
+    key = stream_key(seed, tensor_id)
+    idx = np.asarray(index, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        return mix64(key + (idx + np.uint64(1)) * GAMMA)
+
+
+def codes4(seed: int, tensor_id: int, index: np.ndarray) -> np.ndarray:
+    """Uniform 4-bit codes (0..15) from the top bits."""
+    return (raw64(seed, tensor_id, index) >> np.uint64(60)).astype(np.uint8)
+
+
+def _unit(z: np.ndarray) -> np.ndarray:
+    return ((z >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+
+
+def normals(seed: int, tensor_id: int, index: np.ndarray) -> np.ndarray:
+    """Standard normals (float64) by Box-Muller on counters 2i and 2i+1."""
+    idx = np.asarray(index, dtype=np.uint64)
+    u1 = _unit(raw64(seed, tensor_id, idx * np.uint64(2)))
+    u2 = _unit(raw64(seed, tensor_id, idx * np.uint64(2) + np.uint64(1)))
+    return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+
+
+# ---------------------------------------------------------------- rounding to storage types
+
+
+def to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """Round float64 values to BF16 (round to nearest, ties to even); uint16 bits.
+
+    Normal range: keep 8 significant bits of the binary mantissa from frexp;
+    BF16 subnormal range (below 2**-126): quantum 2**-133.  Values here stay
+    far from overflow.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(v)
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+    small = np.abs(v) < 2.0 ** -126
+    r = np.where(small, np.ldexp(np.rint(np.ldexp(v, 133)), -133), r)
+    return (r.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def to_e4m3_bytes(v: np.ndarray) -> np.ndarray:
+    """Round non-negative float64 values to OCP FP8-E4M3 (RNE, saturating at 448)."""
+    v = np.asarray(v, dtype=np.float64)
+    if np.any(v < 0) or np.any(~np.isfinite(v)):
+        raise ValueError("e4m3 scale draws must be finite and non-negative")
+    m, e = np.frexp(v)
+    r = np.ldexp(np.rint(np.ldexp(m, 4)), e - 4)          # 4 significant bits
+    sub = v < 2.0 ** -6
+    r = np.where(sub, np.ldexp(np.rint(np.ldexp(v, 9)), -9), r)  # quantum 2**-9
+    r = np.minimum(r, 448.0)
+    out = np.zeros(v.shape, dtype=np.uint8)
+    nz = r > 0
+    is_sub = nz & (r < 2.0 ** -6)
+    out[is_sub] = np.ldexp(r[is_sub], 9).astype(np.uint8)
+    nrm = nz & ~is_sub
+    mm, ee = np.frexp(r[nrm])                              # r = mm * 2**ee, mm in [0.5, 1)
+    field = (ee - 1 + 7).astype(np.int64)
+    mant = (np.ldexp(mm, 4) - 8).astype(np.int64)          # 3 fraction bits
+    out[nrm] = ((field << 3) | mant).astype(np.uint8)
+    return out
+
+
+# ---------------------------------------------------------------- problem tensors
+
+
+def int4_weights(seed: int, N: int, K: int, rows=None) -> np.ndarray:
+    """q[n][k] as int8 in [-8, 7]; ``rows`` selects a subset of output columns n."""
+    rows = np.arange(N, dtype=np.uint64) if rows is None else np.asarray(rows, dtype=np.uint64)
+    idx = rows[:, None] * np.uint64(K) + np.arange(K, dtype=np.uint64)[None, :]
+    return (codes4(seed, T_Q, idx).astype(np.int16) - 8).astype(np.int8)
+
+
+def int4_scales(seed: int, N: int, K: int, rows=None) -> np.ndarray:
+    """BF16 bits of the per-(column, 128-group) scales, shape [len(rows)][K/128]."""
+    G = K // INT4_GROUP
+    rows = np.arange(N, dtype=np.uint64) if rows is None else np.asarray(rows, dtype=np.uint64)
+    idx = rows[:, None] * np.uint64(G) + np.arange(G, dtype=np.uint64)[None, :]
+    return to_bf16_bits(0.01 * np.exp(0.25 * normals(seed, T_S, idx)))
+
+
+def activations(seed: int, M: int, K: int) -> np.ndarray:
+    """BF16 bits of x[m][k] ~ N(0, 1), shape [M][K]."""
+    idx = np.arange(M * K, dtype=np.uint64).reshape(M, K)
+    return to_bf16_bits(normals(seed, T_X, idx))
+
+
+def nvfp4_codes(seed: int, N: int, K: int, rows=None) -> np.ndarray:
+    rows = np.arange(N, dtype=np.uint64) if rows is None else np.asarray(rows, dtype=np.uint64)
+    idx = rows[:, None] * np.uint64(K) + np.arange(K, dtype=np.uint64)[None, :]
+    return codes4(seed, T_C, idx)
+
+
+def nvfp4_scales(seed: int, N: int, K: int, rows=None) -> np.ndarray:
+    """E4M3 bytes of the per-(column, 16-group) scales, shape [len(rows)][K/16]."""
+    G = K // NVFP4_GROUP
+    rows = np.arange(N, dtype=np.uint64) if rows is None else np.asarray(rows, dtype=np.uint64)
+    idx = rows[:, None] * np.uint64(G) + np.arange(G, dtype=np.uint64)[None, :]
+    return to_e4m3_bytes(np.abs(normals(seed, T_S8, idx)) * 0.05)
+
+
+NVFP4_GLOBAL_SCALE = float(np.float32(1.0 / 448.0))
+
+
+def problem(fmt: str, seed: int, M: int, N: int, K: int, rows=None) -> dict:
+    """All logical tensors of one seeded problem (host numpy arrays).
+
+    fmt: "int4" or "nvfp4".  Returns codes/scales/x (+ g for nvfp4).  The
+    activations of a problem are keyed by the same seed as its weights.
+    """
+    if fmt == "int4":
+        return {"fmt": fmt, "M": M, "N": N, "K": K,
+                "codes": int4_weights(seed, N, K, rows),
+                "scales": int4_scales(seed, N, K, rows),
+                "x": activations(seed, M, K), "g": None}
+    if fmt == "nvfp4":
+        return {"fmt": fmt, "M": M, "N": N, "K": K,
+                "codes": nvfp4_codes(seed, N, K, rows),
+                "scales": nvfp4_scales(seed, N, K, rows),
+                "x": activations(seed, M, K), "g": NVFP4_GLOBAL_SCALE}
+    raise ValueError(fmt)

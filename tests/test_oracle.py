@@ -1,0 +1,365 @@
+"""Pins for the fp64 oracle: decoders, rounding, dequantisation and the matmul.
+
+Each check compares the oracle against something other than itself: exact
+rational arithmetic built from the formats' bit fields (tests/exact.py),
+hand-derived worked examples, closed forms and invariants.  CPU only.
+"""
+
+from __future__ import annotations
+
+import random
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import formats
+import synth
+from exact import (bf16_bits_of, bf16_value, e2m1_value, e4m3_value, fp32_value,
+                   E2M1_MAGNITUDES, pow2)
+
+G_NVFP4 = synth.NVFP4_GLOBAL_SCALE          # fp32(1/448)
+G_BITS = int(np.float32(G_NVFP4).view(np.uint32))
+
+
+# ---------------------------------------------------------------- decoders
+
+
+def test_bf16_decoder_exhaustive():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = formats.bf16_to_f64(bits)
+    for b in range(65536):
+        ref = bf16_value(b)
+        if ref == "nan":
+            assert np.isnan(got[b])
+        elif ref == "+inf":
+            assert got[b] == np.inf
+        elif ref == "-inf":
+            assert got[b] == -np.inf
+        else:
+            assert Fraction(got[b]) == ref, hex(b)
+
+
+def test_e4m3_decoder_exhaustive():
+    got = formats.e4m3_to_f64(np.arange(256, dtype=np.uint8))
+    for b in range(256):
+        ref = e4m3_value(b)
+        if ref == "nan":
+            assert np.isnan(got[b]), hex(b)
+        else:
+            assert Fraction(got[b]) == ref, hex(b)
+    # landmarks of the OCP definition
+    assert got[0x38] == 1.0
+    assert got[0x7E] == 448.0
+    assert got[0x01] == 2.0 ** -9
+    assert got[0x08] == 2.0 ** -6
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF])
+    assert got[0xFE] == -448.0
+
+
+def test_e2m1_decoder_table():
+    got = formats.e2m1_to_f64(np.arange(16, dtype=np.uint8))
+    listed = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    for c in range(16):
+        want = listed[c & 7] * (-1 if c & 8 else 1)
+        assert got[c] == want
+        assert Fraction(got[c]) == e2m1_value(c)
+    assert np.signbit(got[8])                      # code 0x8 is -0
+    # field decode agrees with the listed magnitudes
+    for c in range(8):
+        e, m = (c >> 1) & 3, c & 1
+        v = Fraction(m, 2) if e == 0 else (1 + Fraction(m, 2)) * pow2(e - 1)
+        assert v == E2M1_MAGNITUDES[c]
+
+
+# ---------------------------------------------------------------- rounding onto BF16
+
+
+def _random_bf16(rng):
+    e = rng.randint(1, 254)
+    return (rng.randint(0, 1) << 15) | (e << 7) | rng.randint(0, 127)
+
+
+def test_rne_bf16_against_exact_rationals():
+    rng = random.Random(1234)
+    vals = []
+    # exact products of the kinds the method forms, plus ties and subnormals
+    for _ in range(3000):
+        q = rng.randint(-8, 7)
+        s = _random_bf16(rng)
+        vals.append(q * bf16_value(s))
+    for _ in range(2000):
+        c = rng.randint(0, 15)
+        b = rng.randint(0, 0x7E)
+        g = fp32_value(rng.randint(0x30000000, 0x42000000))
+        vals.append(e2m1_value(c) * e4m3_value(b) * g)
+    # exact midpoints between adjacent BF16 values (ties), subnormal to large
+    for b in list(range(0, 0x0100, 7)) + list(range(0x0100, 0x7F7F, 97)):
+        lo, hi = bf16_value(b), bf16_value(b + 1)
+        vals.append((lo + hi) / 2)
+        vals.append(-(lo + hi) / 2)
+    x = np.array([float(v) for v in vals], dtype=np.float64)
+    assert all(Fraction(float(v)) == v for v in vals)  # binary64 holds every case exactly
+    got = formats.f64_to_bf16_rne(x)
+    for v, g in zip(vals, got):
+        assert int(g) == bf16_bits_of(v), (v, hex(int(g)), hex(bf16_bits_of(v)))
+
+
+def test_worked_examples_hand_derived():
+    # s = BF16 0x3C24 = 1.28125 * 2**-7 = 0.010009765625.
+    s = np.array([[0x3C24]], dtype=np.uint16)
+    assert formats.bf16_to_f64(s)[0, 0] == 0.010009765625
+    # q = 7: 7 s = 0.070068359375 = 143.5 * 2**-11 sits exactly between the BF16
+    # neighbours 143 * 2**-11 (0x3D8F) and 144 * 2**-11 (0x3D90); ties go to the
+    # even mantissa, 0x3D90 = 0.0703125 (truncation would give 0x3D8F).
+    q = np.full((1, 128), 7, dtype=np.int8)
+    w = oracle.dequant_int4_g128(q, s)
+    assert int(w[0, 0]) == 0x3D90
+    # q = -8: -8 s = -0.080078125 is exact in BF16: 0xBDA4.
+    w = oracle.dequant_int4_g128(np.full((1, 128), -8, dtype=np.int8), s)
+    assert int(w[0, 0]) == 0xBDA4
+    # NVFP4: code 7 (6.0) x E4M3 0x38 (1.0) x fp32(1/448): 6/448 = 1.7142857 * 2**-7
+    # -> 8-bit significand 219.43/128 -> 219 -> 0x3C5B = 0.01336669921875.
+    c = np.full((1, 16), 7, dtype=np.uint8)
+    w = oracle.dequant_nvfp4(c, np.array([[0x38]], dtype=np.uint8), G_NVFP4)
+    assert int(w[0, 0]) == 0x3C5B
+    assert formats.bf16_to_f64(w)[0, 0] == 0.01336669921875
+    # code 3 (1.5) x 0x30 (0.5) x g = 0.75/448 -> 0.00167083740234375
+    c = np.full((1, 16), 3, dtype=np.uint8)
+    w = oracle.dequant_nvfp4(c, np.array([[0x30]], dtype=np.uint8), G_NVFP4)
+    assert formats.bf16_to_f64(w)[0, 0] == 0.00167083740234375
+
+
+# ---------------------------------------------------------------- dequantisation
+
+
+def _stratified_bf16_scales():
+    """Every sign/exponent with 16 mantissas, plus all mantissas of 3 binades."""
+    out = set()
+    for sign in (0, 1):
+        for e in range(0, 255):                  # finite exponents incl. subnormal
+            for m in range(0, 128, 8):
+                out.add((sign << 15) | (e << 7) | m)
+            out.add((sign << 15) | (e << 7) | 127)
+    for e in (1, 120, 254):
+        for m in range(128):
+            out.add((e << 7) | m)
+    return sorted(out)
+
+
+def test_dequant_int4_all_codes_stratified_scales():
+    scales = _stratified_bf16_scales()
+    q = np.tile(np.repeat(np.arange(-8, 8, dtype=np.int8), 8), (len(scales), 1))  # K = 128
+    s = np.array(scales, dtype=np.uint16)[:, None]
+    w = oracle.dequant_int4_g128(q, s)
+    for i, sb in enumerate(scales):
+        sv = bf16_value(sb)
+        for j in range(0, 128, 8):
+            qv = int(q[i, j])
+            prod = qv * sv
+            neg_zero = (prod == 0) and ((qv < 0) != (sb >= 0x8000)) and qv != 0
+            want = bf16_bits_of(prod, negative_zero=neg_zero)
+            got = int(w[i, j])
+            if prod == 0:
+                assert got & 0x7FFF == 0
+            else:
+                assert got == want, (qv, hex(sb), hex(got), hex(want))
+
+
+@pytest.mark.parametrize("g_bits", [G_BITS, 0x3F800000, 0x3DCCCCCD, 0x3B449BA6, 0x4B7FFFFF])
+def test_dequant_nvfp4_all_code_scale_pairs(g_bits):
+    g = float(np.array([g_bits], dtype=np.uint32).view(np.float32)[0])
+    finite = [b for b in range(256) if e4m3_value(b) != "nan"]
+    codes = np.tile(np.arange(16, dtype=np.uint8), (len(finite), 1))     # K = 16
+    s8 = np.array(finite, dtype=np.uint8)[:, None]
+    w = oracle.dequant_nvfp4(codes, s8, g)
+    gv = fp32_value(g_bits)
+    for i, b in enumerate(finite):
+        for c in range(16):
+            prod = e2m1_value(c) * e4m3_value(b) * gv
+            got = int(w[i, c])
+            if prod == 0:
+                assert got & 0x7FFF == 0
+            else:
+                assert got == bf16_bits_of(prod), (c, hex(b), hex(got))
+
+
+def test_dequant_group_index_is_k_div_group():
+    # one distinct power-of-two scale per group: the group a k belongs to is
+    # read back from the exponent of W_deq when q = 1
+    N, K = 3, 512
+    q = np.ones((N, K), dtype=np.int8)
+    s = np.zeros((N, K // 128), dtype=np.uint16)
+    for n in range(N):
+        for g in range(K // 128):
+            s[n, g] = (127 + 4 * g + n) << 7     # 2**(4g+n)
+    w = formats.bf16_to_f64(oracle.dequant_int4_g128(q, s))
+    for n in range(N):
+        for k in range(K):
+            assert w[n, k] == 2.0 ** (4 * (k // 128) + n)
+    c = np.full((2, 64), 2, dtype=np.uint8)        # e2m1 code 2 = 1.0
+    s8 = np.zeros((2, 4), dtype=np.uint8)
+    for n in range(2):
+        for g in range(4):
+            s8[n, g] = (7 + g + 2 * n) << 3       # 2**(g+2n)
+    w = formats.bf16_to_f64(oracle.dequant_nvfp4(c, s8, 1.0))
+    for n in range(2):
+        for k in range(64):
+            assert w[n, k] == 2.0 ** ((k // 16) + 2 * n)
+
+
+def test_dequant_rejects_out_of_contract_inputs():
+    with pytest.raises(ValueError):
+        oracle.dequant_int4_g128(np.full((1, 128), 8, dtype=np.int8), np.zeros((1, 1), np.uint16))
+    with pytest.raises(ValueError):
+        oracle.dequant_int4_g128(np.zeros((1, 100), dtype=np.int8), np.zeros((1, 1), np.uint16))
+    with pytest.raises(ValueError):
+        oracle.dequant_nvfp4(np.zeros((1, 16), np.uint8), np.array([[0x7F]], np.uint8), 1.0)
+
+
+# ---------------------------------------------------------------- the matmul
+
+
+def _exact_y(x_bits, w_bits):
+    M, K = x_bits.shape
+    N = w_bits.shape[0]
+    xs = [[bf16_value(int(b)) for b in row] for row in x_bits]
+    ws = [[bf16_value(int(b)) for b in row] for row in w_bits]
+    return [[sum(xs[m][k] * ws[n][k] for k in range(K)) for n in range(N)] for m in range(M)]
+
+
+@pytest.mark.parametrize("fmt,M,N,K,seed", [("int4", 1, 4, 128, 11), ("int4", 3, 2, 256, 12),
+                                             ("nvfp4", 2, 3, 128, 13), ("nvfp4", 1, 4, 256, 14)])
+def test_gemm_brute_force_exact(fmt, M, N, K, seed):
+    p = synth.problem(fmt, seed, M, N, K)
+    w = (oracle.dequant_int4_g128(p["codes"], p["scales"]) if fmt == "int4"
+         else oracle.dequant_nvfp4(p["codes"], p["scales"], p["g"]))
+    y = oracle.gemm_ref(p["x"], w)
+    bound = oracle.abs_bound(p["x"], w)
+    ex = _exact_y(p["x"], w)
+    for m in range(M):
+        for n in range(N):
+            # binary64 accumulation of K exact products: error <= K * 2**-53 * bound
+            assert abs(Fraction(y[m, n]) - ex[m][n]) <= Fraction(K) * pow2(-52) * Fraction(bound[m, n])
+            assert abs(y[m, n]) <= bound[m, n] * (1 + 1e-12)
+
+
+def _int4_case(seed=21, M=4, N=40, K=384):
+    p = synth.problem("int4", seed, M, N, K)
+    return p, oracle.dequant_int4_g128(p["codes"], p["scales"])
+
+
+def test_invariant_zero_scales_give_zero():
+    p, _ = _int4_case()
+    w = oracle.dequant_int4_g128(p["codes"], np.zeros_like(p["scales"]))
+    assert np.all(oracle.gemm_ref(p["x"], w) == 0)
+    c = synth.nvfp4_codes(3, 8, 64)
+    w = oracle.dequant_nvfp4(c, np.zeros((8, 4), np.uint8), G_NVFP4)
+    assert np.all(formats.bf16_to_f64(w) == 0)
+
+
+def test_invariant_one_hot_selects_a_dequantised_column():
+    p, w = _int4_case()
+    K = p["K"]
+    for k in (0, 1, 127, 128, 200, K - 1):
+        x = np.zeros((1, K), dtype=np.uint16)
+        x[0, k] = 0x3F80                               # 1.0
+        y = oracle.gemm_ref(x, w)
+        assert np.array_equal(y[0], formats.bf16_to_f64(w[:, k]))
+
+
+def test_invariant_power_of_two_scaling_is_exact():
+    p, w = _int4_case()
+    x2 = (p["x"].astype(np.int32) + (1 << 7)).astype(np.uint16)     # exponent + 1: 2x
+    nz = (p["x"] & 0x7F80) != 0
+    x2 = np.where(nz, x2, p["x"])
+    assert np.array_equal(oracle.gemm_ref(x2, w), 2 * oracle.gemm_ref(p["x"], w))
+
+
+def test_invariant_linearity_and_row_independence():
+    p, w = _int4_case()
+    x1 = formats.bf16_to_f64(p["x"])
+    x2 = formats.bf16_to_f64(synth.activations(99, p["M"], p["K"]))
+    # a and b chosen so that a*x1 + b*x2 stays exact enough: compare in fp64
+    lhs = (0.5 * x1 + 0.25 * x2) @ formats.bf16_to_f64(w).T
+    rhs = 0.5 * oracle.gemm_ref(p["x"], w) + 0.25 * oracle.gemm_ref(synth.activations(99, p["M"], p["K"]), w)
+    bound = oracle.abs_bound(p["x"], w) + oracle.abs_bound(synth.activations(99, p["M"], p["K"]), w)
+    assert np.all(np.abs(lhs - rhs) <= 1e-12 * bound + 1e-300)
+    y = oracle.gemm_ref(p["x"], w)
+    for m in range(p["M"]):
+        assert np.array_equal(oracle.gemm_ref(p["x"][m:m + 1], w)[0], y[m])
+
+
+def test_invariant_column_permutation():
+    p, w = _int4_case()
+    perm = np.random.default_rng(5).permutation(p["N"])
+    wp = oracle.dequant_int4_g128(p["codes"][perm], p["scales"][perm])
+    assert np.array_equal(oracle.gemm_ref(p["x"], wp), oracle.gemm_ref(p["x"], w)[:, perm])
+
+
+def test_tolerance_helper():
+    y_ref = np.array([[1.0, -2.0]])
+    bound = np.array([[128.0, 0.0]])
+    ok, ex = oracle.within_tolerance(np.array([[2.0, -2.0005]]), y_ref, bound)
+    assert ok.all()
+    ok, ex = oracle.within_tolerance(np.array([[2.01, -2.002]]), y_ref, bound)
+    assert not ok.any()
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+
+def _pin_suite(dequant_int4, gemm):
+    """A compact re-run of the pins above against a (possibly mutated) oracle."""
+    fails = []
+    s = np.array([[0x3C24]], dtype=np.uint16)
+    if int(dequant_int4(np.full((1, 128), 7, np.int8), s)[0, 0]) != 0x3D90:
+        fails.append("tie")
+    if int(dequant_int4(np.full((1, 128), -8, np.int8), s)[0, 0]) != 0xBDA4:
+        fails.append("sign")
+    N, K = 2, 256
+    q = np.ones((N, K), dtype=np.int8)
+    sc = np.array([[0x3F80, 0x4000], [0x4080, 0x4100]], dtype=np.uint16)   # 1, 2, 4, 8
+    w = formats.bf16_to_f64(dequant_int4(q, sc))
+    if not (np.all(w[0, :128] == 1) and np.all(w[0, 128:] == 2) and np.all(w[1, :128] == 4)
+            and np.all(w[1, 128:] == 8)):
+        fails.append("group index")
+    p = synth.problem("int4", 31, 2, 3, 256)
+    wd = oracle.dequant_int4_g128(p["codes"], p["scales"])
+    y = gemm(p["x"], wd)
+    ex = _exact_y(p["x"], wd)
+    if any(abs(Fraction(y[m, n]) - ex[m][n]) > Fraction(1, 1 << 30) for m in range(2) for n in range(3)):
+        fails.append("matmul")
+    return fails
+
+
+def test_pins_catch_planted_mistakes():
+    assert _pin_suite(oracle.dequant_int4_g128, oracle.gemm_ref) == []
+
+    def truncating(q, s):          # rounds toward zero instead of to nearest even
+        v = q.astype(np.float64) * np.repeat(formats.bf16_to_f64(s), 128, axis=1)
+        return (v.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+    def wrong_group(q, s):         # scale index k // 64 instead of k // 128
+        idx = np.minimum(np.arange(q.shape[1]) // 64, s.shape[1] - 1)
+        v = q.astype(np.float64) * formats.bf16_to_f64(s)[:, idx]
+        return formats.f64_to_bf16_rne(v)
+
+    def offset_sign(q, s):         # uses the stored offset-binary code q + 8 as the value
+        v = (q.astype(np.float64) + 8) * np.repeat(formats.bf16_to_f64(s), 128, axis=1)
+        return formats.f64_to_bf16_rne(v)
+
+    def transposed(x, w):          # transposed operand / wrong axis of the sum
+        xf, wf = formats.bf16_to_f64(x), formats.bf16_to_f64(w)
+        return (xf[:, ::-1] @ wf.T)
+
+    def dropped_term(x, w):        # drops the last product of every dot product
+        xf, wf = formats.bf16_to_f64(x), formats.bf16_to_f64(w)
+        return xf[:, :-1] @ wf[:, :-1].T
+
+    assert "tie" in _pin_suite(truncating, oracle.gemm_ref)
+    assert "group index" in _pin_suite(wrong_group, oracle.gemm_ref)
+    assert "sign" in _pin_suite(offset_sign, oracle.gemm_ref)
+    assert "matmul" in _pin_suite(oracle.dequant_int4_g128, transposed)
+    assert "matmul" in _pin_suite(oracle.dequant_int4_g128, dropped_term)
