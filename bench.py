@@ -1,0 +1,592 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 weight-only matmul on B200.
+
+Metric: W4A16 GEMM achieved HBM GB/s (and fraction of roofline) at decode and
+speculative-verify row counts, one B200.
+
+One step = the four decode linears of the 5120-hidden, 64-layer dense model at
+M = 1 (int4 GPTQ g128): QKV 5120->8192, O 6144->5120, gate/up 5120->34816,
+down 17408->5120, run back to back on one stream.  ``value`` is algorithmic
+bytes (packed weights + scales + activations + outputs) per second over the
+timed steps, aggregated over all GPUs.  The other configurations (every row
+count, NVFP4, the 64-layer sweep) are reported in ``sweep`` / ``whole_stack``.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+Multi-GPU: launched by torchrun, one process per GPU; each GPU runs its own
+replica of the workload (the path needs no exchange between GPUs).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DECODE_SHAPES = [("qkv", 5120, 8192, 1), ("o", 6144, 5120, 2), ("gate_up", 5120, 34816, 3),
+                 ("down", 17408, 5120, 4)]
+METRIC = "W4A16 GEMM achieved HBM GB/s & % of roofline at M=1/4/9/16/64 (1 B200)"
+UNIT = "GB/s"
+WORKLOAD = ("decode-shape int4 g128 W4A16, M=1: QKV 5120->8192, O 6144->5120, "
+            "gate/up 5120->34816, down 17408->5120 (seeds 1-4)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def alg_bytes(fmt, M, N, K):
+    w = N * K * (0.5 + (2 / 128 if fmt == "int4" else 1 / 16)) + (4 if fmt == "nvfp4" else 0)
+    return w + 2 * M * K + 2 * M * N
+
+
+def flops(M, N, K):
+    return 2.0 * M * N * K
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def load_traffic():
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu summary,
+    valid only while the kernel sources hash the same as when it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_weight_only_dequant_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, out_path=None):
+        self.samples = []
+        self.proc = None
+        self.gpu_id = gpu_id
+        self.out_path = out_path
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+        if self.out_path:
+            with open(self.out_path, "w") as f:
+                for ts, line in self.samples:
+                    f.write(f"{ts:.3f},{line}\n")
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.samples:
+            if t0 <= ts <= t1:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- the CPU oracle baseline
+
+
+def cpu_oracle_sample(seconds: float):
+    """Run the fp64 oracle on blocks of output columns of the decode shapes until
+    ``seconds`` of oracle time have passed (input generation not counted);
+    returns (GB/s of weight+scale bytes processed, description, seconds)."""
+    import oracle
+    import synth
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        pass
+    block = 256
+    done_bytes = 0.0
+    done_rows = {name: 0 for name, *_ in DECODE_SHAPES}
+    xs = {K: synth.activations(seed, 1, K) for _, K, _, seed in DECODE_SHAPES}
+    busy = 0.0
+    wall0 = time.perf_counter()
+    i = 0
+    while busy < seconds and time.perf_counter() - wall0 < 4 * seconds:
+        name, K, N, seed = DECODE_SHAPES[i % len(DECODE_SHAPES)]
+        r0 = done_rows[name] % N
+        rows = np.arange(r0, min(N, r0 + block))
+        p = synth.problem("int4", seed, 1, N, K, rows=rows)
+        t0 = time.perf_counter()
+        wd = oracle.dequant_int4_g128(p["codes"], p["scales"])
+        oracle.gemm_ref(xs[K], wd)
+        busy += time.perf_counter() - t0
+        done_rows[name] += len(rows)
+        done_bytes += len(rows) * K * (0.5 + 2 / 128)
+        i += 1
+    desc = (f"fp64 oracle (dequantise then matmul), 1 thread, on blocks of {block} output columns "
+            f"of the four decode shapes at M=1, round robin, {busy:.1f} s of oracle time: "
+            + ", ".join(f"{k} {v} rows" for k, v in done_rows.items())
+            + "; GB/s of packed weight+scale bytes; input generation not counted")
+    return done_bytes / busy / 1e9, desc, busy
+
+
+def cpu_oracle_step(rows_per_shape: int):
+    """One reference step: the oracle on the first rows of every decode shape."""
+    import oracle
+    import synth
+    total = 0.0
+    t_work = 0.0
+    for name, K, N, seed in DECODE_SHAPES:
+        rows = np.arange(min(N, rows_per_shape))
+        p = synth.problem("int4", seed, 1, N, K, rows=rows)
+        t0 = time.perf_counter()
+        wd = oracle.dequant_int4_g128(p["codes"], p["scales"])
+        oracle.gemm_ref(p["x"], wd)
+        t_work += time.perf_counter() - t0
+        total += len(rows) * K * (0.5 + 2 / 128)
+    return total, t_work
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:
+        pass
+    rows = 256
+    for _ in range(args.warmup):
+        cpu_oracle_step(rows)
+    tot_b = tot_t = 0.0
+    for _ in range(args.steps):
+        b, t = cpu_oracle_step(rows)
+        tot_b += b
+        tot_t += t
+    value = tot_b / tot_t / 1e9
+    sample = (f"fp64 oracle on the first {rows} output columns of each decode shape per step "
+              f"(weights + scales of {tot_b / args.steps / 1e6:.1f} MB per step), 1 thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded SplitMix64)",
+            "config": {"workload": WORKLOAD, "M": 1, "fmt": "int4_g128"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU side
+
+
+def make_weights(fmt, seed, N, K, copies):
+    import torch
+    import synth
+    from bit_weight_only_dequant_b200 import w4a16 as W
+    p = synth.device_problem(fmt, seed, 1, N, K)
+    pw, ps = W.pack_on_device(fmt, N, K, p["codes"], p["scales"])
+    del p
+    ws = [(pw, ps)]
+    for _ in range(copies - 1):
+        ws.append((pw.clone(), ps.clone()))
+    torch.cuda.synchronize()
+    return ws
+
+
+def make_x(fmt, seed, M, K):
+    import torch
+    import synth
+    x = torch.empty((M, K), dtype=torch.int16, device="cuda")
+    synth.device_fill(synth.KIND_X, seed, synth.T_X, x)
+    return x.view(torch.bfloat16)
+
+
+def copies_for(weight_bytes):
+    """Weight copies to rotate so one cycle is at least 3x the L2 size."""
+    return max(2, min(16, int(np.ceil(3 * L2_BYTES / max(1, weight_bytes)))))
+
+
+def time_launch_list(launches, reps, stream):
+    """Capture ``reps`` rounds of ``launches`` (callables issuing one GEMM each)
+    in a CUDA graph with an event pair around every launch; replay it once.
+    Returns (total ms, per-launch ms list of lists)."""
+    import torch
+    evs = [[(torch.cuda.Event(enable_timing=True, external=True),
+             torch.cuda.Event(enable_timing=True, external=True)) for _ in launches]
+           for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for r in range(reps):
+            for j, fn in enumerate(launches):
+                evs[r][j][0].record()
+                fn(r)
+                evs[r][j][1].record()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    g.replay()  # warm replay
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record()
+        g.replay()
+        end.record()
+    torch.cuda.synchronize()
+    per = [[b.elapsed_time(e) for b, e in row] for row in evs]
+    total = start.elapsed_time(end)
+    del g
+    return total, per
+
+
+def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
+    import torch
+    from bit_weight_only_dequant_b200 import w4a16 as W
+    f = W.FMTS[fmt]
+    wbytes = W.w4a16_packed_weight_bytes(f, N, K) + W.w4a16_packed_scale_bytes(f, N, K)
+    copies = copies_for(wbytes)
+    ws = make_weights(fmt, seed, N, K, copies)
+    x = make_x(fmt, seed, M, K)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
+    path = W.w4a16_gemm_path(f, M, N, K)
+
+    def launch(r, ws=ws):
+        pw, ps = ws[r % len(ws)]
+        W.check(W.w4a16_gemm(f, M, N, K, x, pw, ps, g, y, stream.cuda_stream), "gemm")
+
+    with torch.cuda.stream(stream):
+        for r in range(3):
+            launch(r)
+    torch.cuda.synchronize()
+    _, per = time_launch_list([launch], reps, stream)
+    us = float(np.mean([p[0] for p in per[1:]])) * 1e3
+    b = alg_bytes(fmt, M, N, K)
+    fl = flops(M, N, K)
+    t_mem = b / (peaks["hbm_gbs"] * 1e9)
+    t_tc = fl / (peaks["bf16_tflops"] * 1e12)
+    t_roof = max(t_mem, t_tc)
+    del ws
+    torch.cuda.empty_cache()
+    return {"fmt": fmt, "shape": name, "K": K, "N": N, "M": M, "path": int(path),
+            "us": round(us, 3), "GBps": round(b / us / 1e3, 1), "TFLOPs": round(fl / us / 1e6, 2),
+            "bound": "hbm" if t_mem >= t_tc else "tensor",
+            "frac_roofline": round(t_roof * 1e6 / us, 4),
+            "frac_of_8TBps": round(b / us / 1e3 / 8000.0, 4)}
+
+
+def whole_stack(Ms, peaks, stream, reps=3):
+    """64 layers x (QKV, O, gate/up, down) + the 5120->248320 output projection,
+    int4 g128, weights of layer l drawn with seed 7+l and the output projection
+    with seed 71; the linears do not feed each other (one x per distinct K)."""
+    import torch
+    from bit_weight_only_dequant_b200 import w4a16 as W
+    layers = []
+    for l in range(64):
+        for name, K, N, _ in DECODE_SHAPES:
+            (pw, ps), = make_weights("int4", 7 + l, N, K, 1)
+            layers.append((K, N, pw, ps))
+    (pw, ps), = make_weights("int4", 71, 248320, 5120, 1)
+    layers.append((5120, 248320, pw, ps))
+    wbytes = sum(W.w4a16_packed_weight_bytes(0, N, K) + W.w4a16_packed_scale_bytes(0, N, K)
+                 for K, N, _, _ in layers)
+    out = {"layers": 64, "gemms_per_step": len(layers), "weight_and_scale_bytes_per_step": int(wbytes),
+           "weights_per_step": int(sum(N * K for K, N, _, _ in layers)), "by_M": {}}
+    for M in Ms:
+        xs = {K: make_x("int4", 7, M, K) for K in (5120, 6144, 17408)}
+        ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+              for N in (8192, 5120, 34816, 248320)}
+
+        def step(r, M=M, xs=xs, ys=ys):
+            for K, N, pw, ps in layers:
+                W.check(W.w4a16_gemm(0, M, N, K, xs[K], pw, ps, None, ys[N], stream.cuda_stream),
+                        "gemm")
+
+        with torch.cuda.stream(stream):
+            step(0)
+        torch.cuda.synchronize()
+        total, _ = time_launch_list([step], reps, stream)
+        ms = total / reps
+        b = sum(alg_bytes("int4", M, N, K) for K, N, _, _ in layers)
+        fl = sum(flops(M, N, K) for K, N, _, _ in layers)
+        out["by_M"][str(M)] = {"ms_per_step": round(ms, 4), "steps_per_s": round(1e3 / ms, 2),
+                               "GBps": round(b / ms / 1e6, 1), "TFLOPs": round(fl / ms / 1e9, 2),
+                               "weight_bound_steps_per_s_at_peak": round(
+                                   peaks["hbm_gbs"] * 1e9 / wbytes, 1)}
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from bit_weight_only_dequant_b200 import w4a16 as W
+
+    torch.cuda.set_device(local_rank)
+    W.lib()
+    peaks = load_peaks()
+    stream = torch.cuda.Stream()
+    M = 1
+
+    # ---- the workload: four decode linears, weights rotated over enough copies
+    wsets = []
+    for name, K, N, seed in DECODE_SHAPES:
+        wsets.append((name, K, N, seed))
+    step_wbytes = sum(W.w4a16_packed_weight_bytes(0, N, K) + W.w4a16_packed_scale_bytes(0, N, K)
+                      for _, K, N, _ in wsets)
+    copies = copies_for(step_wbytes)
+    weights = {name: make_weights("int4", seed, N, K, copies) for name, K, N, seed in wsets}
+    xs = {name: make_x("int4", seed, M, K) for name, K, N, seed in wsets}
+    ys = {name: torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for name, K, N, _ in wsets}
+    step_bytes = sum(alg_bytes("int4", M, N, K) for _, K, N, _ in wsets)
+
+    def gemm_fn(name, K, N):
+        def fn(r):
+            pw, ps = weights[name][r % copies]
+            W.check(W.w4a16_gemm(0, M, N, K, xs[name], pw, ps, None, ys[name],
+                                 stream.cuda_stream), "gemm")
+        return fn
+
+    launches = [gemm_fn(name, K, N) for name, K, N, _ in wsets]
+    with torch.cuda.stream(stream):
+        for w in range(max(3, args.warmup)):
+            for fn in launches:
+                fn(w)
+    torch.cuda.synchronize()
+    W.check(W.w4a16_device_status(stream.cuda_stream), "device status")
+
+    # ---- capture the K timed steps (per-launch events), soak, then time one replay
+    evs = [[(torch.cuda.Event(enable_timing=True, external=True),
+             torch.cuda.Event(enable_timing=True, external=True)) for _ in launches]
+           for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(args.steps):
+            for j, fn in enumerate(launches):
+                evs[i][j][0].record()
+                fn(i)
+                evs[i][j][1].record()
+    props = torch.cuda.get_device_properties(local_rank)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
+    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+    sampler = ClockSampler(gpu_id, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv"))
+    sampler.start()
+    time.sleep(0.3)
+    t_soak = time.time()
+    soak_until = t_soak + args.soak
+    while time.time() < soak_until:
+        graph.replay()
+        torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        start.record()
+        graph.replay()
+        end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_end = time.time()
+    time.sleep(0.25)
+    sampler.stop()
+    ms_total = start.elapsed_time(end)
+    per = np.array([[b.elapsed_time(e) for b, e in row] for row in evs])  # ms
+    W.check(W.w4a16_device_status(stream.cuda_stream), "device status")
+    if world > 1:
+        tt = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_per_step = ms_total / args.steps
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    clocks = sampler.summary(t_soak, t_end)
+    del graph
+
+    # ---- dominant kernel: the GEMV launches (every launch of the step)
+    launch_bytes = np.array([alg_bytes("int4", M, N, K) for _, K, N, _ in wsets])
+    avg_ms = float(per.mean())
+    achieved = float(launch_bytes.mean() / (avg_ms * 1e-3) / 1e9)
+    traffic = load_traffic()
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": (traffic or {}).get("dram_bytes_per_launch"),
+                "peak_source": peaks["source"] + " (STREAM-style copy)",
+                "kernel": "gemv_kernel<int4, 1 m-tile> (all four launches of the step)",
+                "per_shape_us": {name: round(float(per[:, j].mean()) * 1e3, 3)
+                                 for j, (name, *_) in enumerate(wsets)},
+                "per_shape_frac": {name: round(float(launch_bytes[j] / (per[:, j].mean() * 1e-3)
+                                                     / 1e9 / peaks["hbm_gbs"]), 4)
+                                   for j, (name, *_) in enumerate(wsets)}}
+
+    # ---- end to end through the C ABI with host buffers
+    xh = {name: torch.empty((M, K), dtype=torch.bfloat16).pin_memory() for name, K, _, _ in wsets}
+    yh = {name: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for name, _, N, _ in wsets}
+    for name in xh:
+        xh[name].copy_(xs[name].cpu())
+    h2d = sum(M * K * 2 for _, K, _, _ in wsets)
+    d2h = sum(M * N * 2 for _, _, N, _ in wsets)
+
+    def e2e_step(i):
+        with torch.cuda.stream(stream):
+            for (name, K, N, _), fn in zip(wsets, launches):
+                xs[name].copy_(xh[name], non_blocking=True)
+                fn(i)
+                yh[name].copy_(ys[name], non_blocking=True)
+        stream.synchronize()
+
+    for i in range(3):
+        e2e_step(i)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        e2e_step(i)
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        tt = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_s = float(tt.item())
+    e2e = {"value": round(world * step_bytes * args.steps / e2e_s / 1e9, 1), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": round(e2e_s / args.steps * 1e3, 4),
+           "how": "pinned host x -> device copy, w4a16_gemm via the C ABI, device -> pinned host y, "
+                  "stream synchronize, per step, wall clock"}
+    del weights
+    torch.cuda.empty_cache()
+
+    extra = {}
+    if world == 1 and not args.no_sweep:
+        entries = []
+        target = [("int4", "target", 5120, 17408, 1, 3)]
+        cfg2 = [("int4", n, K, N, 1, s) for n, K, N, s in DECODE_SHAPES]
+        cfg3 = [("int4", n, K, N, Mv, 5) for Mv in (2, 4, 9, 16, 64) for n, K, N, _ in DECODE_SHAPES]
+        cfg4 = [("nvfp4", n, K, N, Mv, 6) for Mv in (1, 9, 64) for n, K, N, _ in DECODE_SHAPES]
+        for fmt, n, K, N, Mv, s in target + cfg2 + cfg3 + cfg4:
+            entries.append(sweep_entry(fmt, n, K, N, Mv, s, peaks, stream))
+        extra["sweep"] = entries
+    if world == 1 and not args.no_stack:
+        extra["whole_stack"] = whole_stack((1, 16, 64), peaks, stream)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        v, desc, secs = cpu_oracle_sample(args.cpu_seconds)
+        cpu = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded SplitMix64 draws with the checkpoint geometry)",
+                "config": {"workload": WORKLOAD, "M": 1, "fmt": "int4_g128",
+                           "bytes_per_step": int(step_bytes),
+                           "l2": f"inputs larger than L2: {copies} weight copies rotated "
+                                 f"({copies * step_wbytes / 1e6:.0f} MB per cycle, L2 126 MB)",
+                           "timing": "CUDA graph of the K steps, CUDA events on the launching "
+                                     "stream, max over ranks",
+                           "replicas": world},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+                "gpu_launches": len(launches) * args.steps,
+                "peaks": peaks}
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--soak", type=float, default=1.5, help="seconds of untimed replays first")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-stack", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,241 @@
+// C ABI of the library (include/w4a16.h): argument validation, per-device
+// state, the row-count dispatcher and the split-K workspace.
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/w4a16.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+struct DeviceState {
+  bool checked = false;
+  bool ok = false;        // sm_100
+  int num_sms = 0;
+  unsigned* err = nullptr;  // device error word
+};
+
+struct Workspace {
+  void* base = nullptr;   // [counters (uint32)] [partials (fp32)]
+  size_t counters = 0;
+  size_t floats = 0;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceState> g_dev;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.checked) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return W4A16_ERR_CUDA;
+    d.ok = prop.major == 10 && prop.minor == 0;
+    d.num_sms = prop.multiProcessorCount;
+    if (d.ok) {
+      if (cudaMalloc(&d.err, sizeof(unsigned)) != cudaSuccess) return W4A16_ERR_NOMEM;
+      if (cudaMemset(d.err, 0, sizeof(unsigned)) != cudaSuccess) return W4A16_ERR_CUDA;
+    }
+    d.checked = true;
+  }
+  if (!d.ok) return W4A16_ERR_DEVICE;
+  *out = &d;
+  return W4A16_OK;
+}
+
+// Workspace of at least (counters, floats) for the current device and `st`.
+// Grows by reallocation in stream order; counters start (and are left) zero.
+int workspace(cudaStream_t st, size_t counters, size_t floats, unsigned** cnt, float** part) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[std::make_pair(dev, st)];
+  if (w.base == nullptr || w.counters < counters || w.floats < floats) {
+    size_t nc = counters > w.counters ? counters : w.counters;
+    size_t nf = floats > w.floats ? floats : w.floats;
+    if (nc < 65536) nc = 65536;
+    if (nf < (1u << 20)) nf = 1u << 20;
+    nc = (nc + 63) / 64 * 64;
+    void* base = nullptr;
+    if (cudaMallocAsync(&base, nc * sizeof(unsigned) + nf * sizeof(float), st) != cudaSuccess)
+      return W4A16_ERR_NOMEM;
+    if (cudaMemsetAsync(base, 0, nc * sizeof(unsigned), st) != cudaSuccess) return W4A16_ERR_CUDA;
+    if (w.base) cudaFreeAsync(w.base, st);
+    w.base = base;
+    w.counters = nc;
+    w.floats = nf;
+  }
+  *cnt = static_cast<unsigned*>(w.base);
+  *part = reinterpret_cast<float*>(static_cast<unsigned*>(w.base) + w.counters);
+  return W4A16_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_fmt_shape(int fmt, int N, int K) {
+  if (fmt != W4A16_FMT_INT4_G128 && fmt != W4A16_FMT_NVFP4_G16) return W4A16_ERR_ARG;
+  if (N < 1 || K < 128 || K % 128 != 0) return W4A16_ERR_SHAPE;
+  // packed tensors are addressed with 32-bit tile/scale indices in places
+  if ((long long)((N + 15) / 16) * (K / 64) >= (1ll << 31) / 64) return W4A16_ERR_SHAPE;
+  return W4A16_OK;
+}
+
+int choose_path(int fmt, int M, int N, int K) {
+  (void)fmt;
+  (void)N;
+  (void)K;
+  if (M <= 16) return W4A16_PATH_GEMV;
+  return W4A16_PATH_GEMV;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t w4a16_packed_weight_bytes(int fmt, int N, int K) {
+  if (check_fmt_shape(fmt, N, K) != W4A16_OK) return 0;
+  return (size_t)w4::weight_bytes(N, K);
+}
+
+size_t w4a16_packed_scale_bytes(int fmt, int N, int K) {
+  if (check_fmt_shape(fmt, N, K) != W4A16_OK) return 0;
+  return (size_t)w4::scale_bytes(fmt, N, K);
+}
+
+int w4a16_pack_host(int fmt, int N, int K, const void* codes, const void* scales, void* packed_w,
+                    void* packed_scales) {
+  const int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (!codes || !scales || !packed_w || !packed_scales) return W4A16_ERR_ARG;
+  return w4::pack_host(fmt, N, K, codes, scales, packed_w, packed_scales) == 0 ? W4A16_OK
+                                                                               : W4A16_ERR_ARG;
+}
+
+int w4a16_unpack_host(int fmt, int N, int K, const void* packed_w, const void* packed_scales,
+                      void* codes, void* scales) {
+  const int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (!codes || !scales || !packed_w || !packed_scales) return W4A16_ERR_ARG;
+  return w4::unpack_host(fmt, N, K, packed_w, packed_scales, codes, scales) == 0 ? W4A16_OK
+                                                                                 : W4A16_ERR_ARG;
+}
+
+int w4a16_pack(int fmt, int N, int K, const void* codes, const void* scales, void* packed_w,
+               void* packed_scales, void* stream) {
+  int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (!codes || !scales || !packed_w || !packed_scales) return W4A16_ERR_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(packed_w) || !aligned16(packed_scales))
+    return W4A16_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if ((r = device_state(&d)) != W4A16_OK) return r;
+  return status_of(w4::launch_pack(fmt, N, K, codes, scales, packed_w, packed_scales,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packed_scales,
+                  const float* global_scale, void* w_bf16, void* stream) {
+  int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (!packed_w || !packed_scales || !w_bf16) return W4A16_ERR_ARG;
+  if ((fmt == W4A16_FMT_NVFP4_G16) != (global_scale != nullptr)) return W4A16_ERR_ARG;
+  if (!aligned16(packed_w) || !aligned16(packed_scales) || !aligned16(w_bf16))
+    return W4A16_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if ((r = device_state(&d)) != W4A16_OK) return r;
+  return status_of(w4::launch_dequant(fmt, N, K, packed_w, packed_scales, global_scale, w_bf16,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int w4a16_gemm_path(int fmt, int M, int N, int K) {
+  const int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (M < 1 || M > W4A16_MAX_M) return W4A16_ERR_SHAPE;
+  return choose_path(fmt, M, N, K);
+}
+
+int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
+                  const void* packed_scales, const float* global_scale, void* y_bf16,
+                  void* stream) {
+  int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (M < 1 || M > W4A16_MAX_M) return W4A16_ERR_SHAPE;
+  if (path != W4A16_PATH_AUTO && path != W4A16_PATH_GEMV && path != W4A16_PATH_TC)
+    return W4A16_ERR_ARG;
+  if (!x_bf16 || !packed_w || !packed_scales || !y_bf16) return W4A16_ERR_ARG;
+  if ((fmt == W4A16_FMT_NVFP4_G16) != (global_scale != nullptr)) return W4A16_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(packed_w) || !aligned16(packed_scales) ||
+      !aligned16(y_bf16))
+    return W4A16_ERR_ALIGN;
+  if (path == W4A16_PATH_AUTO) path = choose_path(fmt, M, N, K);
+  if (path == W4A16_PATH_TC) return W4A16_ERR_SHAPE;  // not available in this build
+  DeviceState* d = nullptr;
+  if ((r = device_state(&d)) != W4A16_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  w4::GemmArgs a;
+  a.fmt = fmt;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.x = x_bf16;
+  a.w = packed_w;
+  a.s = packed_scales;
+  a.g = global_scale;
+  a.y = y_bf16;
+  a.ws = nullptr;
+  a.counters = nullptr;
+  a.err = d->err;
+  const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, d->num_sms);
+  const size_t nf = w4::gemv_workspace_floats(pl, M, N);
+  if (nf > 0) {
+    if ((r = workspace(st, w4::gemv_counters(pl, N), nf, &a.counters, &a.ws)) != W4A16_OK) return r;
+  }
+  return status_of(w4::launch_gemv(pl, a, st));
+}
+
+int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
+               const void* packed_scales, const float* global_scale, void* y_bf16, void* stream) {
+  return w4a16_gemm_ex(W4A16_PATH_AUTO, fmt, M, N, K, x_bf16, packed_w, packed_scales,
+                       global_scale, y_bf16, stream);
+}
+
+int w4a16_device_status(void* stream) {
+  DeviceState* d = nullptr;
+  int r = device_state(&d);
+  if (r != W4A16_OK) return r;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return W4A16_ERR_CUDA;
+  unsigned h = 0;
+  if (cudaMemcpy(&h, d->err, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return W4A16_ERR_CUDA;
+  if (h) {
+    if (cudaMemset(d->err, 0, sizeof(unsigned)) != cudaSuccess) return W4A16_ERR_CUDA;
+    return W4A16_ERR_TIMEOUT;
+  }
+  return W4A16_OK;
+}
+
+const char* w4a16_status_string(int status) {
+  switch (status) {
+    case W4A16_OK: return "W4A16_OK";
+    case W4A16_ERR_ARG: return "W4A16_ERR_ARG: bad argument";
+    case W4A16_ERR_SHAPE: return "W4A16_ERR_SHAPE: unsupported M, N or K";
+    case W4A16_ERR_ALIGN: return "W4A16_ERR_ALIGN: pointer not 16-byte aligned";
+    case W4A16_ERR_DEVICE: return "W4A16_ERR_DEVICE: current device is not sm_100";
+    case W4A16_ERR_CUDA: return "W4A16_ERR_CUDA: CUDA runtime error";
+    case W4A16_ERR_TIMEOUT: return "W4A16_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    case W4A16_ERR_NOMEM: return "W4A16_ERR_NOMEM: workspace allocation failed";
+    default: return "unknown status";
+  }
+}
+
+int w4a16_version(void) { return 100; }
+
+}  // extern "C"

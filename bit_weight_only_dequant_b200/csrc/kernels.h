@@ -1,0 +1,48 @@
+// Internal launch interface between the C ABI (capi.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace w4 {
+
+struct GemmArgs {
+  int fmt;
+  int M, N, K;
+  const void* x;        // [M][K] bf16
+  const void* w;        // packed weights
+  const void* s;        // packed scales
+  const float* g;       // nvfp4 per-tensor scale (device) or null
+  void* y;              // [M][N] bf16
+  float* ws;            // split-K partials (fp32), may be null when no split is used
+  unsigned* counters;   // per 16-row band arrival counters (zero between calls)
+  unsigned* err;        // device error word
+};
+
+// ---------------------------------------------------------------- GEMV (M <= 16)
+
+struct GemvPlan {
+  int S;         // K splits
+  int kslice;    // K elements per split (multiple of 128)
+  int ctas_x;    // CTAs per split
+  int mt;        // 8-row activation tiles (1: M <= 8, 2: M <= 16)
+  int smem;      // dynamic shared memory bytes
+};
+
+GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms);
+// Bytes of fp32 workspace and number of counters the plan needs.
+size_t gemv_workspace_floats(const GemvPlan& p, int M, int N);
+size_t gemv_counters(const GemvPlan& p, int N);
+cudaError_t launch_gemv(const GemvPlan& p, const GemmArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- dequant export / packer
+
+cudaError_t launch_dequant(int fmt, int N, int K, const void* w, const void* s, const float* g,
+                           void* out, cudaStream_t st);
+cudaError_t launch_pack(int fmt, int N, int K, const void* codes, const void* scales, void* w,
+                        void* s, cudaStream_t st);
+// Host packer / unpacker; 0 on success, -1 on an out-of-range code or scale.
+int pack_host(int fmt, int N, int K, const void* codes, const void* scales, void* w, void* s);
+int unpack_host(int fmt, int N, int K, const void* w, const void* s, void* codes, void* scales);
+
+}  // namespace w4

@@ -1,0 +1,158 @@
+/*
+ * w4a16.h - C ABI of the W4A16 weight-only 4-bit matmul library for NVIDIA
+ * B200 (sm_100a).
+ *
+ * What it computes: y[M][N] = x[M][K] . W_deq[N][K]^T, with BF16 activations
+ * x, BF16 outputs y, and weights stored in one of two 4-bit checkpoint
+ * formats, dequantised on the fly:
+ *
+ *  - W4A16_FMT_INT4_G128: symmetric GPTQ-style int4, q in [-8, 7], one BF16
+ *    scale per group of 128 K-elements per output column, no zero point, no
+ *    act-order (the checkpoint contract in the NVIDIA developer-forum post
+ *    "Qwen3.8-27B on single DGX Spark ...", section "Quality").
+ *    W_deq[n][k] = RNE_bf16(q[n][k] * s[n][k/128]).
+ *  - W4A16_FMT_NVFP4_G16: FP4-E2M1 values, one FP8-E4M3 scale per 16
+ *    K-elements per output column, one FP32 per-tensor scale g (the
+ *    compressed-tensors nvfp4-pack-quantized format of the model card
+ *    "Qwen3.8 27B - NVFP4 for veloGB10", section "Specifications"; group 16
+ *    per "SuperQwen3.8-27b-abliterated-NVFP4-2xDGX", "Release highlights").
+ *    W_deq[n][k] = RNE_bf16(e2m1(c[n][k]) * e4m3(s8[n][k/16]) * g).
+ *
+ * Row counts are those of single-token decode and speculative verification
+ * (M = 1 .. 64): the full model checks several drafted tokens in one batched
+ * pass (blog post "One Config Line Made My 27B Model 2.7x Faster", section
+ * "The fix: use the MTP head you already downloaded").  The kernel is picked
+ * by row count (forum post above, section "How").
+ *
+ * Conventions shared by every entry point:
+ *  - Every call returns a status (W4A16_OK or a negative W4A16_ERR_*), never
+ *    throws and never aborts.  Arguments are validated before any launch.
+ *  - Device calls are asynchronous and ordered on the given stream (a
+ *    cudaStream_t passed as void*, NULL = legacy default stream).  The library
+ *    keeps no pointer after a call returns; buffers must stay alive until the
+ *    stream has executed the work.
+ *  - The caller owns every buffer passed in.  The GEMM keeps a small
+ *    library-owned fp32 workspace per (device, stream) for split-K partial
+ *    sums; it is allocated on the first call that needs it on that stream
+ *    (make that first call before capturing the stream into a CUDA graph).
+ *  - Accuracy: per element |y - y_ref| <= 2^-7 * sum_k |W_deq[n][k] x[m][k]|
+ *    + 1e-3 against the fp64 dequantise-then-matmul, and w4a16_dequant is
+ *    bit-exact.  The NVFP4 path rescales each activation row slice by a power
+ *    of two into FP16 for the tensor cores: elements more than 2^29 below their
+ *    row slice's largest magnitude lose low bits (absolute error at most
+ *    2^-40 of that largest magnitude per element).
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Weight formats. */
+#define W4A16_FMT_INT4_G128 0
+#define W4A16_FMT_NVFP4_G16 1
+
+/* Status codes. */
+#define W4A16_OK 0
+#define W4A16_ERR_ARG (-1)     /* bad format, null pointer, out-of-range code, bad path id */
+#define W4A16_ERR_SHAPE (-2)   /* M, N or K outside the supported range */
+#define W4A16_ERR_ALIGN (-3)   /* a device pointer is not 16-byte aligned */
+#define W4A16_ERR_DEVICE (-4)  /* the current device is not sm_100 */
+#define W4A16_ERR_CUDA (-5)    /* a CUDA runtime call or launch failed */
+#define W4A16_ERR_TIMEOUT (-6) /* a kernel gave up a bounded wait (see w4a16_device_status) */
+#define W4A16_ERR_NOMEM (-7)   /* the workspace could not be allocated */
+
+/* Limits of this version. */
+#define W4A16_MAX_M 64         /* decode / speculative-verify row counts */
+
+/* Kernel paths (for w4a16_gemm_path / w4a16_gemm_ex). */
+#define W4A16_PATH_AUTO 0      /* row-count dispatch */
+#define W4A16_PATH_GEMV 1      /* CUDA-core/mma.sync split-K GEMV, M <= 16 */
+#define W4A16_PATH_TC 2        /* tcgen05 tensor-core path, 16 <= M <= 64 */
+
+/*
+ * Shape rules: 1 <= M <= 64; N >= 1 (any value; packed buffers are padded to
+ * a multiple of 16 rows); K >= 128 and K a multiple of 128 (both formats).
+ */
+
+/* Bytes of the packed weight buffer: ceil(N/16)*16 * K / 2.  0 on bad args. */
+size_t w4a16_packed_weight_bytes(int fmt, int N, int K);
+
+/* Bytes of the packed scale buffer: INT4 ceil(N/16)*16 * K/128 * 2;
+ * NVFP4 ceil(N/16)*16 * K/16.  0 on bad args. */
+size_t w4a16_packed_scale_bytes(int fmt, int N, int K);
+
+/*
+ * Host-side packer: logical checkpoint tensors -> the library's packed layout.
+ *   codes:  INT4: int8 q[N][K] in [-8, 7];  NVFP4: uint8 e2m1 codes c[N][K] in 0..15.
+ *   scales: INT4: BF16 bit patterns (uint16) s[N][K/128];
+ *           NVFP4: E4M3 bytes s8[N][K/16] (0x7F/0xFF NaN patterns rejected).
+ *   packed_w / packed_scales: host buffers of the sizes above.
+ * All pointers are host pointers.  Returns W4A16_ERR_ARG on an out-of-range
+ * code or scale (nothing useful is left in the outputs then).
+ */
+int w4a16_pack_host(int fmt, int N, int K, const void* codes, const void* scales,
+                    void* packed_w, void* packed_scales);
+
+/* Inverse of w4a16_pack_host (host pointers), for round-trip checks. */
+int w4a16_unpack_host(int fmt, int N, int K, const void* packed_w, const void* packed_scales,
+                      void* codes, void* scales);
+
+/*
+ * Device-side packer: same layouts as w4a16_pack_host, all four pointers are
+ * device pointers, asynchronous on `stream`.  Codes outside the format's range
+ * are not detected (only their low 4 bits are stored).
+ */
+int w4a16_pack(int fmt, int N, int K, const void* codes, const void* scales,
+               void* packed_w, void* packed_scales, void* stream);
+
+/*
+ * Dequantise to BF16, bit-exact:
+ *   w_bf16[n][k] = W_deq[n][k] for n < N, k < K (row-major [N][K], device).
+ * global_scale: NVFP4: device pointer to one fp32 g; INT4: must be NULL.
+ */
+int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packed_scales,
+                  const float* global_scale, void* w_bf16, void* stream);
+
+/*
+ * The matmul: y[M][N] = x[M][K] . W_deq[N][K]^T.
+ *   x_bf16:   device, [M][K] BF16 row-major, 16-byte aligned.
+ *   packed_w, packed_scales: device, produced by a packer above, 16-byte aligned.
+ *   global_scale: NVFP4: device pointer to one fp32 g; INT4: must be NULL.
+ *   y_bf16:   device, [M][N] BF16 row-major; must not overlap any input.
+ * Picks the kernel by row count (W4A16_PATH_AUTO).
+ */
+int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
+               const void* packed_scales, const float* global_scale, void* y_bf16, void* stream);
+
+/* Same as w4a16_gemm with an explicit path (W4A16_PATH_*); W4A16_ERR_SHAPE if
+ * the path does not support M. */
+int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16,
+                  const void* packed_w, const void* packed_scales, const float* global_scale,
+                  void* y_bf16, void* stream);
+
+/* The path W4A16_PATH_AUTO would take for these arguments (>0), or a status. */
+int w4a16_gemm_path(int fmt, int M, int N, int K);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word that
+ * kernels set when a bounded wait gives up.  Returns W4A16_OK,
+ * W4A16_ERR_TIMEOUT, or W4A16_ERR_CUDA if the synchronisation itself failed.
+ */
+int w4a16_device_status(void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* w4a16_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int w4a16_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

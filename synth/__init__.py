@@ -195,3 +195,77 @@ def problem(fmt: str, seed: int, M: int, N: int, K: int, rows=None) -> dict:
                 "scales": nvfp4_scales(seed, N, K, rows),
                 "x": activations(seed, M, K), "g": NVFP4_GLOBAL_SCALE}
     raise ValueError(fmt)
+
+
+# ---------------------------------------------------------------- device twin (CUDA)
+
+import ctypes as _ctypes
+import os as _os
+
+_HERE = _os.path.dirname(_os.path.abspath(__file__))
+_DEV_LIB_PATH = _os.path.join(_HERE, "libw4a16_synth.so")
+_dev_lib = None
+
+KIND_INT4_Q, KIND_INT4_S, KIND_X, KIND_NVFP4_C, KIND_NVFP4_S = 0, 1, 2, 3, 4
+
+
+def build_device_generator(force: bool = False, verbose: bool = False) -> str:
+    """Compile synth/csrc/synth_gen.cu into synth/libw4a16_synth.so (sm_100a)."""
+    import shutil
+    import subprocess
+    src = _os.path.join(_HERE, "csrc", "synth_gen.cu")
+    if not force and _os.path.exists(_DEV_LIB_PATH) and \
+            _os.path.getmtime(_DEV_LIB_PATH) >= _os.path.getmtime(src):
+        return _DEV_LIB_PATH
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
+           "-Xcompiler", "-fPIC", "-shared", "-o", _DEV_LIB_PATH, src, "-lcudart"]
+    if verbose:
+        import sys
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.run(cmd, check=True)
+    return _DEV_LIB_PATH
+
+
+def _device_lib():
+    global _dev_lib
+    if _dev_lib is None:
+        if not _os.path.exists(_DEV_LIB_PATH):
+            raise RuntimeError(f"{_DEV_LIB_PATH} is missing: run __graft_entry__.build()")
+        lib = _ctypes.CDLL(_DEV_LIB_PATH)
+        lib.synth_generate.argtypes = [_ctypes.c_int, _ctypes.c_ulonglong, _ctypes.c_int,
+                                       _ctypes.c_longlong, _ctypes.c_void_p, _ctypes.c_void_p]
+        lib.synth_generate.restype = _ctypes.c_int
+        _dev_lib = lib
+    return _dev_lib
+
+
+def device_fill(kind: int, seed: int, tensor_id: int, out, stream=None) -> None:
+    """Fill a contiguous torch CUDA tensor with the stream's first numel() draws."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(out.device).cuda_stream
+    r = _device_lib().synth_generate(kind, seed & 0xFFFFFFFFFFFFFFFF, tensor_id, out.numel(),
+                                     out.data_ptr(), stream)
+    if r != 0:
+        raise RuntimeError(f"synth_generate failed ({r})")
+
+
+def device_problem(fmt: str, seed: int, M: int, N: int, K: int, device="cuda"):
+    """The tensors of ``problem(fmt, seed, M, N, K)``, drawn on the GPU (torch tensors)."""
+    import torch
+    if fmt == "int4":
+        codes = torch.empty((N, K), dtype=torch.int8, device=device)
+        scales = torch.empty((N, K // INT4_GROUP), dtype=torch.int16, device=device)
+        device_fill(KIND_INT4_Q, seed, T_Q, codes)
+        device_fill(KIND_INT4_S, seed, T_S, scales)
+        g = None
+    else:
+        codes = torch.empty((N, K), dtype=torch.uint8, device=device)
+        scales = torch.empty((N, K // NVFP4_GROUP), dtype=torch.uint8, device=device)
+        device_fill(KIND_NVFP4_C, seed, T_C, codes)
+        device_fill(KIND_NVFP4_S, seed, T_S8, scales)
+        g = NVFP4_GLOBAL_SCALE
+    x = torch.empty((M, K), dtype=torch.int16, device=device)
+    device_fill(KIND_X, seed, T_X, x)
+    return {"fmt": fmt, "M": M, "N": N, "K": K, "codes": codes, "scales": scales, "x": x, "g": g}

@@ -1,0 +1,290 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Bars: dequantised weights bit-exact; GEMM outputs within
+|y - y_ref| <= 2^-7 * sum_k |W_deq x| + 1e-3 per element.
+"""
+
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import formats
+import synth
+from bit_weight_only_dequant_b200 import w4a16 as W
+from gpu_util import (SEEDS, SHAPES, assert_parity, bf16_bits, gscale_tensor, oracle_weights,
+                      run_gemm, to_device_problem, torch)
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    t = torch()
+    if not t.cuda.is_available():
+        pytest.skip("no CUDA device")
+    W.lib()
+    yield
+
+
+# ---------------------------------------------------------------- the generator's two twins agree
+
+
+@pytest.mark.parametrize("kind,tensor,dtype,count", [
+    (synth.KIND_INT4_Q, synth.T_Q, "int8", 1 << 20),
+    (synth.KIND_INT4_S, synth.T_S, "int16", 1 << 18),
+    (synth.KIND_X, synth.T_X, "int16", 1 << 18),
+    (synth.KIND_NVFP4_C, synth.T_C, "uint8", 1 << 20),
+    (synth.KIND_NVFP4_S, synth.T_S8, "uint8", 1 << 18)])
+def test_device_generator_matches_host(kind, tensor, dtype, count):
+    t = torch()
+    out = t.empty(count, dtype=getattr(t, dtype), device="cuda")
+    synth.device_fill(kind, 17, tensor, out)
+    got = out.cpu().numpy()
+    idx = np.arange(count, dtype=np.uint64)
+    if kind == synth.KIND_INT4_Q:
+        want = (synth.codes4(17, tensor, idx).astype(np.int16) - 8).astype(np.int8)
+    elif kind == synth.KIND_NVFP4_C:
+        want = synth.codes4(17, tensor, idx)
+    elif kind == synth.KIND_INT4_S:
+        want = synth.to_bf16_bits(0.01 * np.exp(0.25 * synth.normals(17, tensor, idx))).view(np.int16)
+    elif kind == synth.KIND_X:
+        want = synth.to_bf16_bits(synth.normals(17, tensor, idx)).view(np.int16)
+    else:
+        want = synth.to_e4m3_bytes(np.abs(synth.normals(17, tensor, idx)) * 0.05)
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------- dequantisation, bit-exact
+
+
+def test_dequant_int4_exhaustive_codes_and_scales():
+    """All 16 codes x every finite BF16 scale pattern (65,024 rows of K = 128)."""
+    t = torch()
+    pats = np.array([b for b in range(65536) if (b & 0x7F80) != 0x7F80], dtype=np.uint16)
+    N, K = len(pats), 128
+    q = np.tile(((np.arange(K) % 16) - 8).astype(np.int8), (N, 1))
+    s = pats[:, None]
+    codes = t.from_numpy(q).cuda()
+    scales = t.from_numpy(s.view(np.int16).copy()).cuda()
+    pw, ps = W.pack_on_device("int4", N, K, codes, scales)
+    got = bf16_bits(W.dequant("int4", N, K, pw, ps))
+    want = oracle.dequant_int4_g128(q, s)
+    diff = np.argwhere(got != want)
+    assert diff.size == 0, [(int(pats[i]), int(q[i, j]), hex(got[i, j]), hex(want[i, j]))
+                            for i, j in diff[:8]]
+
+
+@pytest.mark.parametrize("g_bits", [0x3B124925, 0x3F800000, 0x3DCCCCCD, 0x4B7FFFFF, 0x0DA24260])
+def test_dequant_nvfp4_exhaustive_codes_and_scales(g_bits):
+    """All 16 codes x all 254 finite E4M3 scales, for several per-tensor scales."""
+    t = torch()
+    finite = np.array([b for b in range(256) if (b & 0x7F) != 0x7F], dtype=np.uint8)
+    N, K = len(finite), 128
+    c = np.tile((np.arange(K) % 16).astype(np.uint8), (N, 1))
+    s8 = np.repeat(finite[:, None], K // 16, axis=1)
+    g = float(np.array([g_bits], np.uint32).view(np.float32)[0])
+    pw, ps = W.pack_on_device("nvfp4", N, K, t.from_numpy(c).cuda(), t.from_numpy(s8).cuda())
+    got = bf16_bits(W.dequant("nvfp4", N, K, pw, ps, global_scale=gscale_tensor(g)))
+    want = oracle.dequant_nvfp4(c, s8, g)
+    diff = np.argwhere(got != want)
+    assert diff.size == 0, [(hex(int(finite[i])), int(c[i, j]), hex(got[i, j]), hex(want[i, j]))
+                            for i, j in diff[:8]]
+
+
+@pytest.mark.parametrize("fmt,name", [("int4", "qkv"), ("int4", "down"), ("nvfp4", "o"),
+                                      ("nvfp4", "gate_up")])
+def test_dequant_full_shapes_sampled_rows(fmt, name):
+    K, N = SHAPES[name]
+    seed = SEEDS[name] if fmt == "int4" else 6
+    t = torch()
+    p = synth.device_problem(fmt, seed, 1, N, K)
+    pw, ps = W.pack_on_device(fmt, N, K, p["codes"], p["scales"])
+    out = W.dequant(fmt, N, K, pw, ps, global_scale=gscale_tensor(p["g"]))
+    rows = np.unique(np.concatenate([[0, 15, 16, N - 1], np.random.default_rng(1).integers(0, N, 60)]))
+    got = bf16_bits(out[t.from_numpy(rows).cuda()])
+    ph = synth.problem(fmt, seed, 1, N, K, rows=rows)
+    assert np.array_equal(got, oracle_weights(ph))
+
+
+# ---------------------------------------------------------------- GEMM parity, full oracle
+
+
+CASES = [  # fmt, M, N, K, seed
+    ("int4", 1, 256, 512, 0),          # the tiny configuration
+    ("int4", 1, 272, 640, 40),         # 17 bands, ragged against every CTA split
+    ("int4", 3, 1000, 1024, 41),       # N not a multiple of 16
+    ("int4", 8, 520, 2048, 42),
+    ("int4", 9, 304, 1152, 43),
+    ("int4", 16, 160, 3072, 44),
+    ("int4", 1, 1, 128, 45),           # one output column, one group
+    ("int4", 2, 24, 17408, 46),        # long K: several splits
+    ("nvfp4", 1, 272, 640, 50),
+    ("nvfp4", 5, 1000, 1024, 51),
+    ("nvfp4", 9, 304, 1152, 52),
+    ("nvfp4", 16, 64, 4096, 53),
+    ("nvfp4", 1, 1, 128, 54),
+]
+
+
+@pytest.mark.parametrize("fmt,M,N,K,seed", CASES)
+def test_gemm_parity_small(fmt, M, N, K, seed):
+    p = synth.problem(fmt, seed, M, N, K)
+    codes, scales, x = to_device_problem(p)
+    y, _ = run_gemm(fmt, codes, scales, x, N, g=p["g"])
+    assert_parity(y, p["x"], oracle_weights(p), f"{fmt} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("path", [W.PATH_GEMV])
+@pytest.mark.parametrize("M", [1, 2, 4, 7, 8, 9, 15, 16, 17, 24, 32, 33, 48, 64])
+def test_gemm_parity_every_row_count(path, M):
+    fmt, N, K = "int4", 400, 1536
+    p = synth.problem(fmt, 100 + M, M, N, K)
+    codes, scales, x = to_device_problem(p)
+    y, _ = run_gemm(fmt, codes, scales, x, N, path=path)
+    assert_parity(y, p["x"], oracle_weights(p), f"path {path} M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 8, 9, 33, 64])
+def test_gemm_parity_every_row_count_nvfp4(M):
+    fmt, N, K = "nvfp4", 208, 1280
+    p = synth.problem(fmt, 200 + M, M, N, K)
+    codes, scales, x = to_device_problem(p)
+    y, _ = run_gemm(fmt, codes, scales, x, N, g=p["g"])
+    assert_parity(y, p["x"], oracle_weights(p), f"nvfp4 M={M}")
+
+
+# ---------------------------------------------------------------- GEMM parity at the full shapes
+
+
+FULL = ([("int4", name, 1, SEEDS[name]) for name in SHAPES] +
+        [("int4", name, M, 5) for name in ("qkv", "o", "gate_up", "down") for M in (2, 4, 9, 16, 64)] +
+        [("nvfp4", name, M, 6) for name in ("qkv", "o", "gate_up", "down") for M in (1, 9, 64)])
+
+
+@pytest.mark.parametrize("fmt,name,M,seed", FULL)
+def test_gemm_parity_full_shapes_sampled(fmt, name, M, seed):
+    K, N = SHAPES[name]
+    t = torch()
+    p = synth.device_problem(fmt, seed, M, N, K)
+    y, _ = run_gemm(fmt, p["codes"], p["scales"], p["x"], N, g=p["g"])
+    rows = np.unique(np.concatenate([[0, 7, 8, 15, 16, N - 16, N - 1],
+                                     np.random.default_rng(seed + M).integers(0, N, 48)]))
+    ph = synth.problem(fmt, seed, M, N, K, rows=rows)
+    assert np.array_equal(ph["x"].view(np.int16), p["x"].cpu().numpy())
+    assert_parity(y[:, rows], ph["x"], oracle_weights(ph), f"{fmt} {name} M={M}")
+    del p
+    t.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- invariants and edge cases
+
+
+def _packed(fmt, p):
+    codes, scales, x = to_device_problem(p)
+    pw, ps = W.pack_on_device(fmt, p["N"], p["K"], codes, scales)
+    return pw, ps, x
+
+
+def test_one_hot_selects_dequantised_column_bit_exact():
+    t = torch()
+    for fmt in ("int4", "nvfp4"):
+        N, K = 96, 640
+        p = synth.problem(fmt, 61, 1, N, K)
+        pw, ps, _ = _packed(fmt, p)
+        g = gscale_tensor(p["g"])
+        wd = bf16_bits(W.dequant(fmt, N, K, pw, ps, global_scale=g))
+        for k in (0, 5, 127, 128, 333, K - 1):
+            x = t.zeros((1, K), dtype=t.bfloat16, device="cuda")
+            x[0, k] = 1.0
+            y = W.gemm(fmt, x, pw, ps, N, global_scale=g)
+            t.cuda.synchronize()
+            assert np.array_equal(bf16_bits(y)[0], wd[:, k]), (fmt, k)
+
+
+def test_doubling_x_doubles_y_bit_exact_and_zero_scales_give_zero():
+    t = torch()
+    for fmt in ("int4", "nvfp4"):
+        for M in (1, 9, 64):
+            N, K = 128, 1024
+            p = synth.problem(fmt, 62 + M, M, N, K)
+            pw, ps, x = _packed(fmt, p)
+            g = gscale_tensor(p["g"])
+            xb = x.view(t.bfloat16)
+            y1 = bf16_bits(W.gemm(fmt, xb, pw, ps, N, global_scale=g))
+            y2 = bf16_bits(W.gemm(fmt, xb * 2, pw, ps, N, global_scale=g))
+            v1 = formats.bf16_to_f64(y1)
+            assert np.array_equal(formats.bf16_to_f64(y2), 2 * v1), (fmt, M)
+            zs = t.zeros_like(t.from_numpy(np.ascontiguousarray(
+                p["scales"].view(np.int16) if p["scales"].dtype == np.uint16 else p["scales"])).cuda())
+            codes, _, _ = to_device_problem(p)
+            pw0, ps0 = W.pack_on_device(fmt, N, K, codes, zs)
+            y0 = W.gemm(fmt, xb, pw0, ps0, N, global_scale=g).float().cpu().numpy()
+            assert np.all(y0 == 0), (fmt, M)
+
+
+def test_output_guard_bands_and_full_coverage():
+    t = torch()
+    for fmt, M, N, K in (("int4", 3, 50, 640), ("int4", 8, 24, 17408), ("nvfp4", 9, 40, 512),
+                         ("int4", 64, 33, 384)):
+        p = synth.problem(fmt, 70 + M, M, N, K)
+        pw, ps, x = _packed(fmt, p)
+        pad = 64
+        buf = t.full((M * N + 2 * pad,), float("nan"), dtype=t.bfloat16, device="cuda")
+        sentinel = t.tensor(12345.0, dtype=t.bfloat16)
+        buf[:pad] = sentinel
+        buf[-pad:] = sentinel
+        y = buf[pad:pad + M * N].view(M, N)
+        W.gemm(fmt, x.view(t.bfloat16), pw, ps, N, global_scale=gscale_tensor(p["g"]), y=y)
+        t.cuda.synchronize()
+        host = buf.float().cpu().numpy()
+        assert np.all(host[:pad] == 12352.0) and np.all(host[-pad:] == 12352.0), (fmt, M, N, K)
+        assert not np.any(np.isnan(host[pad:-pad])), (fmt, M, N, K)
+
+
+def test_repeated_calls_are_bit_identical():
+    t = torch()
+    for fmt, M, N, K in (("int4", 8, 5120, 17408), ("int4", 1, 17408, 5120), ("nvfp4", 9, 1024, 6144)):
+        p = synth.device_problem(fmt, 80, M, N, K)
+        pw, ps = W.pack_on_device(fmt, N, K, p["codes"], p["scales"])
+        g = gscale_tensor(p["g"])
+        xb = p["x"].view(t.bfloat16)
+        ys = [bf16_bits(W.gemm(fmt, xb, pw, ps, N, global_scale=g)) for _ in range(3)]
+        assert all(np.array_equal(ys[0], yy) for yy in ys[1:]), (fmt, M, N, K)
+
+
+def test_golden_examples_on_gpu():
+    t = torch()
+    d = json.load(open(os.path.join(GOLDEN, "int4_worked_example.json")))
+    k = np.arange(128)
+    q = np.stack([(k % 16) - 8, 7 - (k % 16)]).astype(np.int8)
+    s = np.array(d["inputs"]["scale_bits"], dtype=np.uint16)
+    pw, ps = W.pack_on_device("int4", 2, 128, t.from_numpy(q).cuda(),
+                              t.from_numpy(s.view(np.int16).copy()).cuda())
+    wd = bf16_bits(W.dequant("int4", 2, 128, pw, ps))
+    assert [int(v) for v in wd[0, :16]] == [int(h, 16) for h in d["expected"]["w_row0_hex_k0_to_15"]]
+    x = t.zeros((1, 128), dtype=t.bfloat16, device="cuda")
+    x[0, :16] = 1.0
+    y = W.gemm("int4", x, pw, ps, 2).float().cpu().numpy()[0]
+    assert list(y) == d["expected"]["y"]
+    d = json.load(open(os.path.join(GOLDEN, "nvfp4_worked_example.json")))
+    c = np.tile(np.arange(16, dtype=np.uint8), (2, 8))
+    s8 = np.repeat(np.array(d["inputs"]["scale_e4m3"], dtype=np.uint8), 8, axis=1)
+    pw, ps = W.pack_on_device("nvfp4", 2, 128, t.from_numpy(c).cuda(), t.from_numpy(s8).cuda())
+    g = gscale_tensor(1.0)
+    wd = bf16_bits(W.dequant("nvfp4", 2, 128, pw, ps, global_scale=g))
+    assert [int(v) for v in wd[0, :16]] == [int(h, 16) for h in d["expected"]["w_row0_hex_k0_to_15"]]
+    x = t.zeros((1, 128), dtype=t.bfloat16, device="cuda")
+    x[0, :8] = 1.0
+    y = W.gemm("nvfp4", x, pw, ps, 2, global_scale=g).float().cpu().numpy()[0]
+    assert list(y) == d["expected"]["y"]
+
+
+def test_device_status_is_clean():
+    assert W.w4a16_device_status() == W.OK

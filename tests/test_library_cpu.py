@@ -1,0 +1,161 @@
+"""The C-ABI library without a GPU: symbols, host packer, argument checks."""
+
+from __future__ import annotations
+
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from bit_weight_only_dequant_b200 import w4a16 as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "w4a16.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a16_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = W.lib()
+    names = _declared_functions()
+    assert "w4a16_gemm" in names and "w4a16_dequant" in names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert W.w4a16_version() >= 100
+
+
+def test_status_strings():
+    for st in (W.OK, W.ERR_ARG, W.ERR_SHAPE, W.ERR_ALIGN, W.ERR_DEVICE, W.ERR_CUDA,
+               W.ERR_TIMEOUT, W.ERR_NOMEM):
+        assert W.status_string(st).startswith("W4A16_")
+
+
+def test_packed_sizes():
+    assert W.w4a16_packed_weight_bytes(0, 8192, 5120) == 8192 * 5120 // 2
+    assert W.w4a16_packed_scale_bytes(0, 8192, 5120) == 8192 * 40 * 2
+    assert W.w4a16_packed_scale_bytes(1, 8192, 5120) == 8192 * 320
+    assert W.w4a16_packed_weight_bytes(0, 17, 128) == 32 * 64          # rows padded to 16
+    assert W.w4a16_packed_weight_bytes(0, 16, 100) == 0                 # K not a multiple of 128
+    assert W.w4a16_packed_weight_bytes(2, 16, 128) == 0                 # bad format
+
+
+@pytest.mark.parametrize("fmt,N,K", [("int4", 16, 128), ("int4", 37, 384), ("nvfp4", 16, 128),
+                                     ("nvfp4", 45, 256)])
+def test_host_pack_round_trip(fmt, N, K):
+    p = synth.problem(fmt, 7, 1, N, K)
+    f = W.FMTS[fmt]
+    w = np.zeros(W.w4a16_packed_weight_bytes(f, N, K), np.uint8)
+    s = np.zeros(W.w4a16_packed_scale_bytes(f, N, K), np.uint8)
+    assert W.w4a16_pack_host(f, N, K, p["codes"], p["scales"], w, s) == W.OK
+    codes = np.zeros_like(p["codes"])
+    scales = np.zeros_like(p["scales"])
+    assert W.w4a16_unpack_host(f, N, K, w, s, codes, scales) == W.OK
+    assert np.array_equal(codes, p["codes"])
+    assert np.array_equal(scales, p["scales"])
+
+
+def _layout_position(fmt, n, k, K):
+    """The packed position of (n, k) restated from the layout description."""
+    nt, kb = n // 16, k // 64
+    r, kk = n % 16, k % 64
+    g, hi = r % 8, r // 8
+    j, kin = kk // 16, kk % 16
+    t, e = kin // 4, kin % 4
+    pair = hi + 2 * (e // 2)
+    second = e % 2
+    nib = pair + 4 * second if fmt == 0 else 2 * pair + second
+    word = (nt * (K // 64) + kb) * 512 + (4 * g + t) * 16 + 4 * j
+    return word + nib // 2, 4 * (nib % 2)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_host_pack_matches_the_documented_layout(fmt):
+    N, K = 32, 256
+    codes = np.zeros((N, K), dtype=np.int8 if fmt == 0 else np.uint8)
+    rng = np.random.default_rng(3)
+    picks = [(int(rng.integers(N)), int(rng.integers(K))) for _ in range(40)]
+    for n, k in picks:
+        codes[n, k] = 5 if fmt == 0 else 11
+    scales = np.zeros((N, K // (128 if fmt == 0 else 16)), dtype=np.uint16 if fmt == 0 else np.uint8)
+    w = np.zeros(W.w4a16_packed_weight_bytes(fmt, N, K), np.uint8)
+    s = np.zeros(W.w4a16_packed_scale_bytes(fmt, N, K), np.uint8)
+    assert W.w4a16_pack_host(fmt, N, K, codes, scales, w, s) == W.OK
+    zero = 8 if fmt == 0 else 0                  # the stored nibble of value 0
+    expect = np.zeros_like(w)
+    for n in range(N):
+        for k in range(K):
+            b, sh = _layout_position(fmt, n, k, K)
+            v = (int(codes[n, k]) + 8) & 15 if fmt == 0 else int(codes[n, k])
+            expect[b] |= v << sh
+    assert np.array_equal(w, expect)
+    assert zero in (0, 8)
+
+
+def test_host_pack_scale_layout():
+    N, K = 32, 256
+    q = np.zeros((N, K), np.int8)
+    sc = (np.arange(N * 2, dtype=np.uint16) + 0x3F00).reshape(N, 2)
+    w = np.zeros(W.w4a16_packed_weight_bytes(0, N, K), np.uint8)
+    s = np.zeros(W.w4a16_packed_scale_bytes(0, N, K), np.uint8)
+    assert W.w4a16_pack_host(0, N, K, q, sc, w, s) == W.OK
+    s16 = s.view(np.uint16)
+    for n in range(N):
+        for gi in range(2):
+            off = ((n // 16) * 2 + gi) * 32 + (n % 8) * 4 + (n % 16 // 8) * 2
+            assert s16[off // 2] == sc[n, gi]
+    c = np.zeros((N, K), np.uint8)
+    s8 = (np.arange(N * 16) % 0x70).astype(np.uint8).reshape(N, 16)
+    w = np.zeros(W.w4a16_packed_weight_bytes(1, N, K), np.uint8)
+    s = np.zeros(W.w4a16_packed_scale_bytes(1, N, K), np.uint8)
+    assert W.w4a16_pack_host(1, N, K, c, s8, w, s) == W.OK
+    for n in range(N):
+        for gi in range(16):
+            off = ((n // 16) * 4 + gi // 4) * 64 + (n % 8) * 8 + (gi % 4) * 2 + (n % 16) // 8
+            assert s[off] == s8[n, gi]
+
+
+def test_host_pack_rejects_out_of_range():
+    N, K = 16, 128
+    w = np.zeros(W.w4a16_packed_weight_bytes(0, N, K), np.uint8)
+    s = np.zeros(W.w4a16_packed_scale_bytes(0, N, K), np.uint8)
+    q = np.zeros((N, K), np.int8)
+    q[3, 5] = 8
+    assert W.w4a16_pack_host(0, N, K, q, np.zeros((N, 1), np.uint16), w, s) == W.ERR_ARG
+    nanscale = np.full((N, 1), 0x7FC0, np.uint16)
+    assert W.w4a16_pack_host(0, N, K, np.zeros((N, K), np.int8), nanscale, w, s) == W.ERR_ARG
+    w = np.zeros(W.w4a16_packed_weight_bytes(1, N, K), np.uint8)
+    s = np.zeros(W.w4a16_packed_scale_bytes(1, N, K), np.uint8)
+    c = np.zeros((N, K), np.uint8)
+    c[0, 0] = 16
+    assert W.w4a16_pack_host(1, N, K, c, np.zeros((N, 8), np.uint8), w, s) == W.ERR_ARG
+    assert W.w4a16_pack_host(1, N, K, np.zeros((N, K), np.uint8), np.full((N, 8), 0x7F, np.uint8),
+                             w, s) == W.ERR_ARG
+
+
+def test_argument_validation_before_any_device_call():
+    x = w = s = y = 1 << 20          # fake, aligned, never dereferenced
+    assert W.w4a16_gemm(0, 0, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE       # M = 0
+    assert W.w4a16_gemm(0, 65, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE      # M > 64
+    assert W.w4a16_gemm(0, 1, 16, 100, x, w, s, None, y, 0) == W.ERR_SHAPE       # K % 128
+    assert W.w4a16_gemm(0, 1, 0, 128, x, w, s, None, y, 0) == W.ERR_SHAPE        # N = 0
+    assert W.w4a16_gemm(3, 1, 16, 128, x, w, s, None, y, 0) == W.ERR_ARG         # format
+    assert W.w4a16_gemm(0, 1, 16, 128, None, w, s, None, y, 0) == W.ERR_ARG      # null x
+    assert W.w4a16_gemm(0, 1, 16, 128, x, w, s, 1 << 21, y, 0) == W.ERR_ARG      # g for int4
+    assert W.w4a16_gemm(1, 1, 16, 128, x, w, s, None, y, 0) == W.ERR_ARG         # no g for nvfp4
+    assert W.w4a16_gemm(0, 1, 16, 128, x + 2, w, s, None, y, 0) == W.ERR_ALIGN
+    assert W.w4a16_gemm_ex(7, 0, 1, 16, 128, x, w, s, None, y, 0) == W.ERR_ARG   # bad path
+    assert W.w4a16_dequant(0, 16, 128, w, s, None, y + 8, 0) == W.ERR_ALIGN
+    assert W.w4a16_pack(0, 16, 100, x, s, w, s, 0) == W.ERR_SHAPE
+
+
+def test_dispatcher_path_table():
+    for M in range(1, 65):
+        path = W.w4a16_gemm_path(0, M, 5120, 5120)
+        assert path in (W.PATH_GEMV, W.PATH_TC)
+    assert W.w4a16_gemm_path(0, 1, 17408, 5120) == W.PATH_GEMV
+    assert W.w4a16_gemm_path(0, 65, 5120, 5120) == W.ERR_SHAPE
