@@ -32,13 +32,23 @@ namespace w4 {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kStages = 3;
-constexpr int kStageKB = 8;                                  // k64 blocks per stage
+#ifndef W4_GEMV_WARPS
+#define W4_GEMV_WARPS 8
+#endif
+#ifndef W4_GEMV_STAGES
+#define W4_GEMV_STAGES 3
+#endif
+#ifndef W4_GEMV_STAGE_KB
+#define W4_GEMV_STAGE_KB 8
+#endif
+constexpr int kWarps = W4_GEMV_WARPS;
+constexpr int kStages = W4_GEMV_STAGES;
+constexpr int kStageKB = W4_GEMV_STAGE_KB;                   // k64 blocks per stage
 constexpr int kStageWBytes = kStageKB * kTileBytes;         // 4096
 constexpr int kStageSBytes = kStageKB * 64;                  // scales, room for NVFP4
 constexpr int kStageBytes = kStageWBytes + kStageSBytes;    // 4608
-constexpr int kHeaderBytes = 1024;                           // mbarriers + row multipliers
+constexpr int kBarBytes = (kWarps * kStages * 8 + 127) / 128 * 128;
+constexpr int kHeaderBytes = kBarBytes + 512;                // mbarriers + 2 x 64 row words
 constexpr int kMaxSmem = 232448;                             // 227 KB opt-in
 
 struct Params {
@@ -68,7 +78,7 @@ __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t*
   const int chunks_per_row = k_len / 8;  // 8 elements per 16-byte load
   if (FMT == 1) {
     // per-row largest magnitude over the slice
-    if (tid < 16) row_max_bits[tid] = 0u;
+    if (tid < 64) row_max_bits[tid] = 0u;
     __syncthreads();
     for (int m = 0; m < p.M; ++m) {
       float mx = 0.f;
@@ -128,8 +138,8 @@ template <int FMT, int MT>
 __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                 // kWarps * kStages
-  float* row_mul = reinterpret_cast<float*>(smem + 512);              // 16
-  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + 640);        // 16
+  float* row_mul = reinterpret_cast<float*>(smem + kBarBytes);        // W4A16_MAX_M
+  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kBarBytes + 256);
   uint8_t* ring = smem + kHeaderBytes;
   uint8_t* xs = ring + kWarps * kStages * kStageBytes;
 
