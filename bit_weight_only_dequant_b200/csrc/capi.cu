@@ -18,9 +18,10 @@ struct DeviceState {
 };
 
 struct Workspace {
-  void* base = nullptr;   // [counters (uint32)] [partials (fp32)]
+  void* base = nullptr;   // [counters (uint32)] [partials (fp32)] [scratch bytes]
   size_t counters = 0;
   size_t floats = 0;
+  size_t bytes = 0;
 };
 
 std::mutex g_mu;
@@ -48,30 +49,36 @@ int device_state(DeviceState** out) {
   return W4A16_OK;
 }
 
-// Workspace of at least (counters, floats) for the current device and `st`.
-// Grows by reallocation in stream order; counters start (and are left) zero.
-int workspace(cudaStream_t st, size_t counters, size_t floats, unsigned** cnt, float** part) {
+// Workspace of at least (counters, floats, bytes) for the current device and
+// `st`.  Grows by reallocation in stream order; counters start (and are left) zero.
+int workspace(cudaStream_t st, size_t counters, size_t floats, size_t bytes, unsigned** cnt,
+              float** part, void** scratch) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   Workspace& w = g_ws[std::make_pair(dev, st)];
-  if (w.base == nullptr || w.counters < counters || w.floats < floats) {
+  if (w.base == nullptr || w.counters < counters || w.floats < floats || w.bytes < bytes) {
     size_t nc = counters > w.counters ? counters : w.counters;
     size_t nf = floats > w.floats ? floats : w.floats;
+    size_t nb = bytes > w.bytes ? bytes : w.bytes;
     if (nc < 65536) nc = 65536;
     if (nf < (1u << 20)) nf = 1u << 20;
     nc = (nc + 63) / 64 * 64;
+    nf = (nf + 63) / 64 * 64;
+    nb = (nb + 255) / 256 * 256;
     void* base = nullptr;
-    if (cudaMallocAsync(&base, nc * sizeof(unsigned) + nf * sizeof(float), st) != cudaSuccess)
+    if (cudaMallocAsync(&base, nc * sizeof(unsigned) + nf * sizeof(float) + nb, st) != cudaSuccess)
       return W4A16_ERR_NOMEM;
     if (cudaMemsetAsync(base, 0, nc * sizeof(unsigned), st) != cudaSuccess) return W4A16_ERR_CUDA;
     if (w.base) cudaFreeAsync(w.base, st);
     w.base = base;
     w.counters = nc;
     w.floats = nf;
+    w.bytes = nb;
   }
   *cnt = static_cast<unsigned*>(w.base);
   *part = reinterpret_cast<float*>(static_cast<unsigned*>(w.base) + w.counters);
+  *scratch = reinterpret_cast<uint8_t*>(*part + w.floats);
   return W4A16_OK;
 }
 
@@ -85,12 +92,13 @@ int check_fmt_shape(int fmt, int N, int K) {
   return W4A16_OK;
 }
 
+// Row-count dispatch: the weight-streaming GEMV while the activations are a
+// thin n8 operand, the tcgen05 path once the tensor cores carry real work.
 int choose_path(int fmt, int M, int N, int K) {
   (void)fmt;
   (void)N;
   (void)K;
-  if (M <= 16) return W4A16_PATH_GEMV;
-  return W4A16_PATH_GEMV;
+  return M <= 8 ? W4A16_PATH_GEMV : W4A16_PATH_TC;
 }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA; }
@@ -175,7 +183,7 @@ int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16, co
       !aligned16(y_bf16))
     return W4A16_ERR_ALIGN;
   if (path == W4A16_PATH_AUTO) path = choose_path(fmt, M, N, K);
-  if (path == W4A16_PATH_TC) return W4A16_ERR_SHAPE;  // not available in this build
+  if (path == W4A16_PATH_GEMV && M > W4A16_GEMV_MAX_M) return W4A16_ERR_SHAPE;
   DeviceState* d = nullptr;
   if ((r = device_state(&d)) != W4A16_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -193,12 +201,24 @@ int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16, co
   a.ws = nullptr;
   a.counters = nullptr;
   a.err = d->err;
-  const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, d->num_sms);
-  const size_t nf = w4::gemv_workspace_floats(pl, M, N);
-  if (nf > 0) {
-    if ((r = workspace(st, w4::gemv_counters(pl, N), nf, &a.counters, &a.ws)) != W4A16_OK) return r;
+  void* scratch = nullptr;
+  if (path == W4A16_PATH_GEMV) {
+    const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, d->num_sms);
+    const size_t nf = w4::gemv_workspace_floats(pl, M, N);
+    if (nf > 0) {
+      r = workspace(st, w4::gemv_counters(pl, N), nf, 0, &a.counters, &a.ws, &scratch);
+      if (r != W4A16_OK) return r;
+    }
+    return status_of(w4::launch_gemv(pl, a, st));
   }
-  return status_of(w4::launch_gemv(pl, a, st));
+  const w4::TcPlan pl = w4::plan_tc(fmt, M, N, K, d->num_sms);
+  const size_t nf = w4::tc_workspace_floats(pl, M, N);
+  const size_t nb = w4::tc_x_f16_bytes(fmt, M, K);
+  if (nf > 0 || nb > 0) {
+    r = workspace(st, w4::tc_counters(pl, N), nf, nb, &a.counters, &a.ws, &scratch);
+    if (r != W4A16_OK) return r;
+  }
+  return status_of(w4::launch_tc(pl, a, scratch, st));
 }
 
 int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,

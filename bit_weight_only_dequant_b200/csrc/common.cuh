@@ -15,9 +15,17 @@ namespace w4 {
 // w4a16_device_status().
 constexpr unsigned kErrTimeout = 1u;
 
-// Iteration bound of every spin on an mbarrier: about a second of polling,
-// far above the longest legitimate wait (a few microseconds).
-constexpr uint32_t kSpinLimit = 1u << 26;
+// Bounds of every spin on an mbarrier: about two seconds of wall time (read
+// from %globaltimer every 256 polls) or 2^30 polls, far above the longest
+// legitimate wait (microseconds).
+constexpr uint32_t kSpinLimit = 1u << 30;
+constexpr uint64_t kSpinNanos = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -55,11 +63,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   return ok != 0;
 }
 
-// Bounded wait: returns false (and records the timeout) if the phase never
-// completes within kSpinLimit polls.
+// Bounded wait: returns false (and records the timeout) if the phase does not
+// complete within the bounds above.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigned* err) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, phase)) return true;
+    if ((i & 255u) == 0u && global_ns() - t0 > kSpinNanos) break;
   }
   atomicOr(err, kErrTimeout);
   return false;

@@ -1,30 +1,32 @@
-// Split-K weight-streaming GEMV for decode row counts on sm_100a.
+// Split-K weight-streaming GEMV for decode row counts (M <= 16) on sm_100a.
 //
-// Why this shape: at M <= 16 the matmul moves ~0.5 byte of packed weight per
+// Why this shape: at small M the matmul moves ~0.5 byte of packed weight per
 // 2*M flops, so the time is the time to stream the weights from HBM once (the
 // bandwidth argument of the blog post "One Config Line Made My 27B Model 2.7x
 // Faster", section "Gotcha #2").  The kernel's job is to keep enough bytes in
-// flight and to spend as few instructions per weight as possible on turning
-// nibbles into multiply operands: B200 issues ~2 lane-instructions per weight
-// at full HBM speed.
+// flight and to spend as few instructions per weight as possible turning
+// nibbles into multiply operands: at 7+ TB/s a B200 SM has about two
+// lane-instructions per weight.
 //
-// Structure (one CTA per SM, 8 worker warps, no producer warp):
-//  * Each CTA owns one K-slice [k_lo, k_hi) and a contiguous range of 16-row
-//    bands.  It first copies its slice of the activations into shared memory
-//    (k reordered inside every 16-block to match the operand fragments of the
-//    packed layout); NVFP4 rows are rescaled by a power of two into FP16.
-//  * Each warp streams its bands' packed weights and scales through a private
-//    3-stage ring of 4.5 KB stages filled by 1-D bulk copies (TMA) completing
-//    on mbarriers, so ~64-96 KB per SM are in flight.
+// Structure (one CTA of 16 warps per SM, no producer warp):
+//  * A CTA owns one K-slice and a contiguous range of 16-row bands.  Its
+//    warps form a (Wn x Wk) grid: Wn bands in flight at a time, each band's
+//    slice cut into Wk equal group-aligned pieces, one per warp, so every warp
+//    streams the same number of bytes.  The Wk partial sums of a band are
+//    added in piece order through shared memory (deterministic).
+//  * The CTA first copies its slice of the activations into shared memory,
+//    k reordered inside every 16-block to match the packed operand fragments
+//    (NVFP4: rows rescaled by a power of two into FP16).
+//  * Each warp streams its pieces through a private 2-stage ring of 4.5 KB
+//    stages filled by 1-D bulk copies (TMA) completing on mbarriers.
 //  * Per 32-bit word (8 weights) a lane builds the A fragment of one
-//    mma.sync m16n8k16 (rows = 16 output columns, k = 16) with 3 shifts,
-//    4 LOP3 and 4 BF16 subtractions (int4), or 4 hardware e2m1 -> f16
-//    conversions (NVFP4); the activations are the n8 side, so every MMA
-//    serves M <= 8 rows at once.  Group scales are applied to the fp32 MMA
-//    results (per 128-group for int4, per 16-group for NVFP4).
-//  * Split-K partials go to a fp32 workspace; the last warp to finish a band
-//    (arrival counter) adds the S partials in split order and writes BF16, so
-//    the result does not depend on arrival order.
+//    mma.sync m16n8k16 (16 output columns x 16 k): 3 shifts, 4 LOP3 and
+//    4 exact BF16 subtractions (int4), or 4 hardware e2m1 -> f16 conversions
+//    (NVFP4).  The activations are the n8 side: one MMA serves 8 rows.
+//    Group scales multiply the fp32 MMA results (int4: once per 128-group,
+//    NVFP4: once per 16-group).
+//  * Split-K partials across CTAs go to a fp32 workspace; the last CTA to
+//    finish a band (arrival counter) adds them in split order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,24 +34,30 @@ namespace w4 {
 
 namespace {
 
-#ifndef W4_GEMV_WARPS
-#define W4_GEMV_WARPS 8
-#endif
 #ifndef W4_GEMV_STAGES
-#define W4_GEMV_STAGES 3
+#define W4_GEMV_STAGES 2
 #endif
 #ifndef W4_GEMV_STAGE_KB
 #define W4_GEMV_STAGE_KB 8
 #endif
-constexpr int kWarps = W4_GEMV_WARPS;
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
 constexpr int kStages = W4_GEMV_STAGES;
-constexpr int kStageKB = W4_GEMV_STAGE_KB;                   // k64 blocks per stage
-constexpr int kStageWBytes = kStageKB * kTileBytes;         // 4096
-constexpr int kStageSBytes = kStageKB * 64;                  // scales, room for NVFP4
-constexpr int kStageBytes = kStageWBytes + kStageSBytes;    // 4608
+constexpr int kStageKB = W4_GEMV_STAGE_KB;                   // k64 blocks per stage (even)
+constexpr int kStageWBytes = kStageKB * kTileBytes;
+constexpr int kStageSBytes = kStageKB * 64;                  // room for NVFP4 scales
+constexpr int kStageBytes = kStageWBytes + kStageSBytes;
+constexpr int kMaxMT = 2;                                    // M <= 16
 constexpr int kBarBytes = (kWarps * kStages * 8 + 127) / 128 * 128;
-constexpr int kHeaderBytes = kBarBytes + 512;                // mbarriers + 2 x 64 row words
+constexpr int kRowWords = 64;                                // per-row words (M <= 64)
+constexpr int kZeroOff = kBarBytes + 2 * kRowWords * 4;      // 128 zero bytes
+constexpr int kRedOff = kZeroOff + 128;
+constexpr int kRedBytes = kWarps * 32 * 4 * kMaxMT * 4;      // per-lane partial sums
+constexpr int kHeaderBytes = kRedOff + kRedBytes;
+constexpr int kRingBytes = kWarps * kStages * kStageBytes;
 constexpr int kMaxSmem = 232448;                             // 227 KB opt-in
+static_assert(kStageKB % 2 == 0, "stages hold whole 128-groups");
+static_assert(kHeaderBytes % 128 == 0, "ring alignment");
 
 struct Params {
   const __nv_bfloat16* x;
@@ -61,11 +69,11 @@ struct Params {
   unsigned* counters;
   unsigned* err;
   int M, N, K, NT, S, kslice, ctas_x, row_stride;  // row_stride in bytes
+  int wn, wk;                                      // warp grid: bands x pieces
 };
 
-// Element k of a 64-block (local index kin) sits at this element offset of
-// the block's 64-element image in shared memory: lane t = (kin % 16) / 4
-// reads elements [16 t, 16 t + 16) as k = 16 j + 4 t + e, e = 0..3, j = 0..3.
+// Element kin of a 64-block sits at this element offset of the block's image
+// in shared memory: lane t reads 16 contiguous elements k = 16 j + 4 t + e.
 __device__ __forceinline__ int perm64(int kin) {
   const int j = kin >> 4, t = (kin >> 2) & 3, e = kin & 3;
   return t * 16 + j * 4 + e;
@@ -73,19 +81,18 @@ __device__ __forceinline__ int perm64(int kin) {
 
 template <int FMT>
 __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t* xs,
-                                  float* row_mul, unsigned* row_max_bits) {
+                                  float* row_mul, unsigned* row_aux) {
   const int tid = threadIdx.x;
   const int chunks_per_row = k_len / 8;  // 8 elements per 16-byte load
   if (FMT == 1) {
-    // per-row largest magnitude over the slice
-    if (tid < 64) row_max_bits[tid] = 0u;
+    if (tid < kRowWords) row_aux[tid] = 0u;
     __syncthreads();
     for (int m = 0; m < p.M; ++m) {
       float mx = 0.f;
       const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + k_lo);
       for (int c = tid; c < chunks_per_row; c += blockDim.x) {
-        uint4 v = src[c];
-        const uint32_t* u = reinterpret_cast<const uint32_t*>(&v);
+        const uint4 v = src[c];
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           mx = fmaxf(mx, fabsf(__uint_as_float(u[i] << 16)));
@@ -94,39 +101,34 @@ __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t*
       }
 #pragma unroll
       for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if ((tid & 31) == 0) atomicMax(row_max_bits + m, __float_as_uint(mx));
+      if ((tid & 31) == 0) atomicMax(row_aux + m, __float_as_uint(mx));
     }
     __syncthreads();
     if (tid < p.M) {
-      const float mx = __uint_as_float(row_max_bits[tid]);
+      const float mx = __uint_as_float(row_aux[tid]);
       int e = 0;
       if (mx > 0.f && isfinite(mx)) e = ilogbf(mx) - 14;  // max * 2^-e in [2^14, 2^15)
       row_mul[tid] = ldexpf(1.f, e);
-      row_max_bits[tid] = static_cast<unsigned>(-e);       // reused: exponent to apply
+      row_aux[tid] = static_cast<unsigned>(-e);           // exponent applied to the row
     }
     __syncthreads();
   }
   for (int idx = tid; idx < p.M * chunks_per_row; idx += blockDim.x) {
     const int m = idx / chunks_per_row, c = idx - m * chunks_per_row;
     const uint4 v = reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + k_lo)[c];
-    const int kin0 = c * 8;              // slice-local k of the first element
+    const int kin0 = c * 8;
     const int blk = kin0 >> 6, in = kin0 & 63;
-    uint32_t out[4];
-    const uint32_t* u = reinterpret_cast<const uint32_t*>(&v);
-    if (FMT == 0) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) out[i] = u[i];
-    } else {
-      const int sh = static_cast<int>(row_max_bits[m]);
+    uint32_t out[4] = {v.x, v.y, v.z, v.w};
+    if (FMT == 1) {
+      const int sh = static_cast<int>(row_aux[m]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float lo = ldexpf(__uint_as_float(u[i] << 16), sh);
-        const float hi = ldexpf(__uint_as_float(u[i] & 0xFFFF0000u), sh);
+        const float lo = ldexpf(__uint_as_float(out[i] << 16), sh);
+        const float hi = ldexpf(__uint_as_float(out[i] & 0xFFFF0000u), sh);
         __half2 h = __floats2half2_rn(lo, hi);
         out[i] = *reinterpret_cast<uint32_t*>(&h);
       }
     }
-    // elements in..in+3 and in+4..in+7 each land on 4 contiguous slots
     uint8_t* row = xs + (size_t)m * p.row_stride + blk * 128;
     *reinterpret_cast<uint2*>(row + perm64(in) * 2) = make_uint2(out[0], out[1]);
     *reinterpret_cast<uint2*>(row + perm64(in + 4) * 2) = make_uint2(out[2], out[3]);
@@ -134,44 +136,200 @@ __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t*
   __syncthreads();
 }
 
+// c = A . B (fresh accumulator), fp32
+__device__ __forceinline__ void mma_bf16_first(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+__device__ __forceinline__ void mma_f16_first(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+// One 128-group (two 64-blocks) of one band: int4.
+template <int MT>
+__device__ __forceinline__ void group_int4(const uint8_t* sw, const uint8_t* ss, int lane, int g,
+                                           const uint8_t* const* xrow, const int* xstep, int kbl,
+                                           float (*acc)[4]) {
+  const uint4 w0 = *reinterpret_cast<const uint4*>(sw + lane * 16);
+  const uint4 w1 = *reinterpret_cast<const uint4*>(sw + kTileBytes + lane * 16);
+  const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  uint32_t a[8][4];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    a[j][0] = int4_pair_to_bf16x2(wd[j]);
+    a[j][1] = int4_pair_to_bf16x2(wd[j] >> 4);
+    a[j][2] = int4_pair_to_bf16x2(wd[j] >> 8);
+    a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
+  }
+  const uint32_t sp = *reinterpret_cast<const uint32_t*>(ss + g * 4);
+  const float s_lo = __uint_as_float(sp << 16);          // row g
+  const float s_hi = __uint_as_float(sp & 0xFFFF0000u);  // row g + 8
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const uint4* xb0 = reinterpret_cast<const uint4*>(xrow[mt] + kbl * xstep[mt]);
+    const uint4* xb1 = reinterpret_cast<const uint4*>(xrow[mt] + (kbl + 1) * xstep[mt]);
+    const uint4 v0 = xb0[0], v1 = xb0[1], v2 = xb1[0], v3 = xb1[1];
+    const uint32_t bx[16] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w,
+                             v2.x, v2.y, v2.z, v2.w, v3.x, v3.y, v3.z, v3.w};
+    float c[4];
+    mma_bf16_first(c, a[0], bx[0], bx[1]);
+#pragma unroll
+    for (int j = 1; j < 8; ++j) mma_bf16_16816(c, a[j], bx[2 * j], bx[2 * j + 1]);
+    acc[mt][0] = fmaf(s_lo, c[0], acc[mt][0]);
+    acc[mt][1] = fmaf(s_lo, c[1], acc[mt][1]);
+    acc[mt][2] = fmaf(s_hi, c[2], acc[mt][2]);
+    acc[mt][3] = fmaf(s_hi, c[3], acc[mt][3]);
+  }
+}
+
+// One 64-block of one band: NVFP4 (a scale per 16-group, i.e. per MMA).
+template <int MT>
+__device__ __forceinline__ void block_nvfp4(const uint8_t* sw, const uint8_t* ss, int lane, int g,
+                                            const uint8_t* const* xrow, const int* xstep, int kbl,
+                                            float (*acc)[4]) {
+  const uint4 wv = *reinterpret_cast<const uint4*>(sw + lane * 16);
+  const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+  uint32_t a[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    a[j][0] = e2m1x2_to_f16x2(wd[j]);
+    a[j][1] = e2m1x2_to_f16x2(wd[j] >> 8);
+    a[j][2] = e2m1x2_to_f16x2(wd[j] >> 16);
+    a[j][3] = e2m1x2_to_f16x2(wd[j] >> 24);
+  }
+  const uint2 sv = *reinterpret_cast<const uint2*>(ss + g * 8);
+  const uint32_t sw2[2] = {sv.x, sv.y};
+  float2 sf[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t s2 = e4m3x2_to_f16x2(static_cast<uint16_t>(sw2[j >> 1] >> (16 * (j & 1))));
+    sf[j] = __half22float2(*reinterpret_cast<const __half2*>(&s2));
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const uint4* xb = reinterpret_cast<const uint4*>(xrow[mt] + kbl * xstep[mt]);
+    const uint4 v0 = xb[0], v1 = xb[1];
+    const uint32_t bx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float c[4];
+      mma_f16_first(c, a[j], bx[2 * j], bx[2 * j + 1]);
+      acc[mt][0] = fmaf(sf[j].x, c[0], acc[mt][0]);
+      acc[mt][1] = fmaf(sf[j].x, c[1], acc[mt][1]);
+      acc[mt][2] = fmaf(sf[j].y, c[2], acc[mt][2]);
+      acc[mt][3] = fmaf(sf[j].y, c[3], acc[mt][3]);
+    }
+  }
+}
+
 template <int FMT, int MT>
-__global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const Params p) {
+__device__ __forceinline__ void band_epilogue(const Params& p, int band, int split, int lane,
+                                              const float* row_mul, const float (*vals)[4]) {
+  const int g = lane >> 2, t = lane & 3;
+  const float gmul = FMT == 1 ? __ldg(p.g) : 1.f;
+  const int n0 = band * 16 + g;
+  if (p.S == 1) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int m = mt * 8 + 2 * t + (i & 1);
+        const int n = n0 + 8 * (i >> 1);
+        if (m < p.M && n < p.N) {
+          float v = vals[mt][i];
+          if (FMT == 1) v = v * row_mul[m] * gmul;
+          p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v);
+        }
+      }
+    return;
+  }
+  const size_t Npad = (size_t)p.NT * 16;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = mt * 8 + 2 * t + (i & 1);
+      const int n = n0 + 8 * (i >> 1);
+      if (m < p.M) {
+        float v = vals[mt][i];
+        if (FMT == 1) v = v * row_mul[m];
+        __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v);
+      }
+    }
+  __threadfence();
+  __syncwarp();
+  unsigned prev = 0;
+  if (lane == 0) prev = atomicAdd(p.counters + band, 1u);
+  prev = __shfl_sync(0xffffffffu, prev, 0);
+  if (prev != static_cast<unsigned>(p.S - 1)) return;
+  __threadfence();
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = mt * 8 + 2 * t + (i & 1);
+      const int n = n0 + 8 * (i >> 1);
+      if (m < p.M && n < p.N) {
+        float v = 0.f;
+        for (int sp = 0; sp < p.S; ++sp) v += __ldcg(p.ws + ((size_t)sp * p.M + m) * Npad + n);
+        p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v * gmul);
+      }
+    }
+  if (lane == 0) p.counters[band] = 0u;
+}
+
+template <int FMT, int MT>
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                 // kWarps * kStages
-  float* row_mul = reinterpret_cast<float*>(smem + kBarBytes);        // W4A16_MAX_M
-  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kBarBytes + 256);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+  float* row_mul = reinterpret_cast<float*>(smem + kBarBytes);
+  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kBarBytes + kRowWords * 4);
+  const uint8_t* zero = smem + kZeroOff;
+  float* red = reinterpret_cast<float*>(smem + kRedOff);
   uint8_t* ring = smem + kHeaderBytes;
-  uint8_t* xs = ring + kWarps * kStages * kStageBytes;
+  uint8_t* xs = ring + kRingBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int split = blockIdx.y;
   const int k_lo = split * p.kslice;
   const int k_len = min(p.K - k_lo, p.kslice);
-  const int nkb = k_len >> 6;                                          // 64-blocks in the slice
   const int band_lo = (int)(((long long)blockIdx.x * p.NT) / p.ctas_x);
   const int band_hi = (int)(((long long)(blockIdx.x + 1) * p.NT) / p.ctas_x);
+  const int nbands = band_hi - band_lo;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kWarps * kStages; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
   }
+  if (threadIdx.x < 32) reinterpret_cast<uint32_t*>(smem + kZeroOff)[threadIdx.x] = 0u;
   stage_activations<FMT>(p, k_lo, k_len, xs, row_mul, row_aux);  // ends with __syncthreads
 
-  // This warp's bands: band_lo + warp, + kWarps, ...
-  const int my_first = band_lo + warp;
-  const int my_bands = my_first < band_hi ? (band_hi - my_first + kWarps - 1) / kWarps : 0;
-  const int stages_per_band = (nkb + kStageKB - 1) / kStageKB;
-  const int total = my_bands * stages_per_band;
+  // warp grid: wi = band slot, wj = K piece
+  const int wi = warp % p.wn, wj = warp / p.wn;
+  const int groups = k_len >> 7;
+  const int g_lo = wj * groups / p.wk, g_hi = (wj + 1) * groups / p.wk;
+  const int kbl_lo = 2 * g_lo;                 // slice-local first 64-block of the piece
+  const int nkb = 2 * (g_hi - g_lo);           // 64-blocks in the piece
+  const int rounds = (nbands + p.wn - 1) / p.wn;
+  const int my_rounds = wi < nbands ? (nbands - wi + p.wn - 1) / p.wn : 0;
+  const int spb = (nkb + kStageKB - 1) / kStageKB;   // stages per band piece
+  const int total = my_rounds * spb;
   uint64_t* my_bars = bars + warp * kStages;
   uint8_t* my_ring = ring + warp * kStages * kStageBytes;
   const int KB = p.K >> 6;
   const uint64_t pol = policy_evict_first();
 
   auto issue = [&](int L) {
-    const int bi = L / stages_per_band, st = L - bi * stages_per_band;
-    const int band = my_first + bi * kWarps;
-    const int kb0 = (k_lo >> 6) + st * kStageKB;
+    const int r = L / spb, st = L - r * spb;
+    const int band = band_lo + wi + r * p.wn;
+    const int kb0 = (k_lo >> 6) + kbl_lo + st * kStageKB;
     const int nblk = min(kStageKB, nkb - st * kStageKB);
     const int buf = L % kStages;
     uint8_t* dst = my_ring + buf * kStageBytes;
@@ -179,7 +337,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const Params p) {
     uint32_t sbytes;
     const uint8_t* ssrc;
     if (FMT == 0) {
-      sbytes = nblk * 16;  // 32 bytes per 128-group = 2 blocks
+      sbytes = nblk * 16;
       ssrc = p.s + ((size_t)band * (p.K >> 7) + (kb0 >> 1)) * 32;
     } else {
       sbytes = nblk * 64;
@@ -189,181 +347,85 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const Params p) {
     bulk_g2s_evict_first(dst, wsrc, nblk * kTileBytes, my_bars + buf, pol);
     bulk_g2s_evict_first(dst + kStageWBytes, ssrc, sbytes, my_bars + buf, pol);
   };
-
-  if (lane == 0) {
+  if (lane == 0)
     for (int L = 0; L < min(kStages, total); ++L) issue(L);
+
+  // activation rows of this lane (row m = 8 mt + g); rows past M read zeros
+  const uint8_t* xrow[MT];
+  int xstep[MT];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int m = mt * 8 + g;
+    const bool real = m < p.M;
+    xrow[mt] = real ? xs + (size_t)m * p.row_stride + t * 32 : zero;
+    xstep[mt] = real ? 128 : 0;
   }
 
-  float acc[MT][4];
-  float cg[MT][2][4];
   bool failed = false;
   int L = 0;
-  for (int bi = 0; bi < my_bands && !failed; ++bi) {
-    const int band = my_first + bi * kWarps;
+  for (int r = 0; r < rounds; ++r) {
+    float acc[MT][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
-
-    for (int st = 0; st < stages_per_band; ++st, ++L) {
-      const int buf = L % kStages;
-      if (!mbar_wait(my_bars + buf, (L / kStages) & 1, p.err)) {
-        failed = true;
-        break;
-      }
-      const uint8_t* sw = my_ring + buf * kStageBytes;
-      const uint8_t* ss = sw + kStageWBytes;
-      const int nblk = min(kStageKB, nkb - st * kStageKB);
-      for (int bb = 0; bb < nblk; ++bb) {
-        const int kbl = st * kStageKB + bb;  // slice-local 64-block
-        const uint4 wv = *reinterpret_cast<const uint4*>(sw + bb * kTileBytes + lane * 16);
-        const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-        // A fragments of the four k16 sub-blocks (pairs P0..P3 = a0..a3)
-        uint32_t a[4][4];
+    const bool active = r < my_rounds && !failed;
+    if (active) {
+      for (int st = 0; st < spb; ++st, ++L) {
+        const int buf = L % kStages;
+        if (!mbar_wait(my_bars + buf, (L / kStages) & 1, p.err)) {
+          failed = true;
+          break;
+        }
+        const uint8_t* sw = my_ring + buf * kStageBytes;
+        const uint8_t* ss = sw + kStageWBytes;
+        const int nblk = min(kStageKB, nkb - st * kStageKB);
+        const int kbl0 = kbl_lo + st * kStageKB;
         if (FMT == 0) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            a[j][0] = int4_pair_to_bf16x2(wd[j]);
-            a[j][1] = int4_pair_to_bf16x2(wd[j] >> 4);
-            a[j][2] = int4_pair_to_bf16x2(wd[j] >> 8);
-            a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
-          }
+          for (int gi = 0; gi < (nblk >> 1); ++gi)
+            group_int4<MT>(sw + gi * 2 * kTileBytes, ss + gi * 32, lane, g, xrow, xstep,
+                           kbl0 + 2 * gi, acc);
         } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            a[j][0] = e2m1x2_to_f16x2(wd[j]);
-            a[j][1] = e2m1x2_to_f16x2(wd[j] >> 8);
-            a[j][2] = e2m1x2_to_f16x2(wd[j] >> 16);
-            a[j][3] = e2m1x2_to_f16x2(wd[j] >> 24);
-          }
+          for (int bb = 0; bb < nblk; ++bb)
+            block_nvfp4<MT>(sw + bb * kTileBytes, ss + bb * 64, lane, g, xrow, xstep, kbl0 + bb,
+                            acc);
         }
-        const int half = kbl & 1;  // int4: which 64-block of the 128-group
-        float2 sf[4];              // nvfp4: (row g, row g+8) scale of each k16 group
-        if (FMT == 1) {
-          const uint2 sv = *reinterpret_cast<const uint2*>(ss + bb * 64 + g * 8);
-          const uint32_t sw2[2] = {sv.x, sv.y};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t s2 =
-                e4m3x2_to_f16x2(static_cast<uint16_t>(sw2[j >> 1] >> (16 * (j & 1))));
-            sf[j] = __half22float2(*reinterpret_cast<const __half2*>(&s2));
-          }
-        }
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          // activation fragments of row m = 8 mt + g: words (j, pair)
-          uint32_t bx[8];
-          const int m = mt * 8 + g;
-          if (m < p.M) {
-            const uint4* src =
-                reinterpret_cast<const uint4*>(xs + (size_t)m * p.row_stride + kbl * 128 + t * 32);
-            const uint4 v0 = src[0], v1 = src[1];
-            bx[0] = v0.x; bx[1] = v0.y; bx[2] = v0.z; bx[3] = v0.w;
-            bx[4] = v1.x; bx[5] = v1.y; bx[6] = v1.z; bx[7] = v1.w;
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) bx[i] = 0u;
-          }
-          if (FMT == 0) {
-            if (half == 0) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) cg[mt][0][i] = cg[mt][1][i] = 0.f;
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) mma_bf16_16816(cg[mt][half], a[j], bx[2 * j], bx[2 * j + 1]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float c[4] = {0.f, 0.f, 0.f, 0.f};
-              mma_f16_16816(c, a[j], bx[2 * j], bx[2 * j + 1]);
-              acc[mt][0] = fmaf(sf[j].x, c[0], acc[mt][0]);
-              acc[mt][1] = fmaf(sf[j].x, c[1], acc[mt][1]);
-              acc[mt][2] = fmaf(sf[j].y, c[2], acc[mt][2]);
-              acc[mt][3] = fmaf(sf[j].y, c[3], acc[mt][3]);
-            }
-          }
-        }
-        if (FMT == 0 && half == 1) {
-          // fold the group: acc += s_row * (sum over the 128 k of q x)
-          const uint32_t sp = *reinterpret_cast<const uint32_t*>(ss + (bb >> 1) * 32 + g * 4);
-          const float s_lo = __uint_as_float(sp << 16);           // row g
-          const float s_hi = __uint_as_float(sp & 0xFFFF0000u);   // row g + 8
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            acc[mt][0] = fmaf(s_lo, cg[mt][0][0] + cg[mt][1][0], acc[mt][0]);
-            acc[mt][1] = fmaf(s_lo, cg[mt][0][1] + cg[mt][1][1], acc[mt][1]);
-            acc[mt][2] = fmaf(s_hi, cg[mt][0][2] + cg[mt][1][2], acc[mt][2]);
-            acc[mt][3] = fmaf(s_hi, cg[mt][0][3] + cg[mt][1][3], acc[mt][3]);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0 && L + kStages < total) issue(L + kStages);
-    }
-    if (failed) break;
-
-    // ---------------------------------------------------------------- epilogue of a band
-    // lane holds rows n = 16 band + g (+8) and activation rows m = 8 mt + 2t (+1)
-    float gmul = 1.f;
-    if (FMT == 1) gmul = __ldg(p.g);
-    const int n0 = band * 16 + g;
-    if (p.S == 1) {
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = mt * 8 + 2 * t + (i & 1);
-          const int n = n0 + 8 * (i >> 1);
-          if (m < p.M && n < p.N) {
-            float v = acc[mt][i];
-            if (FMT == 1) v = v * row_mul[m] * gmul;
-            p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v);
-          }
-        }
-      }
-    } else {
-      const int Npad = p.NT * 16;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = mt * 8 + 2 * t + (i & 1);
-          const int n = n0 + 8 * (i >> 1);
-          if (m < p.M) {
-            float v = acc[mt][i];
-            if (FMT == 1) v = v * row_mul[m];
-            __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v);
-          }
-        }
-      }
-      __threadfence();
-      __syncwarp();
-      unsigned prev = 0;
-      if (lane == 0) prev = atomicAdd(p.counters + band, 1u);
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev == static_cast<unsigned>(p.S - 1)) {
-        __threadfence();
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int m = mt * 8 + 2 * t + (i & 1);
-            const int n = n0 + 8 * (i >> 1);
-            if (m < p.M && n < p.N) {
-              float v = 0.f;
-              for (int sp = 0; sp < p.S; ++sp) v += __ldcg(p.ws + ((size_t)sp * p.M + m) * Npad + n);
-              p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v * gmul);
-            }
-          }
-        }
-        if (lane == 0) p.counters[band] = 0u;
+        __syncwarp();
+        if (lane == 0 && L + kStages < total) issue(L + kStages);
       }
     }
+    const int band = band_lo + wi + r * p.wn;
+    if (p.wk == 1) {
+      if (active && !failed) band_epilogue<FMT, MT>(p, band, split, lane, row_mul, acc);
+      continue;
+    }
+    // add the wk pieces of each band in piece order
+    float* mine = red + (warp * 32 + lane) * 4 * MT;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mine[mt * 4 + i] = (active && !failed) ? acc[mt][i] : 0.f;
+    __syncthreads();
+    if (wj == 0 && active && !failed) {
+      float sum[MT][4];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum[mt][i] = 0.f;
+      for (int pc = 0; pc < p.wk; ++pc) {
+        const float* o = red + ((pc * p.wn + wi) * 32 + lane) * 4 * MT;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sum[mt][i] += o[mt * 4 + i];
+      }
+      band_epilogue<FMT, MT>(p, band, split, lane, row_mul, sum);
+    }
+    __syncthreads();
   }
 
   if (failed) {
-    // let this warp's outstanding copies (stages L .. L + kStages - 1) land
-    // before the CTA can exit; every wait is bounded again
+    // let this warp's outstanding copies land before the CTA can exit
     for (int LL = L; LL < min(L + kStages, total); ++LL)
       mbar_wait(my_bars + (LL % kStages), (LL / kStages) & 1, p.err);
   }
@@ -388,8 +450,10 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   p.kslice = pl.kslice;
   p.ctas_x = pl.ctas_x;
   p.row_stride = (pl.kslice / 64) * 128 + 16;
-  // raise the kernel's dynamic shared memory limit once (not a stream operation,
-  // but kept out of the steady state so launches can be captured in graphs)
+  p.wn = pl.wn;
+  p.wk = pl.wk;
+  // raise the dynamic shared memory limit once per device (kept out of the
+  // steady state so launches can be captured in CUDA graphs)
   static int smem_set[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -400,46 +464,55 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     smem_set[dev] = kMaxSmem;
   }
-  gemv_kernel<FMT, MT><<<dim3(pl.ctas_x, pl.S), kWarps * 32, pl.smem, st>>>(p);
+  gemv_kernel<FMT, MT><<<dim3(pl.ctas_x, pl.S), kThreads, pl.smem, st>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+// Picks the K splits across CTAs (S) and the warp grid (wn bands x wk pieces)
+// that minimise the largest number of 64-blocks any warp streams, with small
+// penalties for cross-CTA split-K and per-round reductions.
 GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
   (void)fmt;
   GemvPlan pl;
-  pl.mt = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));
+  pl.mt = M <= 8 ? 1 : 2;
   const int NT = (N + 15) / 16;
   const int groups = K / 128;
-  const int ring = kWarps * kStages * kStageBytes;
-  const int xbudget = kMaxSmem - kHeaderBytes - ring;
-  // largest slice (in 128-groups) whose activation image fits
+  const int xbudget = kMaxSmem - kHeaderBytes - kRingBytes;
   const int max_groups = (xbudget / M - 16) / 256;
   const int s_min = (groups + max_groups - 1) / max_groups;
   double best = 1e300;
-  int best_s = s_min;
+  pl.S = s_min;
+  pl.wk = 1;
   for (int S = s_min; S <= groups && S <= 16; ++S) {
     const int gslice = (groups + S - 1) / S;
     if ((S - 1) * gslice >= groups) continue;  // an empty split
     int ctas = num_sms / S;
     if (ctas < 1) ctas = 1;
     if (ctas > NT) ctas = NT;
-    const double bands = static_cast<double>((NT + ctas - 1) / ctas);
-    double cost = bands * gslice * (S > 1 ? 1.03 : 1.0);
-    if (cost < best - 1e-9) {
-      best = cost;
-      best_s = S;
+    const int bands_max = (NT + ctas - 1) / ctas;
+    for (int wk = 1; wk <= kWarps; wk *= 2) {
+      if (wk > gslice) break;
+      const int wn = kWarps / wk;
+      const int rounds = (bands_max + wn - 1) / wn;
+      const int piece = 2 * ((gslice + wk - 1) / wk);
+      double cost = (double)rounds * (piece + (wk > 1 ? 2.0 : 0.5)) + (S > 1 ? 3.0 : 0.0);
+      if (cost < best - 1e-9) {
+        best = cost;
+        pl.S = S;
+        pl.wk = wk;
+      }
     }
   }
-  pl.S = best_s;
+  pl.wn = kWarps / pl.wk;
   const int gslice = (groups + pl.S - 1) / pl.S;
   pl.kslice = gslice * 128;
   int ctas = num_sms / pl.S;
   if (ctas < 1) ctas = 1;
   if (ctas > NT) ctas = NT;
   pl.ctas_x = ctas;
-  pl.smem = kHeaderBytes + ring + M * ((pl.kslice / 64) * 128 + 16);
+  pl.smem = kHeaderBytes + kRingBytes + M * ((pl.kslice / 64) * 128 + 16);
   return pl;
 }
 
@@ -450,20 +523,8 @@ size_t gemv_workspace_floats(const GemvPlan& p, int M, int N) {
 size_t gemv_counters(const GemvPlan& p, int N) { return p.S > 1 ? (N + 15) / 16 : 0; }
 
 cudaError_t launch_gemv(const GemvPlan& p, const GemmArgs& a, cudaStream_t st) {
-  if (a.fmt == 0) {
-    switch (p.mt) {
-      case 1: return launch_t<0, 1>(p, a, st);
-      case 2: return launch_t<0, 2>(p, a, st);
-      case 4: return launch_t<0, 4>(p, a, st);
-      default: return launch_t<0, 8>(p, a, st);
-    }
-  }
-  switch (p.mt) {
-    case 1: return launch_t<1, 1>(p, a, st);
-    case 2: return launch_t<1, 2>(p, a, st);
-    case 4: return launch_t<1, 4>(p, a, st);
-    default: return launch_t<1, 8>(p, a, st);
-  }
+  if (a.fmt == 0) return p.mt == 1 ? launch_t<0, 1>(p, a, st) : launch_t<0, 2>(p, a, st);
+  return p.mt == 1 ? launch_t<1, 1>(p, a, st) : launch_t<1, 2>(p, a, st);
 }
 
 }  // namespace w4

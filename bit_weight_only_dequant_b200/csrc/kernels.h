@@ -26,6 +26,7 @@ struct GemvPlan {
   int kslice;    // K elements per split (multiple of 128)
   int ctas_x;    // CTAs per split
   int mt;        // 8-row activation tiles (1: M <= 8, 2: M <= 16)
+  int wn, wk;    // warps per CTA as (bands in flight) x (K pieces per band)
   int smem;      // dynamic shared memory bytes
 };
 
@@ -34,6 +35,23 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms);
 size_t gemv_workspace_floats(const GemvPlan& p, int M, int N);
 size_t gemv_counters(const GemvPlan& p, int N);
 cudaError_t launch_gemv(const GemvPlan& p, const GemmArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- tensor-core path (tcgen05)
+
+struct TcPlan {
+  int mpad;      // activation rows padded to the MMA N (16, 32, 48, 64)
+  int S;         // K splits
+  int kbs;       // 64-blocks per split
+  int units;     // 256-row tiles x splits
+  int grid;      // persistent CTAs
+  int smem;      // dynamic shared memory bytes
+};
+
+TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms);
+size_t tc_workspace_floats(const TcPlan& p, int M, int N);
+size_t tc_counters(const TcPlan& p, int N);
+size_t tc_x_f16_bytes(int fmt, int M, int K);   // NVFP4: FP16 copy of x + row multipliers
+cudaError_t launch_tc(const TcPlan& p, const GemmArgs& a, void* xf16_scratch, cudaStream_t st);
 
 // ---------------------------------------------------------------- dequant export / packer
 

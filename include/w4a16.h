@@ -71,8 +71,9 @@ extern "C" {
 
 /* Kernel paths (for w4a16_gemm_path / w4a16_gemm_ex). */
 #define W4A16_PATH_AUTO 0      /* row-count dispatch */
-#define W4A16_PATH_GEMV 1      /* CUDA-core/mma.sync split-K GEMV, M <= 16 */
-#define W4A16_PATH_TC 2        /* tcgen05 tensor-core path, 16 <= M <= 64 */
+#define W4A16_PATH_GEMV 1      /* weight-streaming split-K GEMV (mma.sync fragments), M <= 16 */
+#define W4A16_PATH_TC 2        /* tcgen05 tensor-core path (A in tensor memory), M <= 64 */
+#define W4A16_GEMV_MAX_M 16
 
 /*
  * Shape rules: 1 <= M <= 64; N >= 1 (any value; packed buffers are padded to

@@ -141,8 +141,11 @@ def test_gemm_parity_small(fmt, M, N, K, seed):
     assert_parity(y, p["x"], oracle_weights(p), f"{fmt} M={M} N={N} K={K}")
 
 
-@pytest.mark.parametrize("path", [W.PATH_GEMV])
-@pytest.mark.parametrize("M", [1, 2, 4, 7, 8, 9, 15, 16, 17, 24, 32, 33, 48, 64])
+ROW_COUNTS = [(W.PATH_GEMV, M) for M in (1, 2, 3, 4, 5, 7, 8, 9, 12, 15, 16)] + \
+             [(W.PATH_TC, M) for M in (1, 2, 8, 9, 15, 16, 17, 24, 31, 32, 33, 48, 63, 64)]
+
+
+@pytest.mark.parametrize("path,M", ROW_COUNTS)
 def test_gemm_parity_every_row_count(path, M):
     fmt, N, K = "int4", 400, 1536
     p = synth.problem(fmt, 100 + M, M, N, K)
@@ -151,12 +154,14 @@ def test_gemm_parity_every_row_count(path, M):
     assert_parity(y, p["x"], oracle_weights(p), f"path {path} M={M}")
 
 
-@pytest.mark.parametrize("M", [1, 8, 9, 33, 64])
-def test_gemm_parity_every_row_count_nvfp4(M):
+@pytest.mark.parametrize("path,M", [(W.PATH_GEMV, 1), (W.PATH_GEMV, 8), (W.PATH_GEMV, 9),
+                                    (W.PATH_GEMV, 16), (W.PATH_TC, 1), (W.PATH_TC, 9),
+                                    (W.PATH_TC, 33), (W.PATH_TC, 64)])
+def test_gemm_parity_every_row_count_nvfp4(path, M):
     fmt, N, K = "nvfp4", 208, 1280
     p = synth.problem(fmt, 200 + M, M, N, K)
     codes, scales, x = to_device_problem(p)
-    y, _ = run_gemm(fmt, codes, scales, x, N, g=p["g"])
+    y, _ = run_gemm(fmt, codes, scales, x, N, g=p["g"], path=path)
     assert_parity(y, p["x"], oracle_weights(p), f"nvfp4 M={M}")
 
 
@@ -205,7 +210,12 @@ def test_one_hot_selects_dequantised_column_bit_exact():
             x[0, k] = 1.0
             y = W.gemm(fmt, x, pw, ps, N, global_scale=g)
             t.cuda.synchronize()
-            assert np.array_equal(bf16_bits(y)[0], wd[:, k]), (fmt, k)
+            # y = 1 * W_deq[n][k] + (+0) * the rest: the same value, and the same
+            # bits except that a -0 weight sums to +0
+            assert np.array_equal(formats.bf16_to_f64(bf16_bits(y)[0]),
+                                  formats.bf16_to_f64(wd[:, k])), (fmt, k)
+            nz = (wd[:, k] & 0x7FFF) != 0
+            assert np.array_equal(bf16_bits(y)[0][nz], wd[nz, k]), (fmt, k)
 
 
 def test_doubling_x_doubles_y_bit_exact_and_zero_scales_give_zero():
