@@ -554,6 +554,27 @@ def run_native(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_case(spec: str, launches: int):
+    """Launch one GEMM a few times (for profilers): spec = fmt,M,N,K[,path]."""
+    import torch
+    from bit_weight_only_dequant_b200 import w4a16 as W
+    parts = spec.split(",")
+    fmt, M, N, K = parts[0], int(parts[1]), int(parts[2]), int(parts[3])
+    path = int(parts[4]) if len(parts) > 4 else W.PATH_AUTO
+    torch.cuda.set_device(0)
+    f = W.FMTS[fmt]
+    (pw, ps), = make_weights(fmt, 3, N, K, 1)
+    x = make_x(fmt, 3, M, K)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
+    for _ in range(launches):
+        W.check(W.w4a16_gemm_ex(path, f, M, N, K, x, pw, ps, g, y), "gemm")
+    torch.cuda.synchronize()
+    W.check(W.w4a16_device_status(), "device status")
+    print(json.dumps({"case": spec, "launches": launches, "path": W.w4a16_gemm_path(f, M, N, K)
+                      if path == W.PATH_AUTO else path}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -564,7 +585,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-stack", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="profiling mode: launch one GEMM fmt,M,N,K[,path] --launches times")
+    ap.add_argument("--launches", type=int, default=5)
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case, args.launches)
+        return
     if args.warmup < 3:
         args.warmup = 3
     rank = int(os.environ.get("RANK", "0"))
