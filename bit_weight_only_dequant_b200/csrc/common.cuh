@@ -15,17 +15,11 @@ namespace w4 {
 // w4a16_device_status().
 constexpr unsigned kErrTimeout = 1u;
 
-// Bounds of every spin on an mbarrier: about two seconds of wall time (read
-// from %globaltimer every 256 polls) or 2^30 polls, far above the longest
-// legitimate wait (microseconds).
-constexpr uint32_t kSpinLimit = 1u << 30;
-constexpr uint64_t kSpinNanos = 2000000000ull;
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+// Bounds of every spin on an mbarrier: 2^31 polls or about two seconds of
+// SM clock (checked every 1024 polls with clock64, which is cheap), far
+// above the longest legitimate wait (microseconds).
+constexpr uint32_t kSpinLimit = 1u << 31;
+constexpr long long kSpinCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -67,10 +61,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
 // complete within the bounds above.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigned* err) {
   if (mbar_try_wait(bar, phase)) return true;
-  const uint64_t t0 = global_ns();
+  const long long t0 = clock64();
   for (uint32_t i = 1; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, phase)) return true;
-    if ((i & 255u) == 0u && global_ns() - t0 > kSpinNanos) break;
+    if ((i & 1023u) == 0u && clock64() - t0 > kSpinCycles) break;
   }
   atomicOr(err, kErrTimeout);
   return false;
@@ -123,6 +117,22 @@ __device__ __forceinline__ uint32_t int4_pair_to_bf16x2(uint32_t w) {
   uint32_t d;
   const uint32_t bias = 0x43084308u;  // BF16 136.0, twice
   asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(bias));
+  return d;
+}
+
+// FP16 forms of the same conversion.  0x6400 is FP16 1024.0 with a mantissa
+// LSB of 1 and ten mantissa bits, so a nibble at bits 0..3 gives 1024 + u and
+// a nibble at bits 4..7 gives 1024 + 16 u; exact arithmetic then leaves q.
+__device__ __forceinline__ uint32_t int4_lo_pair_to_f16x2(uint32_t w) {
+  const uint32_t v = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(0x64086408u));  // - 1032
+  return d;
+}
+__device__ __forceinline__ uint32_t int4_hi_pair_to_f16x2(uint32_t w) {
+  const uint32_t v = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(v), "r"(0x2C002C00u), "r"(0xD480D480u));  // /16 - 72
   return d;
 }
 

@@ -40,6 +40,15 @@ namespace {
 #ifndef W4_GEMV_STAGE_KB
 #define W4_GEMV_STAGE_KB 8
 #endif
+#ifndef W4_GEMV_INT4_F16
+#define W4_GEMV_INT4_F16 0
+#endif
+// Activations go to the tensor cores as FP16 (rescaled per row slice) for
+// NVFP4 always, and for int4 when W4_GEMV_INT4_F16 is set.
+template <int FMT>
+struct XF16 {
+  static constexpr bool value = FMT == 1 || W4_GEMV_INT4_F16 != 0;
+};
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = W4_GEMV_STAGES;
@@ -84,7 +93,7 @@ __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t*
                                   float* row_mul, unsigned* row_aux) {
   const int tid = threadIdx.x;
   const int chunks_per_row = k_len / 8;  // 8 elements per 16-byte load
-  if (FMT == 1) {
+  if (XF16<FMT>::value) {
     if (tid < kRowWords) row_aux[tid] = 0u;
     __syncthreads();
     for (int m = 0; m < p.M; ++m) {
@@ -119,7 +128,7 @@ __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t*
     const int kin0 = c * 8;
     const int blk = kin0 >> 6, in = kin0 & 63;
     uint32_t out[4] = {v.x, v.y, v.z, v.w};
-    if (FMT == 1) {
+    if (XF16<FMT>::value) {
       const int sh = static_cast<int>(row_aux[m]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -162,10 +171,19 @@ __device__ __forceinline__ void group_int4(const uint8_t* sw, const uint8_t* ss,
   uint32_t a[8][4];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    a[j][0] = int4_pair_to_bf16x2(wd[j]);
-    a[j][1] = int4_pair_to_bf16x2(wd[j] >> 4);
-    a[j][2] = int4_pair_to_bf16x2(wd[j] >> 8);
-    a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
+    if (W4_GEMV_INT4_F16) {
+      // FP16 holds two nibbles per 16-bit half in its mantissa: one shift per word
+      const uint32_t hi = wd[j] >> 8;
+      a[j][0] = int4_lo_pair_to_f16x2(wd[j]);
+      a[j][1] = int4_hi_pair_to_f16x2(wd[j]);
+      a[j][2] = int4_lo_pair_to_f16x2(hi);
+      a[j][3] = int4_hi_pair_to_f16x2(hi);
+    } else {
+      a[j][0] = int4_pair_to_bf16x2(wd[j]);
+      a[j][1] = int4_pair_to_bf16x2(wd[j] >> 4);
+      a[j][2] = int4_pair_to_bf16x2(wd[j] >> 8);
+      a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
+    }
   }
   const uint32_t sp = *reinterpret_cast<const uint32_t*>(ss + g * 4);
   const float s_lo = __uint_as_float(sp << 16);          // row g
@@ -178,9 +196,15 @@ __device__ __forceinline__ void group_int4(const uint8_t* sw, const uint8_t* ss,
     const uint32_t bx[16] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w,
                              v2.x, v2.y, v2.z, v2.w, v3.x, v3.y, v3.z, v3.w};
     float c[4];
-    mma_bf16_first(c, a[0], bx[0], bx[1]);
+    if (W4_GEMV_INT4_F16) {
+      mma_f16_first(c, a[0], bx[0], bx[1]);
 #pragma unroll
-    for (int j = 1; j < 8; ++j) mma_bf16_16816(c, a[j], bx[2 * j], bx[2 * j + 1]);
+      for (int j = 1; j < 8; ++j) mma_f16_16816(c, a[j], bx[2 * j], bx[2 * j + 1]);
+    } else {
+      mma_bf16_first(c, a[0], bx[0], bx[1]);
+#pragma unroll
+      for (int j = 1; j < 8; ++j) mma_bf16_16816(c, a[j], bx[2 * j], bx[2 * j + 1]);
+    }
     acc[mt][0] = fmaf(s_lo, c[0], acc[mt][0]);
     acc[mt][1] = fmaf(s_lo, c[1], acc[mt][1]);
     acc[mt][2] = fmaf(s_hi, c[2], acc[mt][2]);
@@ -243,7 +267,7 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
         const int n = n0 + 8 * (i >> 1);
         if (m < p.M && n < p.N) {
           float v = vals[mt][i];
-          if (FMT == 1) v = v * row_mul[m] * gmul;
+          if (XF16<FMT>::value) v = v * row_mul[m] * gmul;
           p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v);
         }
       }
@@ -258,7 +282,7 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
       const int n = n0 + 8 * (i >> 1);
       if (m < p.M) {
         float v = vals[mt][i];
-        if (FMT == 1) v = v * row_mul[m];
+        if (XF16<FMT>::value) v = v * row_mul[m];
         __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v);
       }
     }

@@ -6,23 +6,25 @@
 // a bandwidth-bound step into a slightly compute-bound one: blog post "One
 // Config Line Made My 27B Model 2.7x Faster", section "The fix").
 //
-// Structure (one persistent CTA per SM, 10 warps, 256-row x M tiles):
-//  * warp 8 (producer): per 64-k block, one 2-D TMA load of the activation
-//    tile (M rows, SWIZZLE_128B, rows past M zero-filled) and 1-D bulk copies
-//    of the 16 packed 512-byte weight tiles and their scales into a 6-stage
-//    shared-memory ring.
-//  * warps 0-7 (dequant, then epilogue): each lane turns its 16 packed bytes
-//    into 32 scaled operands in registers (int4: q -> BF16, times the BF16
-//    group scale with one rounding, i.e. exactly W_deq; NVFP4: e2m1 -> FP16
-//    times the E4M3 scale, exact) and writes them straight into tensor memory
-//    with tcgen05.st 16x256b, whose register layout matches the packed pairs.
-//    Shared memory never holds dequantised weights.
-//  * warp 9 (MMA): tcgen05.mma kind::f16 with A (weights, 128 rows) read from
-//    tensor memory and B (activations, K-major SW128) from shared memory,
-//    accumulating fp32 D (128 lanes x Mpad columns) per 128-row half.
+// Structure (one persistent CTA per SM, 18 warps, 256-row x M tiles):
+//  * warp 16 (producer): per stage of four 64-k blocks, lane b < 16 copies
+//    band b's 2 KB of packed weights and its scales with 1-D bulk copies, and
+//    lanes 16..19 load the four SWIZZLE_128B activation boxes with 2-D TMA
+//    (rows past M zero-filled) into a 3-4 stage shared-memory ring.
+//  * warps 0-15 (dequant, then epilogue): one 16-row band each; every lane
+//    turns its 16 packed bytes per block into 32 scaled operands in registers
+//    (int4: q -> BF16 times the BF16 group scale with one rounding, exactly
+//    W_deq; NVFP4: e2m1 -> FP16 times the E4M3 scale, exact) and writes them
+//    straight into a tensor-memory A slot with tcgen05.st 16x256b, whose
+//    register layout matches the packed pairs.  Shared memory never holds
+//    dequantised weights.
+//  * warp 17 (MMA): tcgen05.mma kind::f16, A (weights, 128 rows) from tensor
+//    memory, B (activations, K-major SW128) from shared memory, fp32 D
+//    (128 lanes x Mpad columns) per 128-row half; issued by one elected lane
+//    of a converged warp.
 //  * epilogue: tcgen05.ld of D, BF16 stores (or fp32 split-K partials reduced
 //    in split order by the last CTA of the tile).
-// Tensor memory: D at columns [0, 128), six A stages of 2 x 32 columns at
+// Tensor memory: D at columns [0, 128), six A slots of 2 x 32 columns at
 // [128, 512).  Every mbarrier wait is bounded; a timeout raises the device
 // error word, the CTA drains its copies and MMAs and frees tensor memory.
 #include <cuda.h>
@@ -35,17 +37,20 @@ namespace w4 {
 
 namespace {
 
-constexpr int kTcStages = 6;
-constexpr int kDeqWarps = 8;
+constexpr int kDeqWarps = 16;                 // one 16-row band per warp
 constexpr int kTcThreads = (kDeqWarps + 2) * 32;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kTcTileRows = 256;  // 16 bands, two 128-row MMA tiles
-constexpr int kWStage = 16 * kTileBytes;       // 8192
-constexpr int kSStage = 16 * 64;               // scales (NVFP4 size; INT4 uses 32 per band)
+constexpr int kProducerWarp = kDeqWarps;
+constexpr int kMmaWarp = kDeqWarps + 1;
+constexpr int kTcTileRows = 256;              // 16 bands, two 128-row MMA tiles
+constexpr int kKS = 4;                        // 64-blocks per shared-memory stage
+constexpr int kMaxStages = 4;
+constexpr int kWStage = 16 * kKS * kTileBytes;  // 32 KB: 2 KB contiguous per band
+constexpr int kSStage = 16 * kKS * 64;          // scales (NVFP4 size; INT4 uses 32 per group)
+constexpr int kSmemBudget = 220 * 1024;
+constexpr int kASlots = 6;                    // tensor-memory A slots of one 64-block each
 constexpr int kTmemCols = 512;
 constexpr int kAColBase = 128;
-constexpr int kMinSmem = 120 * 1024;           // keeps one CTA (and one TMEM owner) per SM
+constexpr int kMinSmem = 120 * 1024;          // keeps one CTA (and one TMEM owner) per SM
 
 struct TcParams {
   const uint8_t* w;
@@ -82,18 +87,16 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, float* v) {
-  uint32_t r[16];
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, float* v) {
+  uint32_t r[8];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
+        "=r"(r[7])
       : "r"(taddr)
       : "memory");
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -148,12 +151,12 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t phase, volatile int* abort_flag,
                                         unsigned* err) {
   if (mbar_try_wait(bar, phase)) return true;
-  const uint64_t t0 = global_ns();
+  const long long t0 = clock64();
   for (uint32_t i = 1; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, phase)) return true;
-    if ((i & 255u) == 0u) {
+    if ((i & 1023u) == 0u) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kSpinNanos) break;
+      if (clock64() - t0 > kSpinCycles) break;
     }
   }
   *abort_flag = 1;
@@ -181,21 +184,51 @@ __device__ __forceinline__ uint32_t hmul2_f16(uint32_t a, uint32_t b) {
 
 // ------------------------------------------------------------------ the kernel
 
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// Warp-wide bounded wait: lane 0 polls, the warp then proceeds together.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t phase, volatile int* abort_flag,
+                                          unsigned* err) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = tc_wait(bar, phase, abort_flag, err) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+template <int FMT, int MPAD>
+struct TcShape {
+  static constexpr int kBBlock = MPAD * 128;                 // one 64-k activation box
+  static constexpr int kBStage = kKS * kBBlock;
+  static constexpr int kStageBytes = kBStage + kWStage + kSStage;
+  static constexpr int kStages = (kSmemBudget / kStageBytes) < kMaxStages
+                                     ? (kSmemBudget / kStageBytes) : kMaxStages;
+  static constexpr int kSmem = kStages * kStageBytes + 1024 /* barriers */ + 1024 /* align */;
+};
+
 template <int FMT, int MPAD>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap xmap, const TcParams p) {
+  using Sh = TcShape<FMT, MPAD>;
+  constexpr int NS = Sh::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  constexpr int kBStage = MPAD * 128;
-  uint8_t* Bs = smem;
-  uint8_t* Ws = Bs + kTcStages * kBStage;
-  uint8_t* Ss = Ws + kTcStages * kWStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Ss + kTcStages * kSStage);
-  uint64_t* full = bars;
-  uint64_t* afull = bars + kTcStages;
-  uint64_t* freeb = bars + 2 * kTcStages;
-  uint64_t* dfull = bars + 3 * kTcStages;
+  uint8_t* Bs = smem;                                   // NS x kKS x (MPAD x 128 B), SW128
+  uint8_t* Ws = Bs + NS * Sh::kBStage;                  // NS x 16 bands x kKS x 512 B
+  uint8_t* Ss = Ws + NS * kWStage;                      // NS x 16 bands x 256 B
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Ss + NS * kSStage);
+  uint64_t* full = bars;                                // NS
+  uint64_t* sfree = bars + NS;                          // NS
+  uint64_t* afull = bars + 2 * NS;                      // kASlots
+  uint64_t* afree = afull + kASlots;                    // kASlots
+  uint64_t* dfull = afree + kASlots;
   uint64_t* dfree = dfull + 1;
   uint64_t* drain = dfull + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -205,10 +238,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kTcStages; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(full + i, 1);
+      mbar_init(sfree + i, kDeqWarps + 1);
+    }
+    for (int i = 0; i < kASlots; ++i) {
       mbar_init(afull + i, kDeqWarps);
-      mbar_init(freeb + i, kDeqWarps + 1);
+      mbar_init(afree + i, 1);
     }
     mbar_init(dfull, 1);
     mbar_init(dfree, kDeqWarps);
@@ -226,175 +262,203 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const uint32_t sbytes_blk = FMT == 0 ? 16u : 64u;     // scale bytes per band per 64-block
 
   if (warp == kProducerWarp) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      int last_use[kTcStages];
-      for (int i = 0; i < kTcStages; ++i) last_use[i] = -1;
-      uint32_t it = 0;
-      bool ok = true;
-      for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
-        const int tile = unit / p.S, split = unit - tile * p.S;
-        const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
-        const int nb0 = tile * 16;
-        const int nvalid = min(16, p.NT - nb0);
-        for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
-          const int s = it % kTcStages;
-          const uint32_t u = it / kTcStages;
-          if (u > 0 && !tc_wait(freeb + s, (u - 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          const uint32_t sb = FMT == 0 ? 32u : 64u;
-          mbar_arrive_expect_tx(full + s, kBStage + nvalid * (kTileBytes + sb));
-          tma_load_2d(Bs + s * kBStage, &xmap, kb * 64, 0, full + s);
-          for (int b = 0; b < nvalid; ++b) {
-            const size_t nb = (size_t)(nb0 + b);
-            bulk_g2s(Ws + s * kWStage + b * kTileBytes, p.w + (nb * p.KB + kb) * kTileBytes,
-                     kTileBytes, full + s);
-            const uint8_t* ssrc = FMT == 0 ? p.s + (nb * (p.K >> 7) + (kb >> 1)) * 32
-                                           : p.s + (nb * p.KB + kb) * 64;
-            bulk_g2s(Ss + s * kSStage + b * sb, ssrc, sb, full + s);
-          }
-          last_use[s] = (int)u;
+    // ---------------------------------------------------------------- producer (whole warp)
+    int last_use[kMaxStages];
+#pragma unroll
+    for (int i = 0; i < kMaxStages; ++i) last_use[i] = -1;
+    uint32_t st_it = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
+      const int tile = unit / p.S, split = unit - tile * p.S;
+      const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
+      const int nb0 = tile * 16;
+      const int nvalid = min(16, p.NT - nb0);
+      for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += kKS, ++st_it) {
+        const int s = st_it % NS;
+        const uint32_t u = st_it / NS;
+        const int nblk = min(kKS, kb_hi - kb0);
+        if (u > 0 && !warp_wait(sfree + s, (u - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
         }
+        if (lane == 0)
+          mbar_arrive_expect_tx(full + s, nblk * Sh::kBBlock +
+                                              nvalid * nblk * (kTileBytes + sbytes_blk));
+        __syncwarp();
+        if (lane < nvalid) {
+          const size_t nb = (size_t)(nb0 + lane);
+          bulk_g2s(Ws + s * kWStage + lane * (kKS * kTileBytes), p.w + (nb * p.KB + kb0) * kTileBytes,
+                   nblk * kTileBytes, full + s);
+          const uint8_t* ssrc = FMT == 0 ? p.s + (nb * (p.K >> 7) + (kb0 >> 1)) * 32
+                                         : p.s + (nb * p.KB + kb0) * 64;
+          bulk_g2s(Ss + s * kSStage + lane * (kKS * 64), ssrc, nblk * sbytes_blk, full + s);
+        } else if (lane >= 16 && lane < 16 + nblk) {
+          const int j = lane - 16;
+          tma_load_2d(Bs + s * Sh::kBStage + j * Sh::kBBlock, &xmap, (kb0 + j) * 64, 0, full + s);
+        }
+        last_use[s] = (int)u;
       }
-      // drain: every issued copy has landed before the CTA may exit
-      for (int s = 0; s < kTcStages; ++s)
-        if (last_use[s] >= 0) mbar_wait(full + s, last_use[s] & 1, p.err);
     }
+    // drain: every issued copy has landed before the CTA may exit
+    if (lane == 0)
+      for (int s = 0; s < NS; ++s)
+        if (last_use[s] >= 0) mbar_wait(full + s, last_use[s] & 1, p.err);
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc(FMT == 0 ? 1 : 0, MPAD);
-      uint32_t it = 0, unit_i = 0;
-      bool ok = true;
-      for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
-        const int tile = unit / p.S, split = unit - tile * p.S;
-        const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
-        (void)tile;
-        if (unit_i > 0) {
-          if (!tc_wait(dfree, (unit_i - 1) & 1, abort_flag, p.err)) break;
-          tc_fence_after();
+    // ---------------------------------------------------------------- MMA issuer (whole warp)
+    constexpr uint32_t idesc = make_idesc(FMT == 0 ? 1 : 0, MPAD);
+    uint32_t st_it = 0, ab = 0, unit_i = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
+      const int tile = unit / p.S, split = unit - tile * p.S;
+      const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
+      (void)tile;
+      if (unit_i > 0) {
+        if (!warp_wait(dfree, (unit_i - 1) & 1, abort_flag, p.err)) break;
+        tc_fence_after();
+      }
+      for (int kb0 = kb_lo; kb0 < kb_hi && ok; kb0 += kKS, ++st_it) {
+        const int s = st_it % NS;
+        const uint32_t u = st_it / NS;
+        const int nblk = min(kKS, kb_hi - kb0);
+        if (!warp_wait(full + s, u & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
         }
-        for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
-          const int s = it % kTcStages;
-          const uint32_t u = it / kTcStages;
-          if (!tc_wait(afull + s, u & 1, abort_flag, p.err) ||
-              !tc_wait(full + s, u & 1, abort_flag, p.err)) {
+        const uint64_t dbase = sw128_desc(smem_u32(Bs + s * Sh::kBStage));
+        for (int j = 0; j < nblk; ++j, ++ab) {
+          const int slot = ab % kASlots;
+          if (!warp_wait(afull + slot, (ab / kASlots) & 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t bbase = smem_u32(Bs + s * kBStage);
+          const uint64_t bj = dbase + (uint64_t)((j * Sh::kBBlock) >> 4);
+          const uint32_t a0 = tmem + kAColBase + slot * 64;
+          if (elect_one()) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t a = tmem + kAColBase + s * 64 + h * 32 + j * 8;
-              umma_ts(tmem + h * 64, a, sw128_desc(bbase + j * 32), idesc,
-                      (kb > kb_lo || j > 0) ? 1u : 0u);
-            }
+              for (int k = 0; k < 4; ++k)
+                umma_ts(tmem + h * 64, a0 + h * 32 + k * 8, bj + (uint64_t)(k * 2), idesc,
+                        (kb0 + j > kb_lo || k > 0) ? 1u : 0u);
+            umma_commit(afree + slot);
           }
-          umma_commit(freeb + s);
+          __syncwarp();
         }
-        if (ok) umma_commit(dfull);
+        if (!ok) break;
+        if (elect_one()) umma_commit(sfree + s);
+        __syncwarp();
       }
-      // drain: all issued MMAs complete before tensor memory is released
+      if (ok) {
+        if (elect_one()) umma_commit(dfull);
+        __syncwarp();
+      }
+    }
+    // drain: all issued MMAs complete before tensor memory is released
+    if (elect_one()) {
       umma_commit(drain);
       mbar_wait(drain, 0, p.err);
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- dequant + epilogue
-    const int h = warp >> 2, q = warp & 3;
+    const int q = warp & 3, h = (warp >> 2) & 1, bp = warp >> 3;
+    const int band = h * 8 + 2 * q + bp;                // 16-row band of the 256-row tile
     const int g = lane >> 2;
-    uint32_t it = 0, unit_i = 0;
+    const uint32_t lane_base = (uint32_t)(32 * q + 16 * bp) << 16;
+    uint32_t st_it = 0, ab = 0, unit_i = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
       const int tile = unit / p.S, split = unit - tile * p.S;
       const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
-      for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
-        const int s = it % kTcStages;
-        const uint32_t u = it / kTcStages;
-        if (!tc_wait(full + s, u & 1, abort_flag, p.err) ||
-            (u > 0 && !tc_wait(freeb + s, (u - 1) & 1, abort_flag, p.err))) {
+      for (int kb0 = kb_lo; kb0 < kb_hi && ok; kb0 += kKS, ++st_it) {
+        const int s = st_it % NS;
+        const uint32_t u = st_it / NS;
+        const int nblk = min(kKS, kb_hi - kb0);
+        if (!warp_wait(full + s, u & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        uint32_t r[2][16];
-#pragma unroll
-        for (int bp = 0; bp < 2; ++bp) {
-          const int band = h * 8 + 2 * q + bp;
-          const uint4 wv =
-              *reinterpret_cast<const uint4*>(Ws + s * kWStage + band * kTileBytes + lane * 16);
+        const uint8_t* wsrc = Ws + s * kWStage + band * (kKS * kTileBytes) + lane * 16;
+        const uint8_t* ssrc = Ss + s * kSStage + band * (kKS * 64);
+        for (int j = 0; j < nblk; ++j, ++ab) {
+          const int slot = ab % kASlots;
+          const uint32_t ua = ab / kASlots;
+          if (ua > 0 && !warp_wait(afree + slot, (ua - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint4 wv = *reinterpret_cast<const uint4*>(wsrc + j * kTileBytes);
           const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+          uint32_t r[16];
           if (FMT == 0) {
-            const uint32_t sp = *reinterpret_cast<const uint32_t*>(Ss + s * kSStage + band * 32 + g * 4);
+            const uint32_t sp = *reinterpret_cast<const uint32_t*>(ssrc + (j >> 1) * 32 + g * 4);
             const uint32_t s_lo = prmt(sp, sp, 0x1010u);  // (s_g, s_g)
             const uint32_t s_hi = prmt(sp, sp, 0x3232u);  // (s_g8, s_g8)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int k = 0; k < 4; ++k) {
               // register order of 16x256b: (row g, col 2t), (row g, col 2t+1),
               // (row g+8, col 2t), (row g+8, col 2t+1) = P0, P2, P1, P3
-              r[bp][4 * j + 0] = hmul2_bf16(int4_pair_to_bf16x2(wd[j]), s_lo);
-              r[bp][4 * j + 1] = hmul2_bf16(int4_pair_to_bf16x2(wd[j] >> 8), s_lo);
-              r[bp][4 * j + 2] = hmul2_bf16(int4_pair_to_bf16x2(wd[j] >> 4), s_hi);
-              r[bp][4 * j + 3] = hmul2_bf16(int4_pair_to_bf16x2(wd[j] >> 12), s_hi);
+              r[4 * k + 0] = hmul2_bf16(int4_pair_to_bf16x2(wd[k]), s_lo);
+              r[4 * k + 1] = hmul2_bf16(int4_pair_to_bf16x2(wd[k] >> 8), s_lo);
+              r[4 * k + 2] = hmul2_bf16(int4_pair_to_bf16x2(wd[k] >> 4), s_hi);
+              r[4 * k + 3] = hmul2_bf16(int4_pair_to_bf16x2(wd[k] >> 12), s_hi);
             }
           } else {
-            const uint2 sv = *reinterpret_cast<const uint2*>(Ss + s * kSStage + band * 64 + g * 8);
+            const uint2 sv = *reinterpret_cast<const uint2*>(ssrc + j * 64 + g * 8);
             const uint32_t sw2[2] = {sv.x, sv.y};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int k = 0; k < 4; ++k) {
               const uint32_t s2 =
-                  e4m3x2_to_f16x2(static_cast<uint16_t>(sw2[j >> 1] >> (16 * (j & 1))));
+                  e4m3x2_to_f16x2(static_cast<uint16_t>(sw2[k >> 1] >> (16 * (k & 1))));
               const uint32_t s_lo = prmt(s2, s2, 0x1010u), s_hi = prmt(s2, s2, 0x3232u);
-              r[bp][4 * j + 0] = hmul2_f16(e2m1x2_to_f16x2(wd[j]), s_lo);
-              r[bp][4 * j + 1] = hmul2_f16(e2m1x2_to_f16x2(wd[j] >> 16), s_lo);
-              r[bp][4 * j + 2] = hmul2_f16(e2m1x2_to_f16x2(wd[j] >> 8), s_hi);
-              r[bp][4 * j + 3] = hmul2_f16(e2m1x2_to_f16x2(wd[j] >> 24), s_hi);
+              r[4 * k + 0] = hmul2_f16(e2m1x2_to_f16x2(wd[k]), s_lo);
+              r[4 * k + 1] = hmul2_f16(e2m1x2_to_f16x2(wd[k] >> 16), s_lo);
+              r[4 * k + 2] = hmul2_f16(e2m1x2_to_f16x2(wd[k] >> 8), s_hi);
+              r[4 * k + 3] = hmul2_f16(e2m1x2_to_f16x2(wd[k] >> 24), s_hi);
             }
           }
+          tmem_st_16x256b_x4(tmem + lane_base + kAColBase + slot * 64 + h * 32, r);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(afull + slot);
         }
+        if (!ok) break;
         __syncwarp();
-        if (lane == 0) mbar_arrive(freeb + s);  // this warp's shared-memory reads are done
-#pragma unroll
-        for (int bp = 0; bp < 2; ++bp) {
-          const uint32_t taddr = tmem + ((uint32_t)(32 * q + 16 * bp) << 16) + kAColBase + s * 64 + h * 32;
-          tmem_st_16x256b_x4(taddr, r[bp]);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(afull + s);
+        if (lane == 0) mbar_arrive(sfree + s);  // this warp's shared-memory reads are done
       }
       if (!ok) break;
 
       // ---------------------------------------------------------------- epilogue of a unit
-      if (!tc_wait(dfull, unit_i & 1, abort_flag, p.err)) break;
+      if (!warp_wait(dfull, unit_i & 1, abort_flag, p.err)) break;
       tc_fence_after();
-      float v[MPAD];
+      constexpr int kHalf = MPAD / 2;                   // columns this warp reads
+      float v[kHalf];
 #pragma unroll
-      for (int c = 0; c < MPAD / 16; ++c)
-        tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * q) << 16) + h * 64 + c * 16, v + 16 * c);
+      for (int c = 0; c < kHalf / 8; ++c)
+        tmem_ld_32x32b_x8(tmem + ((uint32_t)(32 * q) << 16) + h * 64 + bp * kHalf + c * 8, v + 8 * c);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dfree);
 
       const int n = tile * kTcTileRows + h * 128 + 32 * q + lane;
+      const int m0 = bp * kHalf;
       float gmul = 1.f;
       if (FMT == 1) gmul = __ldg(p.g);
       if (p.S == 1) {
         if (n < p.N) {
 #pragma unroll
-          for (int m = 0; m < MPAD; ++m) {
+          for (int c = 0; c < kHalf; ++c) {
+            const int m = m0 + c;
             if (m < p.M) {
-              float val = v[m];
+              float val = v[c];
               if (FMT == 1) val = val * __ldg(p.row_mul + m) * gmul;
               p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
             }
@@ -404,8 +468,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const size_t Npad = (size_t)p.NT * 16;
         if (n < p.N) {
 #pragma unroll
-          for (int m = 0; m < MPAD; ++m)
-            if (m < p.M) __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v[m]);
+          for (int c = 0; c < kHalf; ++c) {
+            const int m = m0 + c;
+            if (m < p.M) __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v[c]);
+          }
         }
         __threadfence();
         asm volatile("bar.sync 1, %0;" ::"n"(kDeqWarps * 32));
@@ -414,7 +480,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (*fix_word == static_cast<unsigned>(p.S - 1)) {
           __threadfence();
           if (n < p.N) {
-            for (int m = 0; m < p.M; ++m) {
+            for (int c = 0; c < kHalf; ++c) {
+              const int m = m0 + c;
+              if (m >= p.M) break;
               float acc = 0.f;
               for (int sp = 0; sp < p.S; ++sp) acc += __ldcg(p.ws + ((size_t)sp * p.M + m) * Npad + n);
               if (FMT == 1) acc = acc * __ldg(p.row_mul + m) * gmul;
@@ -549,27 +617,33 @@ TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
   pl.mpad = (M + 15) / 16 * 16;
   const int tiles = (N + kTcTileRows - 1) / kTcTileRows;
   const int KB = K / 64;
+  const int groups = K / 128;
   double best = 1e300;
   int best_s = 1;
-  for (int S = 1; S <= 16 && S <= KB; ++S) {
-    const int kbs = (KB + S - 1) / S;
+  for (int S = 1; S <= 16 && S <= groups; ++S) {
+    const int kbs = 2 * ((groups + S - 1) / S);   // whole 128-groups per split
     if ((S - 1) * kbs >= KB) continue;
     const int units = tiles * S;
     const int waves = (units + num_sms - 1) / num_sms;
-    const double cost = (double)waves * kbs + (S > 1 ? 2.0 : 0.0);
+    const double cost = (double)waves * kbs + (S > 1 ? 4.0 : 0.0);
     if (cost < best - 1e-9) {
       best = cost;
       best_s = S;
     }
   }
   pl.S = best_s;
-  pl.kbs = (KB + pl.S - 1) / pl.S;
+  pl.kbs = 2 * ((groups + pl.S - 1) / pl.S);
   pl.units = tiles * pl.S;
   pl.grid = pl.units < num_sms ? pl.units : num_sms;
-  int smem = kTcStages * (pl.mpad * 128 + kWStage + kSStage) + 256 + 1024;
+  int smem = 0;
+  switch (pl.mpad) {
+    case 16: smem = fmt == 0 ? TcShape<0, 16>::kSmem : TcShape<1, 16>::kSmem; break;
+    case 32: smem = fmt == 0 ? TcShape<0, 32>::kSmem : TcShape<1, 32>::kSmem; break;
+    case 48: smem = fmt == 0 ? TcShape<0, 48>::kSmem : TcShape<1, 48>::kSmem; break;
+    default: smem = fmt == 0 ? TcShape<0, 64>::kSmem : TcShape<1, 64>::kSmem; break;
+  }
   if (smem < kMinSmem) smem = kMinSmem;
   pl.smem = smem;
-  (void)fmt;
   return pl;
 }
 
