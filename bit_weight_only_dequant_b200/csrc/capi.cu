@@ -252,6 +252,7 @@ const char* w4a16_status_string(int status) {
     case W4A16_ERR_CUDA: return "W4A16_ERR_CUDA: CUDA runtime error";
     case W4A16_ERR_TIMEOUT: return "W4A16_ERR_TIMEOUT: a kernel gave up a bounded wait";
     case W4A16_ERR_NOMEM: return "W4A16_ERR_NOMEM: workspace allocation failed";
+    case W4A16_ERR_SCRATCH: return "W4A16_ERR_SCRATCH: problem exceeds the fixed no-alloc scratch";
     default: return "unknown status";
   }
 }

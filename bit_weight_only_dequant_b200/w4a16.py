@@ -22,6 +22,7 @@ FMTS = {"int4": FMT_INT4_G128, "nvfp4": FMT_NVFP4_G16}
 
 OK = 0
 ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_DEVICE, ERR_CUDA, ERR_TIMEOUT, ERR_NOMEM = -1, -2, -3, -4, -5, -6, -7
+ERR_SCRATCH = -8
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 MAX_M = 64
 
@@ -39,6 +40,7 @@ _SIGS = {
     "w4a16_gemm": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_ex": (_i, [_i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_path": (_i, [_i, _i, _i, _i]),
+    "w4a16_gemm_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_device_status": (_i, [_vp]),
     "w4a16_status_string": (ctypes.c_char_p, [_i]),
     "w4a16_version": (_i, []),
@@ -132,6 +134,11 @@ def w4a16_gemm(fmt, M, N, K, x, packed_w, packed_scales, global_scale, y, stream
 def w4a16_gemm_ex(path, fmt, M, N, K, x, packed_w, packed_scales, global_scale, y, stream=None):
     return lib().w4a16_gemm_ex(path, fmt, M, N, K, _ptr(x), _ptr(packed_w), _ptr(packed_scales),
                                _ptr(global_scale), _ptr(y), _stream(stream))
+
+
+def w4a16_gemm_noalloc(fmt, M, N, K, x, packed_w, packed_scales, global_scale, y, stream=None):
+    return lib().w4a16_gemm_noalloc(fmt, M, N, K, _ptr(x), _ptr(packed_w), _ptr(packed_scales),
+                                    _ptr(global_scale), _ptr(y), _stream(stream))
 
 
 def w4a16_gemm_path(fmt, M, N, K):

@@ -65,6 +65,7 @@ extern "C" {
 #define W4A16_ERR_CUDA (-5)    /* a CUDA runtime call or launch failed */
 #define W4A16_ERR_TIMEOUT (-6) /* a kernel gave up a bounded wait (see w4a16_device_status) */
 #define W4A16_ERR_NOMEM (-7)   /* the workspace could not be allocated */
+#define W4A16_ERR_SCRATCH (-8) /* w4a16_gemm_noalloc: the problem needs more than its fixed scratch */
 
 /* Limits of this version. */
 #define W4A16_MAX_M 64         /* decode / speculative-verify row counts */
@@ -135,6 +136,31 @@ int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* pac
 int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16,
                   const void* packed_w, const void* packed_scales, const float* global_scale,
                   void* y_bf16, void* stream);
+
+/*
+ * The split-K GEMV (M <= W4A16_GEMV_MAX_M) for callers that cannot allocate
+ * device memory: code that issues the matmul while its stream is being
+ * captured into a CUDA graph, where cudaMalloc is not allowed, and
+ * applications that reserve all device memory up front in their own pool and
+ * forbid later allocations.  No counterpart on the source pages: it is a
+ * deployment variant of w4a16_gemm.
+ *   Same arguments, layouts and results as w4a16_gemm on the GEMV path.
+ *   Scratch: a fixed 8 MiB array in device global memory owned by the library
+ *   (every GPU that loads the library holds it until the process exits).  A
+ *   call that would need more (split-K partials of large N) returns
+ *   W4A16_ERR_SCRATCH without launching; M > W4A16_GEMV_MAX_M returns
+ *   W4A16_ERR_SHAPE.  Calls neither allocate nor free device memory.
+ *   The first call on a device resolves the array's device address and sets
+ *   kernel attributes; make that first call before any stream capture.
+ *   All calls share the array: calls whose GPU work overlaps (different
+ *   streams, or threads sharing a device) race and must be serialised by the
+ *   caller.  Each call clears, in stream order, the parts that must start at
+ *   zero.  A bounded-wait timeout inside this call is recorded in the array's
+ *   own status word and is not reported by w4a16_device_status.
+ */
+int w4a16_gemm_noalloc(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
+                       const void* packed_scales, const float* global_scale, void* y_bf16,
+                       void* stream);
 
 /* The path W4A16_PATH_AUTO would take for these arguments (>0), or a status. */
 int w4a16_gemm_path(int fmt, int M, int N, int K);
