@@ -8,17 +8,21 @@
 // nibbles into multiply operands: at 7+ TB/s a B200 SM has about two
 // lane-instructions per weight.
 //
-// Structure (one CTA of 16 warps per SM, no producer warp):
+// Structure (one CTA of 16 warps per SM):
 //  * A CTA owns one K-slice and a contiguous range of 16-row bands.  Its
 //    warps form a (Wn x Wk) grid: Wn bands in flight at a time, each band's
 //    slice cut into Wk equal group-aligned pieces, one per warp, so every warp
 //    streams the same number of bytes.  The Wk partial sums of a band are
 //    added in piece order through shared memory (deterministic).
-//  * The CTA first copies its slice of the activations into shared memory,
-//    k reordered inside every 16-block to match the packed operand fragments
+//  * The CTA copies its slice of the activations into shared memory, k
+//    reordered inside every 16-block to match the packed operand fragments
 //    (NVFP4: rows rescaled by a power of two into FP16).
-//  * Each warp streams its pieces through a private 2-stage ring of 4.5 KB
-//    stages filled by 1-D bulk copies (TMA) completing on mbarriers.
+//  * Each warp streams its pieces straight into registers: every lane loads
+//    its 16 bytes of each 512-byte tile with a 128-bit read-only global load
+//    (a warp load covers one whole tile), prefetched four 128-groups ahead, so
+//    ~64 KB per SM are in flight without shared memory, TMA issue or barrier
+//    polling on the weight stream.  The first loads are issued before the
+//    activations are staged.
 //  * Per 32-bit word (8 weights) a lane builds the A fragment of one
 //    mma.sync m16n8k16 (16 output columns x 16 k): 3 shifts, 4 LOP3 and
 //    4 exact BF16 subtractions (int4), or 4 hardware e2m1 -> f16 conversions
@@ -34,14 +38,11 @@ namespace w4 {
 
 namespace {
 
-#ifndef W4_GEMV_STAGES
-#define W4_GEMV_STAGES 2
-#endif
-#ifndef W4_GEMV_STAGE_KB
-#define W4_GEMV_STAGE_KB 8
-#endif
 #ifndef W4_GEMV_INT4_F16
 #define W4_GEMV_INT4_F16 0
+#endif
+#ifndef W4_GEMV_PREFETCH
+#define W4_GEMV_PREFETCH 4
 #endif
 // Activations go to the tensor cores as FP16 (rescaled per row slice) for
 // NVFP4 always, and for int4 when W4_GEMV_INT4_F16 is set.
@@ -51,22 +52,15 @@ struct XF16 {
 };
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = W4_GEMV_STAGES;
-constexpr int kStageKB = W4_GEMV_STAGE_KB;                   // k64 blocks per stage (even)
-constexpr int kStageWBytes = kStageKB * kTileBytes;
-constexpr int kStageSBytes = kStageKB * 64;                  // room for NVFP4 scales
-constexpr int kStageBytes = kStageWBytes + kStageSBytes;
+constexpr int kPD = W4_GEMV_PREFETCH;                       // 128-groups in flight per warp
 constexpr int kMaxMT = 2;                                    // M <= 16
-constexpr int kBarBytes = (kWarps * kStages * 8 + 127) / 128 * 128;
 constexpr int kRowWords = 64;                                // per-row words (M <= 64)
-constexpr int kZeroOff = kBarBytes + 2 * kRowWords * 4;      // 128 zero bytes
+constexpr int kZeroOff = 2 * kRowWords * 4;                  // 128 zero bytes
 constexpr int kRedOff = kZeroOff + 128;
 constexpr int kRedBytes = kWarps * 32 * 4 * kMaxMT * 4;      // per-lane partial sums
 constexpr int kHeaderBytes = kRedOff + kRedBytes;
-constexpr int kRingBytes = kWarps * kStages * kStageBytes;
 constexpr int kMaxSmem = 232448;                             // 227 KB opt-in
-static_assert(kStageKB % 2 == 0, "stages hold whole 128-groups");
-static_assert(kHeaderBytes % 128 == 0, "ring alignment");
+static_assert(kHeaderBytes % 128 == 0, "activation image alignment");
 
 struct Params {
   const __nv_bfloat16* x;
@@ -160,13 +154,38 @@ __device__ __forceinline__ void mma_f16_first(float* c, const uint32_t* a, uint3
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-// One 128-group (two 64-blocks) of one band: int4.
+// Streaming read-only loads of the packed weights (read once: no L1 allocation,
+// evict first from L2).
+__device__ __forceinline__ uint4 ldg_stream16(const uint8_t* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ uint2 ldg_stream8(const uint8_t* p, uint64_t pol) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
+               : "=r"(v.x), "=r"(v.y)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_stream4(const uint8_t* p, uint64_t pol) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.u32 %0, [%1], %2;"
+               : "=r"(v)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+// One 128-group (two 64-blocks) of one band, int4.  w0/w1: this lane's words
+// of the two tiles; sp: BF16 scales of rows g and g+8.
 template <int MT>
-__device__ __forceinline__ void group_int4(const uint8_t* sw, const uint8_t* ss, int lane, int g,
+__device__ __forceinline__ void group_int4(uint4 w0, uint4 w1, uint32_t sp,
                                            const uint8_t* const* xrow, const int* xstep, int kbl,
                                            float (*acc)[4]) {
-  const uint4 w0 = *reinterpret_cast<const uint4*>(sw + lane * 16);
-  const uint4 w1 = *reinterpret_cast<const uint4*>(sw + kTileBytes + lane * 16);
   const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
   uint32_t a[8][4];
 #pragma unroll
@@ -185,7 +204,6 @@ __device__ __forceinline__ void group_int4(const uint8_t* sw, const uint8_t* ss,
       a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
     }
   }
-  const uint32_t sp = *reinterpret_cast<const uint32_t*>(ss + g * 4);
   const float s_lo = __uint_as_float(sp << 16);          // row g
   const float s_hi = __uint_as_float(sp & 0xFFFF0000u);  // row g + 8
 #pragma unroll
@@ -212,12 +230,11 @@ __device__ __forceinline__ void group_int4(const uint8_t* sw, const uint8_t* ss,
   }
 }
 
-// One 64-block of one band: NVFP4 (a scale per 16-group, i.e. per MMA).
+// One 64-block of one band, NVFP4 (a scale per 16-group, i.e. per MMA).  wv:
+// this lane's words of the tile; sv: E4M3 scales of rows g and g+8, 4 groups.
 template <int MT>
-__device__ __forceinline__ void block_nvfp4(const uint8_t* sw, const uint8_t* ss, int lane, int g,
-                                            const uint8_t* const* xrow, const int* xstep, int kbl,
-                                            float (*acc)[4]) {
-  const uint4 wv = *reinterpret_cast<const uint4*>(sw + lane * 16);
+__device__ __forceinline__ void block_nvfp4(uint4 wv, uint2 sv, const uint8_t* const* xrow,
+                                            const int* xstep, int kbl, float (*acc)[4]) {
   const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
   uint32_t a[4][4];
 #pragma unroll
@@ -227,7 +244,6 @@ __device__ __forceinline__ void block_nvfp4(const uint8_t* sw, const uint8_t* ss
     a[j][2] = e2m1x2_to_f16x2(wd[j] >> 16);
     a[j][3] = e2m1x2_to_f16x2(wd[j] >> 24);
   }
-  const uint2 sv = *reinterpret_cast<const uint2*>(ss + g * 8);
   const uint32_t sw2[2] = {sv.x, sv.y};
   float2 sf[4];
 #pragma unroll
@@ -308,16 +324,40 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
   if (lane == 0) p.counters[band] = 0u;
 }
 
+// The words a lane needs for one 128-group of one band.
+struct GroupWords {
+  uint4 w0, w1;   // the two 64-blocks
+  uint2 s0, s1;   // int4: s0.x = scales of rows g, g+8; NVFP4: per-block E4M3 scales
+};
+
+template <int FMT>
+__device__ __forceinline__ GroupWords load_group(const Params& p, int band, int kb, int lane,
+                                                 uint64_t pol) {
+  GroupWords gw;
+  const int g = lane >> 2;
+  const uint8_t* wt = p.w + ((size_t)band * (p.K >> 6) + kb) * kTileBytes + lane * 16;
+  gw.w0 = ldg_stream16(wt, pol);
+  gw.w1 = ldg_stream16(wt + kTileBytes, pol);
+  if (FMT == 0) {
+    gw.s0.x = ldg_stream4(p.s + ((size_t)band * (p.K >> 7) + (kb >> 1)) * 32 + g * 4, pol);
+    gw.s0.y = 0u;
+    gw.s1 = make_uint2(0u, 0u);
+  } else {
+    const uint8_t* st = p.s + ((size_t)band * (p.K >> 6) + kb) * 64 + g * 8;
+    gw.s0 = ldg_stream8(st, pol);
+    gw.s1 = ldg_stream8(st + 64, pol);
+  }
+  return gw;
+}
+
 template <int FMT, int MT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-  float* row_mul = reinterpret_cast<float*>(smem + kBarBytes);
-  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kBarBytes + kRowWords * 4);
+  float* row_mul = reinterpret_cast<float*>(smem);
+  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kRowWords * 4);
   const uint8_t* zero = smem + kZeroOff;
   float* red = reinterpret_cast<float*>(smem + kRedOff);
-  uint8_t* ring = smem + kHeaderBytes;
-  uint8_t* xs = ring + kRingBytes;
+  uint8_t* xs = smem + kHeaderBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -328,51 +368,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
   const int band_hi = (int)(((long long)(blockIdx.x + 1) * p.NT) / p.ctas_x);
   const int nbands = band_hi - band_lo;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kWarps * kStages; ++i) mbar_init(bars + i, 1);
-    fence_mbar_init();
-  }
-  if (threadIdx.x < 32) reinterpret_cast<uint32_t*>(smem + kZeroOff)[threadIdx.x] = 0u;
-  stage_activations<FMT>(p, k_lo, k_len, xs, row_mul, row_aux);  // ends with __syncthreads
-
-  // warp grid: wi = band slot, wj = K piece
+  // warp grid: wi = band slot, wj = K piece of whole 128-groups
   const int wi = warp % p.wn, wj = warp / p.wn;
   const int groups = k_len >> 7;
   const int g_lo = wj * groups / p.wk, g_hi = (wj + 1) * groups / p.wk;
-  const int kbl_lo = 2 * g_lo;                 // slice-local first 64-block of the piece
-  const int nkb = 2 * (g_hi - g_lo);           // 64-blocks in the piece
+  const int ng = g_hi - g_lo;                  // 128-groups in this warp's piece
+  const int kb_base = (k_lo >> 6) + 2 * g_lo;  // first 64-block (global) of the piece
   const int rounds = (nbands + p.wn - 1) / p.wn;
   const int my_rounds = wi < nbands ? (nbands - wi + p.wn - 1) / p.wn : 0;
-  const int spb = (nkb + kStageKB - 1) / kStageKB;   // stages per band piece
-  const int total = my_rounds * spb;
-  uint64_t* my_bars = bars + warp * kStages;
-  uint8_t* my_ring = ring + warp * kStages * kStageBytes;
-  const int KB = p.K >> 6;
   const uint64_t pol = policy_evict_first();
 
-  auto issue = [&](int L) {
-    const int r = L / spb, st = L - r * spb;
-    const int band = band_lo + wi + r * p.wn;
-    const int kb0 = (k_lo >> 6) + kbl_lo + st * kStageKB;
-    const int nblk = min(kStageKB, nkb - st * kStageKB);
-    const int buf = L % kStages;
-    uint8_t* dst = my_ring + buf * kStageBytes;
-    const uint8_t* wsrc = p.w + ((size_t)band * KB + kb0) * kTileBytes;
-    uint32_t sbytes;
-    const uint8_t* ssrc;
-    if (FMT == 0) {
-      sbytes = nblk * 16;
-      ssrc = p.s + ((size_t)band * (p.K >> 7) + (kb0 >> 1)) * 32;
-    } else {
-      sbytes = nblk * 64;
-      ssrc = p.s + ((size_t)band * KB + kb0) * 64;
-    }
-    mbar_arrive_expect_tx(my_bars + buf, nblk * kTileBytes + sbytes);
-    bulk_g2s_evict_first(dst, wsrc, nblk * kTileBytes, my_bars + buf, pol);
-    bulk_g2s_evict_first(dst + kStageWBytes, ssrc, sbytes, my_bars + buf, pol);
-  };
-  if (lane == 0)
-    for (int L = 0; L < min(kStages, total); ++L) issue(L);
+  // the first loads go out before the activations are staged
+  GroupWords buf[kPD];
+  if (my_rounds > 0) {
+#pragma unroll
+    for (int u = 0; u < kPD; ++u)
+      if (u < ng) buf[u] = load_group<FMT>(p, band_lo + wi, kb_base + 2 * u, lane, pol);
+  }
+
+  if (threadIdx.x < 32) reinterpret_cast<uint32_t*>(smem + kZeroOff)[threadIdx.x] = 0u;
+  stage_activations<FMT>(p, k_lo, k_len, xs, row_mul, row_aux);  // ends with __syncthreads
 
   // activation rows of this lane (row m = 8 mt + g); rows past M read zeros
   const uint8_t* xrow[MT];
@@ -384,43 +399,42 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
     xrow[mt] = real ? xs + (size_t)m * p.row_stride + t * 32 : zero;
     xstep[mt] = real ? 128 : 0;
   }
+  const int kbl_base = 2 * g_lo;               // slice-local first 64-block of the piece
 
-  bool failed = false;
-  int L = 0;
   for (int r = 0; r < rounds; ++r) {
     float acc[MT][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
-    const bool active = r < my_rounds && !failed;
+    const bool active = r < my_rounds;
+    const int band = band_lo + wi + r * p.wn;
     if (active) {
-      for (int st = 0; st < spb; ++st, ++L) {
-        const int buf = L % kStages;
-        if (!mbar_wait(my_bars + buf, (L / kStages) & 1, p.err)) {
-          failed = true;
-          break;
+      if (r > 0) {
+#pragma unroll
+        for (int u = 0; u < kPD; ++u)
+          if (u < ng) buf[u] = load_group<FMT>(p, band, kb_base + 2 * u, lane, pol);
+      }
+      for (int gi0 = 0; gi0 < ng; gi0 += kPD) {
+#pragma unroll
+        for (int u = 0; u < kPD; ++u) {
+          const int gi = gi0 + u;
+          if (gi < ng) {
+            const GroupWords cur = buf[u];
+            if (gi + kPD < ng) buf[u] = load_group<FMT>(p, band, kb_base + 2 * (gi + kPD), lane, pol);
+            const int kbl = kbl_base + 2 * gi;
+            if (FMT == 0) {
+              group_int4<MT>(cur.w0, cur.w1, cur.s0.x, xrow, xstep, kbl, acc);
+            } else {
+              block_nvfp4<MT>(cur.w0, cur.s0, xrow, xstep, kbl, acc);
+              block_nvfp4<MT>(cur.w1, cur.s1, xrow, xstep, kbl + 1, acc);
+            }
+          }
         }
-        const uint8_t* sw = my_ring + buf * kStageBytes;
-        const uint8_t* ss = sw + kStageWBytes;
-        const int nblk = min(kStageKB, nkb - st * kStageKB);
-        const int kbl0 = kbl_lo + st * kStageKB;
-        if (FMT == 0) {
-          for (int gi = 0; gi < (nblk >> 1); ++gi)
-            group_int4<MT>(sw + gi * 2 * kTileBytes, ss + gi * 32, lane, g, xrow, xstep,
-                           kbl0 + 2 * gi, acc);
-        } else {
-          for (int bb = 0; bb < nblk; ++bb)
-            block_nvfp4<MT>(sw + bb * kTileBytes, ss + bb * 64, lane, g, xrow, xstep, kbl0 + bb,
-                            acc);
-        }
-        __syncwarp();
-        if (lane == 0 && L + kStages < total) issue(L + kStages);
       }
     }
-    const int band = band_lo + wi + r * p.wn;
     if (p.wk == 1) {
-      if (active && !failed) band_epilogue<FMT, MT>(p, band, split, lane, row_mul, acc);
+      if (active) band_epilogue<FMT, MT>(p, band, split, lane, row_mul, acc);
       continue;
     }
     // add the wk pieces of each band in piece order
@@ -428,9 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) mine[mt * 4 + i] = (active && !failed) ? acc[mt][i] : 0.f;
+      for (int i = 0; i < 4; ++i) mine[mt * 4 + i] = active ? acc[mt][i] : 0.f;
     __syncthreads();
-    if (wj == 0 && active && !failed) {
+    if (wj == 0 && active) {
       float sum[MT][4];
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
@@ -446,12 +460,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
       band_epilogue<FMT, MT>(p, band, split, lane, row_mul, sum);
     }
     __syncthreads();
-  }
-
-  if (failed) {
-    // let this warp's outstanding copies land before the CTA can exit
-    for (int LL = L; LL < min(L + kStages, total); ++LL)
-      mbar_wait(my_bars + (LL % kStages), (LL / kStages) & 1, p.err);
   }
 }
 
@@ -503,7 +511,7 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
   pl.mt = M <= 8 ? 1 : 2;
   const int NT = (N + 15) / 16;
   const int groups = K / 128;
-  const int xbudget = kMaxSmem - kHeaderBytes - kRingBytes;
+  const int xbudget = kMaxSmem - kHeaderBytes;
   const int max_groups = (xbudget / M - 16) / 256;
   const int s_min = (groups + max_groups - 1) / max_groups;
   double best = 1e300;
@@ -536,7 +544,7 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
   if (ctas < 1) ctas = 1;
   if (ctas > NT) ctas = NT;
   pl.ctas_x = ctas;
-  pl.smem = kHeaderBytes + kRingBytes + M * ((pl.kslice / 64) * 128 + 16);
+  pl.smem = kHeaderBytes + M * ((pl.kslice / 64) * 128 + 16);
   return pl;
 }
 
