@@ -50,7 +50,10 @@ template <int FMT>
 struct XF16 {
   static constexpr bool value = FMT == 1 || W4_GEMV_INT4_F16 != 0;
 };
-constexpr int kWarps = 16;
+#ifndef W4_GEMV_WARPS
+#define W4_GEMV_WARPS 16
+#endif
+constexpr int kWarps = W4_GEMV_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kPD = W4_GEMV_PREFETCH;                       // 128-groups in flight per warp
 constexpr int kMaxMT = 2;                                    // M <= 16
@@ -186,47 +189,53 @@ template <int MT>
 __device__ __forceinline__ void group_int4(uint4 w0, uint4 w1, uint32_t sp,
                                            const uint8_t* const* xrow, const int* xstep, int kbl,
                                            float (*acc)[4]) {
-  const uint32_t wd[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-  uint32_t a[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (W4_GEMV_INT4_F16) {
-      // FP16 holds two nibbles per 16-bit half in its mantissa: one shift per word
-      const uint32_t hi = wd[j] >> 8;
-      a[j][0] = int4_lo_pair_to_f16x2(wd[j]);
-      a[j][1] = int4_hi_pair_to_f16x2(wd[j]);
-      a[j][2] = int4_lo_pair_to_f16x2(hi);
-      a[j][3] = int4_hi_pair_to_f16x2(hi);
-    } else {
-      a[j][0] = int4_pair_to_bf16x2(wd[j]);
-      a[j][1] = int4_pair_to_bf16x2(wd[j] >> 4);
-      a[j][2] = int4_pair_to_bf16x2(wd[j] >> 8);
-      a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
-    }
-  }
   const float s_lo = __uint_as_float(sp << 16);          // row g
   const float s_hi = __uint_as_float(sp & 0xFFFF0000u);  // row g + 8
+  float c[MT][4];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint4 wv = half ? w1 : w0;
+    const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+    uint32_t a[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (W4_GEMV_INT4_F16) {
+        // FP16 holds two nibbles per 16-bit half in its mantissa: one shift per word
+        const uint32_t hi = wd[j] >> 8;
+        a[j][0] = int4_lo_pair_to_f16x2(wd[j]);
+        a[j][1] = int4_hi_pair_to_f16x2(wd[j]);
+        a[j][2] = int4_lo_pair_to_f16x2(hi);
+        a[j][3] = int4_hi_pair_to_f16x2(hi);
+      } else {
+        a[j][0] = int4_pair_to_bf16x2(wd[j]);
+        a[j][1] = int4_pair_to_bf16x2(wd[j] >> 4);
+        a[j][2] = int4_pair_to_bf16x2(wd[j] >> 8);
+        a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const uint4* xb = reinterpret_cast<const uint4*>(xrow[mt] + (kbl + half) * xstep[mt]);
+      const uint4 v0 = xb[0], v1 = xb[1];
+      const uint32_t bx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (W4_GEMV_INT4_F16) {
+          if (half == 0 && j == 0) mma_f16_first(c[mt], a[0], bx[0], bx[1]);
+          else mma_f16_16816(c[mt], a[j], bx[2 * j], bx[2 * j + 1]);
+        } else {
+          if (half == 0 && j == 0) mma_bf16_first(c[mt], a[0], bx[0], bx[1]);
+          else mma_bf16_16816(c[mt], a[j], bx[2 * j], bx[2 * j + 1]);
+        }
+      }
+    }
+  }
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
-    const uint4* xb0 = reinterpret_cast<const uint4*>(xrow[mt] + kbl * xstep[mt]);
-    const uint4* xb1 = reinterpret_cast<const uint4*>(xrow[mt] + (kbl + 1) * xstep[mt]);
-    const uint4 v0 = xb0[0], v1 = xb0[1], v2 = xb1[0], v3 = xb1[1];
-    const uint32_t bx[16] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w,
-                             v2.x, v2.y, v2.z, v2.w, v3.x, v3.y, v3.z, v3.w};
-    float c[4];
-    if (W4_GEMV_INT4_F16) {
-      mma_f16_first(c, a[0], bx[0], bx[1]);
-#pragma unroll
-      for (int j = 1; j < 8; ++j) mma_f16_16816(c, a[j], bx[2 * j], bx[2 * j + 1]);
-    } else {
-      mma_bf16_first(c, a[0], bx[0], bx[1]);
-#pragma unroll
-      for (int j = 1; j < 8; ++j) mma_bf16_16816(c, a[j], bx[2 * j], bx[2 * j + 1]);
-    }
-    acc[mt][0] = fmaf(s_lo, c[0], acc[mt][0]);
-    acc[mt][1] = fmaf(s_lo, c[1], acc[mt][1]);
-    acc[mt][2] = fmaf(s_hi, c[2], acc[mt][2]);
-    acc[mt][3] = fmaf(s_hi, c[3], acc[mt][3]);
+    acc[mt][0] = fmaf(s_lo, c[mt][0], acc[mt][0]);
+    acc[mt][1] = fmaf(s_lo, c[mt][1], acc[mt][1]);
+    acc[mt][2] = fmaf(s_hi, c[mt][2], acc[mt][2]);
+    acc[mt][3] = fmaf(s_hi, c[mt][3], acc[mt][3]);
   }
 }
 
@@ -526,6 +535,7 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
     const int bands_max = (NT + ctas - 1) / ctas;
     for (int wk = 1; wk <= kWarps; wk *= 2) {
       if (wk > gslice) break;
+      if (kWarps % wk != 0) continue;
       const int wn = kWarps / wk;
       const int rounds = (bands_max + wn - 1) / wn;
       const int piece = 2 * ((gslice + wk - 1) / wk);
