@@ -102,10 +102,11 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 
 // ------------------------------------------------------------------ bit tricks
 
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
-  // (a & mask) | magic
+// (a & MASK) | MAGIC with both constants as instruction immediates
+template <uint32_t MASK, uint32_t MAGIC>
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a) {
   uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "n"(MAGIC));
   return d;
 }
 
@@ -113,7 +114,7 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
 // q = u - 8, exact.  0x4300 is BF16 128.0 whose last mantissa bit weighs 1, so
 // OR-ing a nibble into it gives 128 + u; subtracting 136 leaves q.
 __device__ __forceinline__ uint32_t int4_pair_to_bf16x2(uint32_t w) {
-  const uint32_t v = lop3_and_or(w, 0x000F000Fu, 0x43004300u);
+  const uint32_t v = lop3_and_or<0x000F000Fu, 0x43004300u>(w);
   uint32_t d;
   const uint32_t bias = 0x43084308u;  // BF16 136.0, twice
   asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(bias));
@@ -124,13 +125,13 @@ __device__ __forceinline__ uint32_t int4_pair_to_bf16x2(uint32_t w) {
 // LSB of 1 and ten mantissa bits, so a nibble at bits 0..3 gives 1024 + u and
 // a nibble at bits 4..7 gives 1024 + 16 u; exact arithmetic then leaves q.
 __device__ __forceinline__ uint32_t int4_lo_pair_to_f16x2(uint32_t w) {
-  const uint32_t v = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
+  const uint32_t v = lop3_and_or<0x000F000Fu, 0x64006400u>(w);
   uint32_t d;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(0x64086408u));  // - 1032
   return d;
 }
 __device__ __forceinline__ uint32_t int4_hi_pair_to_f16x2(uint32_t w) {
-  const uint32_t v = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
+  const uint32_t v = lop3_and_or<0x00F000F0u, 0x64006400u>(w);
   uint32_t d;
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(v), "r"(0x2C002C00u), "r"(0xD480D480u));  // /16 - 72
   return d;

@@ -8,27 +8,34 @@
 // nibbles into multiply operands: at 7+ TB/s a B200 SM has about two
 // lane-instructions per weight.
 //
-// Structure (one CTA of 16 warps per SM):
+// Structure (one CTA per SM; 32 warps for int4 at M <= 8, 24 for NVFP4,
+// 16 for M <= 16):
 //  * A CTA owns one K-slice and a contiguous range of 16-row bands.  Its
 //    warps form a (Wn x Wk) grid: Wn bands in flight at a time, each band's
-//    slice cut into Wk equal group-aligned pieces, one per warp, so every warp
-//    streams the same number of bytes.  The Wk partial sums of a band are
-//    added in piece order through shared memory (deterministic).
-//  * The CTA copies its slice of the activations into shared memory, k
-//    reordered inside every 16-block to match the packed operand fragments
-//    (NVFP4: rows rescaled by a power of two into FP16).
-//  * Each warp streams its pieces straight into registers: every lane loads
-//    its 16 bytes of each 512-byte tile with a 128-bit read-only global load
-//    (a warp load covers one whole tile), prefetched four 128-groups ahead, so
-//    ~64 KB per SM are in flight without shared memory, TMA issue or barrier
-//    polling on the weight stream.  The first loads are issued before the
-//    activations are staged.
+//    slice cut into Wk group-aligned pieces, one per warp.  The Wk partial
+//    sums of a band are added in piece order through shared memory
+//    (deterministic).
+//  * Each warp streams its pieces, one 128-group (two 512-byte tiles and
+//    their scales) at a time, through its own ring of shared-memory stages
+//    filled by cp.async: every lane copies, and later reads back, exactly its
+//    own 16 bytes of each tile (a warp's copies cover the whole tile), so no
+//    barrier guards the ring; only the lane's own cp.async groups are waited
+//    for.  The ring holds up to six groups per warp (about 190 KB per SM in
+//    flight) without spending registers, and runs on from one band's piece
+//    into the next.  The first copies are issued before the activations are
+//    staged and, under programmatic dependent launch, before the previous
+//    kernel on the stream has finished: only the activations depend on it.
+//  * The CTA copies its slice of the activations into shared memory as FP16,
+//    each row rescaled by a power of two so that its largest magnitude lies in
+//    [2^14, 2^15) (exact for every BF16 value in FP16's normal range), k
+//    reordered inside every 16-block to match the packed operand fragments.
 //  * Per 32-bit word (8 weights) a lane builds the A fragment of one
-//    mma.sync m16n8k16 (16 output columns x 16 k): 3 shifts, 4 LOP3 and
-//    4 exact BF16 subtractions (int4), or 4 hardware e2m1 -> f16 conversions
-//    (NVFP4).  The activations are the n8 side: one MMA serves 8 rows.
-//    Group scales multiply the fp32 MMA results (int4: once per 128-group,
-//    NVFP4: once per 16-group).
+//    mma.sync m16n8k16 (16 output columns x 16 k) with exact FP16 arithmetic:
+//    int4: 1 shift, 4 LOP3 that drop each nibble into the mantissa of FP16
+//    1024.0, then 4 subtractions / fused multiply-adds that leave q; NVFP4:
+//    4 hardware e2m1 -> f16 conversions.  The activations are the n8 side:
+//    one MMA serves 8 rows.  Group scales multiply the fp32 MMA results
+//    (int4: once per 128-group, NVFP4: once per 16-group).
 //  * Split-K partials across CTAs go to a fp32 workspace; the last CTA to
 //    finish a band (arrival counter) adds them in split order.
 #include "common.cuh"
@@ -38,32 +45,28 @@ namespace w4 {
 
 namespace {
 
-#ifndef W4_GEMV_INT4_F16
-#define W4_GEMV_INT4_F16 0
-#endif
-#ifndef W4_GEMV_PREFETCH
-#define W4_GEMV_PREFETCH 4
-#endif
-// Activations go to the tensor cores as FP16 (rescaled per row slice) for
-// NVFP4 always, and for int4 when W4_GEMV_INT4_F16 is set.
-template <int FMT>
-struct XF16 {
-  static constexpr bool value = FMT == 1 || W4_GEMV_INT4_F16 != 0;
-};
-#ifndef W4_GEMV_WARPS
-#define W4_GEMV_WARPS 16
-#endif
-constexpr int kWarps = W4_GEMV_WARPS;
-constexpr int kThreads = kWarps * 32;
-constexpr int kPD = W4_GEMV_PREFETCH;                       // 128-groups in flight per warp
-constexpr int kMaxMT = 2;                                    // M <= 16
 constexpr int kRowWords = 64;                                // per-row words (M <= 64)
+constexpr int kRowAuxOff = kRowWords * 4;
 constexpr int kZeroOff = 2 * kRowWords * 4;                  // 128 zero bytes
 constexpr int kRedOff = kZeroOff + 128;
-constexpr int kRedBytes = kWarps * 32 * 4 * kMaxMT * 4;      // per-lane partial sums
-constexpr int kHeaderBytes = kRedOff + kRedBytes;
 constexpr int kMaxSmem = 232448;                             // 227 KB opt-in
-static_assert(kHeaderBytes % 128 == 0, "activation image alignment");
+constexpr int kMaxDepth = 6;                                 // ring stages per warp
+constexpr int kGroupBytes = 2 * kTileBytes;                  // packed weights of one band-group
+
+// Shared-memory bytes of one ring stage: the group's two tiles, then the
+// scales each lane needs (int4: 4 bytes, NVFP4: 2 x 8 bytes per lane).
+__host__ __device__ constexpr int stage_bytes(int fmt) { return kGroupBytes + (fmt == 0 ? 128 : 512); }
+
+// Warps per CTA, per (format, 8-row tiles): a power of two (the warp grid is
+// split with shifts).  32 warps leave 64 registers a thread, enough at
+// M <= 8; M <= 16 needs the registers of a 16-warp CTA.
+template <int FMT, int MT>
+struct Cfg {
+  static constexpr int kWarps = MT == 2 ? 16 : 32;
+  static constexpr int kRedBytes = kWarps * 32 * 4 * MT * 4;  // per-lane partial sums
+  static constexpr int kHeader = (kRedOff + kRedBytes + 127) / 128 * 128;
+  static constexpr int kCache = 4;                              // staging chunks in registers
+};
 
 struct Params {
   const __nv_bfloat16* x;
@@ -74,9 +77,40 @@ struct Params {
   float* ws;
   unsigned* counters;
   unsigned* err;
-  int M, N, K, NT, S, kslice, ctas_x, row_stride;  // row_stride in bytes
-  int wn, wk;                                      // warp grid: bands x pieces
+  int M, N, K, NT, S, kslice, row_stride;          // row_stride in bytes
+  int bq, br;                                      // bands per CTA: bq, plus one for the first br
+  int wn, wn_log2, wk_log2;                        // warp grid: wn bands x 2^wk_log2 pieces
+  int ngp;                                         // groups per piece, padded to the ring depth
 };
+
+// Programmatic dependent launch: let the next kernel on the stream start its
+// prologue, and wait for the previous one before touching data it may write.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ------------------------------------------------------------------ cp.async
+
+__device__ __forceinline__ void cpa16(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void cpa8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cpa_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ------------------------------------------------------------------ activations
 
 // Element kin of a 64-block sits at this element offset of the block's image
 // in shared memory: lane t reads 16 contiguous elements k = 16 j + 4 t + e.
@@ -85,71 +119,87 @@ __device__ __forceinline__ int perm64(int kin) {
   return t * 16 + j * 4 + e;
 }
 
-template <int FMT>
+__device__ __forceinline__ float max_abs8(uint4 v) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  float mx = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    mx = fmaxf(mx, fabsf(__uint_as_float(u[e] << 16)));
+    mx = fmaxf(mx, fabsf(__uint_as_float(u[e] & 0xFFFF0000u)));
+  }
+  return mx;
+}
+
+// Copy x[:, k_lo:k_lo+k_len] into the FP16 image (see the file comment).
+// Each row is handled by W/M whole warps, so a thread's chunks (8 BF16) all
+// belong to one row.  row_aux must be zero and visible to all threads on
+// entry; ends with a barrier after which the image and row_mul are valid.
+template <int CACHE>
 __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t* xs,
                                   float* row_mul, unsigned* row_aux) {
-  const int tid = threadIdx.x;
-  const int chunks_per_row = k_len / 8;  // 8 elements per 16-byte load
-  if (XF16<FMT>::value) {
-    if (tid < kRowWords) row_aux[tid] = 0u;
-    __syncthreads();
-    for (int m = 0; m < p.M; ++m) {
-      float mx = 0.f;
-      const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + k_lo);
-      for (int c = tid; c < chunks_per_row; c += blockDim.x) {
-        const uint4 v = src[c];
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  const int warps = blockDim.x >> 5;
+  const int wpr = warps / p.M;                      // warps per row (>= 1 since M <= warps)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = warp / wpr;
+  const bool worker = m < p.M;
+  const int tpr = wpr * 32;                         // threads per row
+  const int j = (warp - m * wpr) * 32 + lane;       // index within the row's threads
+  const int cpr = k_len / 8;                        // 16-byte chunks per row
+  const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)(worker ? m : 0) * p.K + k_lo);
+  uint4 cache[CACHE];
+  float mx = 0.f;
+  if (worker) {
+    for (int c0 = 0; c0 < cpr; c0 += CACHE * tpr) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          mx = fmaxf(mx, fabsf(__uint_as_float(u[i] << 16)));
-          mx = fmaxf(mx, fabsf(__uint_as_float(u[i] & 0xFFFF0000u)));
-        }
+      for (int i = 0; i < CACHE; ++i) {
+        const int c = c0 + i * tpr + j;
+        const uint4 v = c < cpr ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        if (c0 == 0) cache[i] = v;
+        mx = fmaxf(mx, max_abs8(v));
       }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if ((tid & 31) == 0) atomicMax(row_aux + m, __float_as_uint(mx));
     }
-    __syncthreads();
-    if (tid < p.M) {
-      const float mx = __uint_as_float(row_aux[tid]);
-      int e = 0;
-      if (mx > 0.f && isfinite(mx)) e = ilogbf(mx) - 14;  // max * 2^-e in [2^14, 2^15)
-      row_mul[tid] = ldexpf(1.f, e);
-      row_aux[tid] = static_cast<unsigned>(-e);           // exponent applied to the row
-    }
-    __syncthreads();
+    const unsigned r = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+    if (lane == 0) atomicMax(row_aux + m, r);
   }
-  for (int idx = tid; idx < p.M * chunks_per_row; idx += blockDim.x) {
-    const int m = idx / chunks_per_row, c = idx - m * chunks_per_row;
-    const uint4 v = reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + k_lo)[c];
-    const int kin0 = c * 8;
-    const int blk = kin0 >> 6, in = kin0 & 63;
-    uint32_t out[4] = {v.x, v.y, v.z, v.w};
-    if (XF16<FMT>::value) {
-      const int sh = static_cast<int>(row_aux[m]);
+  __syncthreads();
+  if (!worker) {
+    __syncthreads();
+    return;
+  }
+  const float rmax = __uint_as_float(row_aux[m]);
+  const bool scaled = rmax > 0.f && isfinite(rmax);
+  // max * 2^sh in [2^14, 2^15); |sh| <= 126 keeps 2^sh and 2^-sh normal floats
+  // (rows whose largest magnitude is below 2^-112 keep fewer FP16 bits)
+  const int sh = scaled ? min(126, 14 - ilogbf(rmax)) : 0;
+  const float mul = __int_as_float((127 + sh) << 23);        // 2^sh, exact
+  if (j == 0) row_mul[m] = __int_as_float((127 - sh) << 23);  // 2^-sh
+  uint8_t* row = xs + (size_t)m * p.row_stride;
+  for (int c0 = 0; c0 < cpr; c0 += CACHE * tpr) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = ldexpf(__uint_as_float(out[i] << 16), sh);
-        const float hi = ldexpf(__uint_as_float(out[i] & 0xFFFF0000u), sh);
-        __half2 h = __floats2half2_rn(lo, hi);
-        out[i] = *reinterpret_cast<uint32_t*>(&h);
+    for (int i = 0; i < CACHE; ++i) {
+      const int c = c0 + i * tpr + j;
+      if (c < cpr) {
+        const uint4 v = c0 == 0 ? cache[i] : src[c];
+        uint32_t out[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float lo = __uint_as_float(out[e] << 16) * mul;
+          const float hi = __uint_as_float(out[e] & 0xFFFF0000u) * mul;
+          __half2 h = __floats2half2_rn(lo, hi);
+          out[e] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        const int kin0 = c * 8;
+        uint8_t* blk = row + (kin0 >> 6) * 128;
+        const int in = kin0 & 63;
+        *reinterpret_cast<uint2*>(blk + perm64(in) * 2) = make_uint2(out[0], out[1]);
+        *reinterpret_cast<uint2*>(blk + perm64(in + 4) * 2) = make_uint2(out[2], out[3]);
       }
     }
-    uint8_t* row = xs + (size_t)m * p.row_stride + blk * 128;
-    *reinterpret_cast<uint2*>(row + perm64(in) * 2) = make_uint2(out[0], out[1]);
-    *reinterpret_cast<uint2*>(row + perm64(in + 4) * 2) = make_uint2(out[2], out[3]);
   }
   __syncthreads();
 }
 
 // c = A . B (fresh accumulator), fp32
-__device__ __forceinline__ void mma_bf16_first(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
-      : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
-}
-
 __device__ __forceinline__ void mma_f16_first(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
@@ -157,93 +207,59 @@ __device__ __forceinline__ void mma_f16_first(float* c, const uint32_t* a, uint3
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-// Streaming read-only loads of the packed weights (read once: no L1 allocation,
-// evict first from L2).
-__device__ __forceinline__ uint4 ldg_stream16(const uint8_t* p, uint64_t pol) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p), "l"(pol));
-  return v;
-}
+// The words a lane needs for one 128-group of one band.
+struct GroupWords {
+  uint4 w0, w1;   // the two 64-blocks
+  uint2 s0, s1;   // int4: s0.x = scales of rows g, g+8; NVFP4: per-block E4M3 scales
+};
 
-__device__ __forceinline__ uint2 ldg_stream8(const uint8_t* p, uint64_t pol) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p), "l"(pol));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t ldg_stream4(const uint8_t* p, uint64_t pol) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.u32 %0, [%1], %2;"
-               : "=r"(v)
-               : "l"(p), "l"(pol));
-  return v;
-}
-
-// One 128-group (two 64-blocks) of one band, int4.  w0/w1: this lane's words
-// of the two tiles; sp: BF16 scales of rows g and g+8.
+// One 128-group of one band, int4.  x0[mt]: this lane's activation fragment
+// of the group's first 64-block for 8-row tile mt (the second block follows
+// after xstep[mt] bytes).
 template <int MT>
-__device__ __forceinline__ void group_int4(uint4 w0, uint4 w1, uint32_t sp,
-                                           const uint8_t* const* xrow, const int* xstep, int kbl,
-                                           float (*acc)[4]) {
-  const float s_lo = __uint_as_float(sp << 16);          // row g
-  const float s_hi = __uint_as_float(sp & 0xFFFF0000u);  // row g + 8
-  float c[MT][4];
+__device__ __forceinline__ void group_int4(const GroupWords& gw, const uint8_t* const* x0,
+                                           const int* xstep, float (*acc)[4]) {
+  const float s_lo = __uint_as_float(gw.s0.x << 16);          // row g
+  const float s_hi = __uint_as_float(gw.s0.x & 0xFFFF0000u);  // row g + 8
+  float c[2][MT][4];
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    const uint4 wv = half ? w1 : w0;
+    const uint4 wv = half ? gw.w1 : gw.w0;
     const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
     uint32_t a[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      if (W4_GEMV_INT4_F16) {
-        // FP16 holds two nibbles per 16-bit half in its mantissa: one shift per word
-        const uint32_t hi = wd[j] >> 8;
-        a[j][0] = int4_lo_pair_to_f16x2(wd[j]);
-        a[j][1] = int4_hi_pair_to_f16x2(wd[j]);
-        a[j][2] = int4_lo_pair_to_f16x2(hi);
-        a[j][3] = int4_hi_pair_to_f16x2(hi);
-      } else {
-        a[j][0] = int4_pair_to_bf16x2(wd[j]);
-        a[j][1] = int4_pair_to_bf16x2(wd[j] >> 4);
-        a[j][2] = int4_pair_to_bf16x2(wd[j] >> 8);
-        a[j][3] = int4_pair_to_bf16x2(wd[j] >> 12);
-      }
+      // FP16 holds two nibbles per 16-bit half in its mantissa: one shift per word
+      const uint32_t hi = wd[j] >> 8;
+      a[j][0] = int4_lo_pair_to_f16x2(wd[j]);
+      a[j][1] = int4_hi_pair_to_f16x2(wd[j]);
+      a[j][2] = int4_lo_pair_to_f16x2(hi);
+      a[j][3] = int4_hi_pair_to_f16x2(hi);
     }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      const uint4* xb = reinterpret_cast<const uint4*>(xrow[mt] + (kbl + half) * xstep[mt]);
+      const uint4* xb = reinterpret_cast<const uint4*>(x0[mt] + half * xstep[mt]);
       const uint4 v0 = xb[0], v1 = xb[1];
       const uint32_t bx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      mma_f16_first(c[half][mt], a[0], bx[0], bx[1]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (W4_GEMV_INT4_F16) {
-          if (half == 0 && j == 0) mma_f16_first(c[mt], a[0], bx[0], bx[1]);
-          else mma_f16_16816(c[mt], a[j], bx[2 * j], bx[2 * j + 1]);
-        } else {
-          if (half == 0 && j == 0) mma_bf16_first(c[mt], a[0], bx[0], bx[1]);
-          else mma_bf16_16816(c[mt], a[j], bx[2 * j], bx[2 * j + 1]);
-        }
-      }
+      for (int j = 1; j < 4; ++j) mma_f16_16816(c[half][mt], a[j], bx[2 * j], bx[2 * j + 1]);
     }
   }
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
-    acc[mt][0] = fmaf(s_lo, c[mt][0], acc[mt][0]);
-    acc[mt][1] = fmaf(s_lo, c[mt][1], acc[mt][1]);
-    acc[mt][2] = fmaf(s_hi, c[mt][2], acc[mt][2]);
-    acc[mt][3] = fmaf(s_hi, c[mt][3], acc[mt][3]);
+    acc[mt][0] = fmaf(s_lo, c[0][mt][0] + c[1][mt][0], acc[mt][0]);
+    acc[mt][1] = fmaf(s_lo, c[0][mt][1] + c[1][mt][1], acc[mt][1]);
+    acc[mt][2] = fmaf(s_hi, c[0][mt][2] + c[1][mt][2], acc[mt][2]);
+    acc[mt][3] = fmaf(s_hi, c[0][mt][3] + c[1][mt][3], acc[mt][3]);
   }
 }
 
 // One 64-block of one band, NVFP4 (a scale per 16-group, i.e. per MMA).  wv:
 // this lane's words of the tile; sv: E4M3 scales of rows g and g+8, 4 groups.
 template <int MT>
-__device__ __forceinline__ void block_nvfp4(uint4 wv, uint2 sv, const uint8_t* const* xrow,
-                                            const int* xstep, int kbl, float (*acc)[4]) {
+__device__ __forceinline__ void block_nvfp4(uint4 wv, uint2 sv, const uint8_t* const* xb0,
+                                            float (*acc)[4]) {
   const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
   uint32_t a[4][4];
 #pragma unroll
@@ -262,7 +278,7 @@ __device__ __forceinline__ void block_nvfp4(uint4 wv, uint2 sv, const uint8_t* c
   }
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
-    const uint4* xb = reinterpret_cast<const uint4*>(xrow[mt] + kbl * xstep[mt]);
+    const uint4* xb = reinterpret_cast<const uint4*>(xb0[mt]);
     const uint4 v0 = xb[0], v1 = xb[1];
     const uint32_t bx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
@@ -290,11 +306,8 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
       for (int i = 0; i < 4; ++i) {
         const int m = mt * 8 + 2 * t + (i & 1);
         const int n = n0 + 8 * (i >> 1);
-        if (m < p.M && n < p.N) {
-          float v = vals[mt][i];
-          if (XF16<FMT>::value) v = v * row_mul[m] * gmul;
-          p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v);
-        }
+        if (m < p.M && n < p.N)
+          p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(vals[mt][i] * row_mul[m] * gmul);
       }
     return;
   }
@@ -305,11 +318,7 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
     for (int i = 0; i < 4; ++i) {
       const int m = mt * 8 + 2 * t + (i & 1);
       const int n = n0 + 8 * (i >> 1);
-      if (m < p.M) {
-        float v = vals[mt][i];
-        if (XF16<FMT>::value) v = v * row_mul[m];
-        __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v);
-      }
+      if (m < p.M) __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, vals[mt][i] * row_mul[m]);
     }
   __threadfence();
   __syncwarp();
@@ -333,82 +342,100 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
   if (lane == 0) p.counters[band] = 0u;
 }
 
-// The words a lane needs for one 128-group of one band.
-struct GroupWords {
-  uint4 w0, w1;   // the two 64-blocks
-  uint2 s0, s1;   // int4: s0.x = scales of rows g, g+8; NVFP4: per-block E4M3 scales
-};
 
-template <int FMT>
-__device__ __forceinline__ GroupWords load_group(const Params& p, int band, int kb, int lane,
-                                                 uint64_t pol) {
-  GroupWords gw;
-  const int g = lane >> 2;
-  const uint8_t* wt = p.w + ((size_t)band * (p.K >> 6) + kb) * kTileBytes + lane * 16;
-  gw.w0 = ldg_stream16(wt, pol);
-  gw.w1 = ldg_stream16(wt + kTileBytes, pol);
-  if (FMT == 0) {
-    gw.s0.x = ldg_stream4(p.s + ((size_t)band * (p.K >> 7) + (kb >> 1)) * 32 + g * 4, pol);
-    gw.s0.y = 0u;
-    gw.s1 = make_uint2(0u, 0u);
-  } else {
-    const uint8_t* st = p.s + ((size_t)band * (p.K >> 6) + kb) * 64 + g * 8;
-    gw.s0 = ldg_stream8(st, pol);
-    gw.s1 = ldg_stream8(st + 64, pol);
-  }
-  return gw;
-}
-
-template <int FMT, int MT>
-__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
+template <int FMT, int MT, int D>
+__global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(const Params p) {
+  using C = Cfg<FMT, MT>;
+  constexpr int kSB = stage_bytes(FMT);
+  constexpr int kSStep = FMT == 0 ? 32 : 128;  // scale bytes of one band per 128-group
   extern __shared__ __align__(128) uint8_t smem[];
   float* row_mul = reinterpret_cast<float*>(smem);
-  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kRowWords * 4);
+  unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kRowAuxOff);
   const uint8_t* zero = smem + kZeroOff;
   float* red = reinterpret_cast<float*>(smem + kRedOff);
-  uint8_t* xs = smem + kHeaderBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
+  const uint8_t* ring = smem + C::kHeader + warp * D * kSB;       // this warp's stages
+  uint8_t* xs = smem + C::kHeader + C::kWarps * D * kSB;          // activation image
+  if (threadIdx.x < kRowWords) row_aux[threadIdx.x] = 0u;
+  if (threadIdx.x < 32) reinterpret_cast<uint32_t*>(smem + kZeroOff)[threadIdx.x] = 0u;
+  pdl_launch_dependents();
+
+  // work of this CTA and warp (no divisions: the host passes quotients and
+  // powers of two)
   const int split = blockIdx.y;
   const int k_lo = split * p.kslice;
-  const int k_len = min(p.K - k_lo, p.kslice);
-  const int band_lo = (int)(((long long)blockIdx.x * p.NT) / p.ctas_x);
-  const int band_hi = (int)(((long long)(blockIdx.x + 1) * p.NT) / p.ctas_x);
-  const int nbands = band_hi - band_lo;
-
-  // warp grid: wi = band slot, wj = K piece of whole 128-groups
-  const int wi = warp % p.wn, wj = warp / p.wn;
-  const int groups = k_len >> 7;
-  const int g_lo = wj * groups / p.wk, g_hi = (wj + 1) * groups / p.wk;
-  const int ng = g_hi - g_lo;                  // 128-groups in this warp's piece
-  const int kb_base = (k_lo >> 6) + 2 * g_lo;  // first 64-block (global) of the piece
-  const int rounds = (nbands + p.wn - 1) / p.wn;
-  const int my_rounds = wi < nbands ? (nbands - wi + p.wn - 1) / p.wn : 0;
+  const int bx = blockIdx.x;
+  const int band_lo = bx * p.bq + min(bx, p.br);
+  const int nbands = p.bq + (bx < p.br ? 1 : 0);
+  const int wi = warp & (p.wn - 1), wj = warp >> p.wn_log2;
+  const int groups = min(p.K - k_lo, p.kslice) >> 7;
+  const int g_lo = (wj * groups) >> p.wk_log2, g_hi = ((wj + 1) * groups) >> p.wk_log2;
+  const int ng = g_hi - g_lo;                  // real 128-groups in this warp's piece
+  const int ngp = p.ngp;                       // padded piece length, a multiple of D
+  const int rounds = (nbands + p.wn - 1) >> p.wn_log2;
+  const int my_rounds = wi < nbands ? ((nbands - wi - 1) >> p.wn_log2) + 1 : 0;
+  const int KB = p.K >> 6;
+  const int gk0 = (k_lo >> 7) + g_lo;          // first global 128-group of the piece
   const uint64_t pol = policy_evict_first();
 
-  // the first loads go out before the activations are staged
-  GroupWords buf[kPD];
-  if (my_rounds > 0) {
-#pragma unroll
-    for (int u = 0; u < kPD; ++u)
-      if (u < ng) buf[u] = load_group<FMT>(p, band_lo + wi, kb_base + 2 * u, lane, pol);
-  }
+  // copy cursor over the warp's items (band pieces of ngp groups, round after
+  // round); the groups past the real piece only commit an empty copy group
+  const int b0 = min(band_lo + wi, p.NT - 1);
+  const uint8_t* cw = p.w + ((size_t)b0 * KB + 2 * gk0) * kTileBytes + lane * 16;
+  const uint8_t* cs = FMT == 0 ? p.s + ((size_t)b0 * (p.K >> 7) + gk0) * 32 + g * 4
+                               : p.s + ((size_t)b0 * KB + 2 * gk0) * 64 + g * 8;
+  // from the end of a padded piece to the next band's piece (< 2^31 bytes)
+  const int wjump = p.wn * KB * kTileBytes - ngp * kGroupBytes;
+  const int sjump = FMT == 0 ? p.wn * (p.K >> 7) * 32 - ngp * 32 : p.wn * KB * 64 - ngp * 128;
+  int c_left = my_rounds * ngp;
+  int c_gi = 0;
+  const uint32_t ring_s = smem_u32(ring) + lane * 16;
+  auto issue = [&](int slot) {
+    if (c_left > 0) {
+      if (c_gi < ng) {
+        const uint32_t d = ring_s + slot * kSB;
+        cpa16(d, cw, pol);
+        cpa16(d + kTileBytes, cw + kTileBytes, pol);
+        if (FMT == 0) {
+          cpa4(d + kGroupBytes - lane * 12, cs);   // scale slot: lane * 4
+        } else {
+          cpa8(d + kGroupBytes, cs);
+          cpa8(d + kGroupBytes + 8, cs + 64);
+        }
+      }
+      --c_left;
+      cw += kGroupBytes;
+      cs += kSStep;
+      if (++c_gi == ngp) {
+        c_gi = 0;
+        cw += wjump;
+        cs += sjump;
+      }
+    }
+    cpa_commit();
+  };
 
-  if (threadIdx.x < 32) reinterpret_cast<uint32_t*>(smem + kZeroOff)[threadIdx.x] = 0u;
-  stage_activations<FMT>(p, k_lo, k_len, xs, row_mul, row_aux);  // ends with __syncthreads
+  // the first copies go out before the activations are staged
+#pragma unroll
+  for (int u = 0; u < D - 1; ++u) issue(u);
+
+  pdl_wait();          // the activations may come from the previous kernel
+  __syncthreads();     // row_aux zeroed
+  stage_activations<C::kCache>(p, k_lo, groups * 128, xs, row_mul, row_aux);
 
   // activation rows of this lane (row m = 8 mt + g); rows past M read zeros
-  const uint8_t* xrow[MT];
+  const uint8_t* x0[MT];
   int xstep[MT];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int m = mt * 8 + g;
     const bool real = m < p.M;
-    xrow[mt] = real ? xs + (size_t)m * p.row_stride + t * 32 : zero;
     xstep[mt] = real ? 128 : 0;
+    x0[mt] = real ? xs + (size_t)m * p.row_stride + t * 32 + (2 * g_lo) * 128 : zero;
   }
-  const int kbl_base = 2 * g_lo;               // slice-local first 64-block of the piece
+  const uint8_t* slot0 = ring + lane * 16;
 
   for (int r = 0; r < rounds; ++r) {
     float acc[MT][4];
@@ -419,30 +446,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
     const bool active = r < my_rounds;
     const int band = band_lo + wi + r * p.wn;
     if (active) {
-      if (r > 0) {
+      for (int gi0 = 0; gi0 < ngp; gi0 += D) {
 #pragma unroll
-        for (int u = 0; u < kPD; ++u)
-          if (u < ng) buf[u] = load_group<FMT>(p, band, kb_base + 2 * u, lane, pol);
-      }
-      for (int gi0 = 0; gi0 < ng; gi0 += kPD) {
+        for (int k = 0; k < D; ++k) {
+          issue((k + D - 1) % D);     // the item D-1 ahead lands in the slot read last time
+          cpa_wait<D - 1>();          // this lane's bytes of item gi0 + k have landed
+          const int gi = gi0 + k;
+          if (gi >= ng) continue;     // padding: nothing was copied, nothing to add
+          const uint8_t* st = slot0 + k * kSB;
+          GroupWords cur;
+          cur.w0 = *reinterpret_cast<const uint4*>(st);
+          cur.w1 = *reinterpret_cast<const uint4*>(st + kTileBytes);
+          const uint8_t* xg[MT];
 #pragma unroll
-        for (int u = 0; u < kPD; ++u) {
-          const int gi = gi0 + u;
-          if (gi < ng) {
-            const GroupWords cur = buf[u];
-            if (gi + kPD < ng) buf[u] = load_group<FMT>(p, band, kb_base + 2 * (gi + kPD), lane, pol);
-            const int kbl = kbl_base + 2 * gi;
-            if (FMT == 0) {
-              group_int4<MT>(cur.w0, cur.w1, cur.s0.x, xrow, xstep, kbl, acc);
-            } else {
-              block_nvfp4<MT>(cur.w0, cur.s0, xrow, xstep, kbl, acc);
-              block_nvfp4<MT>(cur.w1, cur.s1, xrow, xstep, kbl + 1, acc);
-            }
+          for (int mt = 0; mt < MT; ++mt) xg[mt] = x0[mt] + gi * 2 * xstep[mt];
+          if (FMT == 0) {
+            cur.s0.x = *reinterpret_cast<const uint32_t*>(st + kGroupBytes - lane * 12);
+            group_int4<MT>(cur, xg, xstep, acc);
+          } else {
+            const uint4 sv = *reinterpret_cast<const uint4*>(st + kGroupBytes);
+            cur.s0 = make_uint2(sv.x, sv.y);
+            cur.s1 = make_uint2(sv.z, sv.w);
+            block_nvfp4<MT>(cur.w0, cur.s0, xg, acc);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) xg[mt] += xstep[mt];
+            block_nvfp4<MT>(cur.w1, cur.s1, xg, acc);
           }
         }
       }
     }
-    if (p.wk == 1) {
+    if (p.wk_log2 == 0) {
       if (active) band_epilogue<FMT, MT>(p, band, split, lane, row_mul, acc);
       continue;
     }
@@ -459,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) sum[mt][i] = 0.f;
-      for (int pc = 0; pc < p.wk; ++pc) {
+      for (int pc = 0; pc < (1 << p.wk_log2); ++pc) {
         const float* o = red + ((pc * p.wn + wi) * 32 + lane) * 4 * MT;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
@@ -470,6 +503,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params p) {
     }
     __syncthreads();
   }
+  cpa_wait<0>();  // nothing is in flight at exit
+}
+
+template <int FMT, int MT, int D>
+cudaError_t launch_d(const Params& p, const GemvPlan& pl, cudaStream_t st) {
+  // raise the dynamic shared memory limit once per device (kept out of the
+  // steady state so launches can be captured in CUDA graphs)
+  static bool smem_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!smem_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MT, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e != cudaSuccess) return e;
+    smem_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.ctas_x, pl.S);
+  cfg.blockDim = dim3(Cfg<FMT, MT>::kWarps * 32);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<FMT, MT, D>, p);
+}
+
+int ilog2(int v) {
+  int l = 0;
+  while ((1 << l) < v) ++l;
+  return l;
 }
 
 template <int FMT, int MT>
@@ -489,72 +556,88 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   p.NT = (a.N + 15) / 16;
   p.S = pl.S;
   p.kslice = pl.kslice;
-  p.ctas_x = pl.ctas_x;
+  p.bq = p.NT / pl.ctas_x;
+  p.br = p.NT % pl.ctas_x;
   p.row_stride = (pl.kslice / 64) * 128 + 16;
   p.wn = pl.wn;
-  p.wk = pl.wk;
-  // raise the dynamic shared memory limit once per device (kept out of the
-  // steady state so launches can be captured in CUDA graphs)
-  static int smem_set[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (smem_set[dev] < pl.smem) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-    if (e != cudaSuccess) return e;
-    smem_set[dev] = kMaxSmem;
+  p.wn_log2 = ilog2(pl.wn);
+  p.wk_log2 = ilog2(pl.wk);
+  p.ngp = pl.ngp;
+  switch (pl.depth) {
+    case 2: return launch_d<FMT, MT, 2>(p, pl, st);
+    case 3: return launch_d<FMT, MT, 3>(p, pl, st);
+    case 4: return launch_d<FMT, MT, 4>(p, pl, st);
+    case 5: return launch_d<FMT, MT, 5>(p, pl, st);
+    default: return launch_d<FMT, MT, 6>(p, pl, st);
   }
-  gemv_kernel<FMT, MT><<<dim3(pl.ctas_x, pl.S), kThreads, pl.smem, st>>>(p);
-  return cudaGetLastError();
+}
+
+int warps_of(int fmt, int mt) {
+  if (fmt == 0) return mt == 1 ? Cfg<0, 1>::kWarps : Cfg<0, 2>::kWarps;
+  return mt == 1 ? Cfg<1, 1>::kWarps : Cfg<1, 2>::kWarps;
+}
+
+int header_of(int fmt, int mt) {
+  if (fmt == 0) return mt == 1 ? Cfg<0, 1>::kHeader : Cfg<0, 2>::kHeader;
+  return mt == 1 ? Cfg<1, 1>::kHeader : Cfg<1, 2>::kHeader;
 }
 
 }  // namespace
 
-// Picks the K splits across CTAs (S) and the warp grid (wn bands x wk pieces)
-// that minimise the largest number of 64-blocks any warp streams, with small
-// penalties for cross-CTA split-K and per-round reductions.
+// Picks the K splits across CTAs (S), the warp grid (wn bands x wk pieces,
+// both powers of two) and the ring depth D.  Every warp's piece is padded to
+// a multiple of D groups (padding groups copy and add nothing) so that ring
+// slots stay compile-time constants across bands.  The cost is the largest
+// number of 64-blocks any warp processes (padding included), with small
+// penalties for cross-CTA split-K, per-round reductions and shallow rings;
+// the activation image and the rings must fit in shared memory together.
 GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
-  (void)fmt;
   GemvPlan pl;
   pl.mt = M <= 8 ? 1 : 2;
+  const int warps = warps_of(fmt, pl.mt);
+  const int header = header_of(fmt, pl.mt);
+  const int sb = stage_bytes(fmt);
   const int NT = (N + 15) / 16;
   const int groups = K / 128;
-  const int xbudget = kMaxSmem - kHeaderBytes;
-  const int max_groups = (xbudget / M - 16) / 256;
-  const int s_min = (groups + max_groups - 1) / max_groups;
   double best = 1e300;
-  pl.S = s_min;
-  pl.wk = 1;
-  for (int S = s_min; S <= groups && S <= 16; ++S) {
+  pl.S = 0;
+  for (int S = 1; S <= groups && S <= 32; ++S) {
     const int gslice = (groups + S - 1) / S;
     if ((S - 1) * gslice >= groups) continue;  // an empty split
+    const int ximg = M * (gslice * 256 + 16);
+    const int dmax = min(kMaxDepth, (kMaxSmem - header - ximg) / (warps * sb));
+    if (dmax < 2) continue;
     int ctas = num_sms / S;
     if (ctas < 1) ctas = 1;
     if (ctas > NT) ctas = NT;
     const int bands_max = (NT + ctas - 1) / ctas;
-    for (int wk = 1; wk <= kWarps; wk *= 2) {
+    for (int wk = 1; wk <= warps; wk *= 2) {
       if (wk > gslice) break;
-      if (kWarps % wk != 0) continue;
-      const int wn = kWarps / wk;
+      const int wn = warps / wk;
       const int rounds = (bands_max + wn - 1) / wn;
-      const int piece = 2 * ((gslice + wk - 1) / wk);
-      double cost = (double)rounds * (piece + (wk > 1 ? 2.0 : 0.5)) + (S > 1 ? 3.0 : 0.0);
-      if (cost < best - 1e-9) {
-        best = cost;
-        pl.S = S;
-        pl.wk = wk;
+      const int piece = (gslice + wk - 1) / wk;
+      for (int d = 2; d <= dmax; ++d) {
+        const int padded = (piece + d - 1) / d * d;
+        const double cost = (double)rounds * (2.0 * padded + (wk > 1 ? 2.0 : 0.5)) +
+                            (S > 1 ? 3.0 : 0.0) + (d < 4 ? 1.5 * (4 - d) : 0.0);
+        if (cost < best - 1e-9) {
+          best = cost;
+          pl.S = S;
+          pl.wk = wk;
+          pl.depth = d;
+          pl.ngp = padded;
+        }
       }
     }
   }
-  pl.wn = kWarps / pl.wk;
+  pl.wn = warps / pl.wk;
   const int gslice = (groups + pl.S - 1) / pl.S;
   pl.kslice = gslice * 128;
   int ctas = num_sms / pl.S;
   if (ctas < 1) ctas = 1;
   if (ctas > NT) ctas = NT;
   pl.ctas_x = ctas;
-  pl.smem = kHeaderBytes + M * ((pl.kslice / 64) * 128 + 16);
+  pl.smem = header + warps * pl.depth * sb + M * ((pl.kslice / 64) * 128 + 16);
   return pl;
 }
 

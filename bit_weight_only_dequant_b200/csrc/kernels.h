@@ -27,6 +27,8 @@ struct GemvPlan {
   int ctas_x;    // CTAs per split
   int mt;        // 8-row activation tiles (1: M <= 8, 2: M <= 16)
   int wn, wk;    // warps per CTA as (bands in flight) x (K pieces per band)
+  int depth;     // shared-memory ring stages (128-groups in flight) per warp
+  int ngp;       // 128-groups per warp piece, padded to a multiple of depth
   int smem;      // dynamic shared memory bytes
 };
 
