@@ -213,12 +213,12 @@ struct GroupWords {
   uint2 s0, s1;   // int4: s0.x = scales of rows g, g+8; NVFP4: per-block E4M3 scales
 };
 
-// One 128-group of one band, int4.  x0[mt]: this lane's activation fragment
+// One 128-group of one band, int4.  xg[mt]: this lane's activation fragment
 // of the group's first 64-block for 8-row tile mt (the second block follows
-// after xstep[mt] bytes).
+// 128 bytes later).
 template <int MT>
-__device__ __forceinline__ void group_int4(const GroupWords& gw, const uint8_t* const* x0,
-                                           const int* xstep, float (*acc)[4]) {
+__device__ __forceinline__ void group_int4(const GroupWords& gw, const uint8_t* const* xg,
+                                           float (*acc)[4]) {
   const float s_lo = __uint_as_float(gw.s0.x << 16);          // row g
   const float s_hi = __uint_as_float(gw.s0.x & 0xFFFF0000u);  // row g + 8
   float c[2][MT][4];
@@ -238,7 +238,7 @@ __device__ __forceinline__ void group_int4(const GroupWords& gw, const uint8_t* 
     }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      const uint4* xb = reinterpret_cast<const uint4*>(x0[mt] + half * xstep[mt]);
+      const uint4* xb = reinterpret_cast<const uint4*>(xg[mt] + half * 128);
       const uint4 v0 = xb[0], v1 = xb[1];
       const uint32_t bx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
       mma_f16_first(c[half][mt], a[0], bx[0], bx[1]);
@@ -351,7 +351,6 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
   extern __shared__ __align__(128) uint8_t smem[];
   float* row_mul = reinterpret_cast<float*>(smem);
   unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kRowAuxOff);
-  const uint8_t* zero = smem + kZeroOff;
   float* red = reinterpret_cast<float*>(smem + kRedOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -380,60 +379,66 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
   const int gk0 = (k_lo >> 7) + g_lo;          // first global 128-group of the piece
   const uint64_t pol = policy_evict_first();
 
-  // copy cursor over the warp's items (band pieces of ngp groups, round after
-  // round); the groups past the real piece only commit an empty copy group
+  // Copies run one block of D groups ahead of the reads: the groups of block
+  // b + 1 refill the slots of block b as those are read.  A block never spans
+  // two bands (pieces are padded to whole blocks), so its groups sit at fixed
+  // offsets from one pointer; padding groups copy nothing.
   const int b0 = min(band_lo + wi, p.NT - 1);
   const uint8_t* cw = p.w + ((size_t)b0 * KB + 2 * gk0) * kTileBytes + lane * 16;
   const uint8_t* cs = FMT == 0 ? p.s + ((size_t)b0 * (p.K >> 7) + gk0) * 32 + g * 4
                                : p.s + ((size_t)b0 * KB + 2 * gk0) * 64 + g * 8;
-  // from the end of a padded piece to the next band's piece (< 2^31 bytes)
-  const int wjump = p.wn * KB * kTileBytes - ngp * kGroupBytes;
-  const int sjump = FMT == 0 ? p.wn * (p.K >> 7) * 32 - ngp * 32 : p.wn * KB * 64 - ngp * 128;
-  int c_left = my_rounds * ngp;
-  int c_gi = 0;
+  // from the last block of a piece to the first block of the next band's piece
+  const int wjump = p.wn * KB * kTileBytes - (ngp - D) * kGroupBytes;
+  const int sjump = FMT == 0 ? p.wn * (p.K >> 7) * 32 - (ngp - D) * 32
+                             : p.wn * KB * 64 - (ngp - D) * 128;
+  const int nbp = ngp / D;                     // blocks per piece
+  int c_blocks = my_rounds * nbp;              // blocks still to copy
+  int c_bb = 0;                                // block index of the cursor within its piece
   const uint32_t ring_s = smem_u32(ring) + lane * 16;
-  auto issue = [&](int slot) {
-    if (c_left > 0) {
-      if (c_gi < ng) {
-        const uint32_t d = ring_s + slot * kSB;
-        cpa16(d, cw, pol);
-        cpa16(d + kTileBytes, cw + kTileBytes, pol);
-        if (FMT == 0) {
-          cpa4(d + kGroupBytes - lane * 12, cs);   // scale slot: lane * 4
-        } else {
-          cpa8(d + kGroupBytes, cs);
-          cpa8(d + kGroupBytes + 8, cs + 64);
-        }
-      }
-      --c_left;
-      cw += kGroupBytes;
-      cs += kSStep;
-      if (++c_gi == ngp) {
-        c_gi = 0;
-        cw += wjump;
-        cs += sjump;
+  auto copy_item = [&](int k) {                // group k of the cursor block -> slot k
+    if (c_blocks > 0 && c_bb * D + k < ng) {
+      const uint32_t d = ring_s + k * kSB;
+      cpa16(d, cw + k * kGroupBytes, pol);
+      cpa16(d + kTileBytes, cw + k * kGroupBytes + kTileBytes, pol);
+      if (FMT == 0) {
+        cpa4(d + kGroupBytes - lane * 12, cs + k * kSStep);   // scale slot: lane * 4
+      } else {
+        cpa8(d + kGroupBytes, cs + k * kSStep);
+        cpa8(d + kGroupBytes + 8, cs + k * kSStep + 64);
       }
     }
     cpa_commit();
   };
+  auto next_block = [&]() {
+    if (c_blocks > 0) {
+      --c_blocks;
+      if (++c_bb == nbp) {
+        c_bb = 0;
+        cw += wjump;
+        cs += sjump;
+      } else {
+        cw += D * kGroupBytes;
+        cs += D * kSStep;
+      }
+    }
+  };
 
-  // the first copies go out before the activations are staged
+  // the first block goes out before the activations are staged
 #pragma unroll
-  for (int u = 0; u < D - 1; ++u) issue(u);
+  for (int k = 0; k < D; ++k) copy_item(k);
+  next_block();
 
   pdl_wait();          // the activations may come from the previous kernel
   __syncthreads();     // row_aux zeroed
   stage_activations<C::kCache>(p, k_lo, groups * 128, xs, row_mul, row_aux);
 
-  // activation rows of this lane (row m = 8 mt + g); rows past M read zeros
+  // activation rows of this lane (row m = 8 mt + g); rows past M alias row 0:
+  // their MMA columns are computed but never stored
   const uint8_t* x0[MT];
-  int xstep[MT];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int m = mt * 8 + g;
-    const bool real = m < p.M;
-    xstep[mt] = real ? 128 : 0;
-    x0[mt] = real ? xs + (size_t)m * p.row_stride + t * 32 + (2 * g_lo) * 128 : zero;
+    x0[mt] = xs + (size_t)(m < p.M ? m : 0) * p.row_stride + t * 32 + (2 * g_lo) * 128;
   }
   const uint8_t* slot0 = ring + lane * 16;
 
@@ -446,33 +451,37 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
     const bool active = r < my_rounds;
     const int band = band_lo + wi + r * p.wn;
     if (active) {
-      for (int gi0 = 0; gi0 < ngp; gi0 += D) {
+      for (int bb = 0; bb < nbp; ++bb) {
+        const uint8_t* xb[MT];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) xb[mt] = x0[mt] + bb * D * 256;
 #pragma unroll
         for (int k = 0; k < D; ++k) {
-          issue((k + D - 1) % D);     // the item D-1 ahead lands in the slot read last time
-          cpa_wait<D - 1>();          // this lane's bytes of item gi0 + k have landed
-          const int gi = gi0 + k;
-          if (gi >= ng) continue;     // padding: nothing was copied, nothing to add
-          const uint8_t* st = slot0 + k * kSB;
-          GroupWords cur;
-          cur.w0 = *reinterpret_cast<const uint4*>(st);
-          cur.w1 = *reinterpret_cast<const uint4*>(st + kTileBytes);
-          const uint8_t* xg[MT];
+          cpa_wait<D - 1>();          // this lane's bytes of group bb * D + k have landed
+          if (bb * D + k < ng) {      // else padding: nothing was copied, nothing to add
+            const uint8_t* st = slot0 + k * kSB;
+            GroupWords cur;
+            cur.w0 = *reinterpret_cast<const uint4*>(st);
+            cur.w1 = *reinterpret_cast<const uint4*>(st + kTileBytes);
+            const uint8_t* xg[MT];
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) xg[mt] = x0[mt] + gi * 2 * xstep[mt];
-          if (FMT == 0) {
-            cur.s0.x = *reinterpret_cast<const uint32_t*>(st + kGroupBytes - lane * 12);
-            group_int4<MT>(cur, xg, xstep, acc);
-          } else {
-            const uint4 sv = *reinterpret_cast<const uint4*>(st + kGroupBytes);
-            cur.s0 = make_uint2(sv.x, sv.y);
-            cur.s1 = make_uint2(sv.z, sv.w);
-            block_nvfp4<MT>(cur.w0, cur.s0, xg, acc);
+            for (int mt = 0; mt < MT; ++mt) xg[mt] = xb[mt] + k * 256;
+            if (FMT == 0) {
+              cur.s0.x = *reinterpret_cast<const uint32_t*>(st + kGroupBytes - lane * 12);
+              group_int4<MT>(cur, xg, acc);
+            } else {
+              const uint4 sv = *reinterpret_cast<const uint4*>(st + kGroupBytes);
+              cur.s0 = make_uint2(sv.x, sv.y);
+              cur.s1 = make_uint2(sv.z, sv.w);
+              block_nvfp4<MT>(cur.w0, cur.s0, xg, acc);
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) xg[mt] += xstep[mt];
-            block_nvfp4<MT>(cur.w1, cur.s1, xg, acc);
+              for (int mt = 0; mt < MT; ++mt) xg[mt] += 128;
+              block_nvfp4<MT>(cur.w1, cur.s1, xg, acc);
+            }
           }
+          copy_item(k);               // refill the slot just read
         }
+        next_block();
       }
     }
     if (p.wk_log2 == 0) {
