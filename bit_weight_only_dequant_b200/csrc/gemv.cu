@@ -423,14 +423,19 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
     }
   };
 
-  // the first block goes out before the activations are staged
+  // The first groups go out before the activations are staged, the rest of
+  // the first block right after: a full block of copies queued ahead of the
+  // activation loads delays them behind the weights (measured).
+  constexpr int kPre = D < 2 ? D : 2;
 #pragma unroll
-  for (int k = 0; k < D; ++k) copy_item(k);
-  next_block();
+  for (int k = 0; k < kPre; ++k) copy_item(k);
 
   pdl_wait();          // the activations may come from the previous kernel
   __syncthreads();     // row_aux zeroed
   stage_activations<C::kCache>(p, k_lo, groups * 128, xs, row_mul, row_aux);
+#pragma unroll
+  for (int k = kPre; k < D; ++k) copy_item(k);
+  next_block();
 
   // activation rows of this lane (row m = 8 mt + g); rows past M alias row 0:
   // their MMA columns are computed but never stored

@@ -6,27 +6,29 @@
 // a bandwidth-bound step into a slightly compute-bound one: blog post "One
 // Config Line Made My 27B Model 2.7x Faster", section "The fix").
 //
-// Structure (one persistent CTA per SM, 18 warps, 256-row x M tiles):
-//  * warp 16 (producer): per stage of four 64-k blocks, lane b < 16 copies
-//    band b's 2 KB of packed weights and its scales with 1-D bulk copies, and
-//    lanes 16..19 load the four SWIZZLE_128B activation boxes with 2-D TMA
-//    (rows past M zero-filled) into a 3-4 stage shared-memory ring.
-//  * warps 0-15 (dequant, then epilogue): one 16-row band each; every lane
-//    turns its 16 packed bytes per block into 32 scaled operands in registers
-//    (int4: q -> BF16 times the BF16 group scale with one rounding, exactly
-//    W_deq; NVFP4: e2m1 -> FP16 times the E4M3 scale, exact) and writes them
-//    straight into a tensor-memory A slot with tcgen05.st 16x256b, whose
-//    register layout matches the packed pairs.  Shared memory never holds
-//    dequantised weights.
+// Structure (one persistent CTA per SM, 18 warps, 256-row x M tiles; the
+// unit of work is one 128-group of K, i.e. one group scale):
+//  * warps 0-15 (dequant, then epilogue): one 16-row band each.  Every warp
+//    streams its band's packed weights and scales through its own ring of
+//    shared-memory stages with cp.async (each lane copies and reads back only
+//    its own bytes, as in the GEMV), turns its 32 bytes per group into 64
+//    scaled operands in registers (int4: q -> BF16 times the BF16 group scale
+//    with one rounding, exactly W_deq; NVFP4: e2m1 -> FP16 times the E4M3
+//    scale, exact) and writes them straight into a tensor-memory A slot with
+//    tcgen05.st 16x256b, whose register layout matches the packed pairs.
+//    Shared memory never holds dequantised weights.
+//  * warp 16 (producer): lane 0 loads the two SWIZZLE_128B activation boxes
+//    of each group with 2-D TMA (rows past M zero-filled) into a ring.
 //  * warp 17 (MMA): tcgen05.mma kind::f16, A (weights, 128 rows) from tensor
 //    memory, B (activations, K-major SW128) from shared memory, fp32 D
-//    (128 lanes x Mpad columns) per 128-row half; issued by one elected lane
-//    of a converged warp.
+//    (128 lanes x Mpad columns) per 128-row half; 16 MMAs per group, issued
+//    by one elected lane of a converged warp.
 //  * epilogue: tcgen05.ld of D, BF16 stores (or fp32 split-K partials reduced
 //    in split order by the last CTA of the tile).
-// Tensor memory: D at columns [0, 128), six A slots of 2 x 32 columns at
-// [128, 512).  Every mbarrier wait is bounded; a timeout raises the device
-// error word, the CTA drains its copies and MMAs and frees tensor memory.
+// Tensor memory: D at columns [0, 128), three A slots of one group (2 halves
+// x 64 columns) at [128, 512).  Every mbarrier wait is bounded; a timeout
+// raises the device error word, the CTA drains its copies and MMAs and frees
+// tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,15 +44,17 @@ constexpr int kTcThreads = (kDeqWarps + 2) * 32;
 constexpr int kProducerWarp = kDeqWarps;
 constexpr int kMmaWarp = kDeqWarps + 1;
 constexpr int kTcTileRows = 256;              // 16 bands, two 128-row MMA tiles
-constexpr int kKS = 4;                        // 64-blocks per shared-memory stage
-constexpr int kMaxStages = 4;
-constexpr int kWStage = 16 * kKS * kTileBytes;  // 32 KB: 2 KB contiguous per band
-constexpr int kSStage = 16 * kKS * 64;          // scales (NVFP4 size; INT4 uses 32 per group)
-constexpr int kSmemBudget = 220 * 1024;
-constexpr int kASlots = 6;                    // tensor-memory A slots of one 64-block each
+constexpr int kWRing = 4;                     // weight stages (groups) per dequant warp
+constexpr int kXRing = 4;                     // activation stages (groups)
+constexpr int kASlots = 3;                    // tensor-memory A slots of one group each
 constexpr int kTmemCols = 512;
 constexpr int kAColBase = 128;
+constexpr int kGroupBytesW = 2 * kTileBytes;  // one band's packed weights per 128-group
 constexpr int kMinSmem = 120 * 1024;          // keeps one CTA (and one TMEM owner) per SM
+
+// Weight ring stage: the group's two tiles (each lane's 16 bytes at 16 lane),
+// then the scales each lane needs (int4: 4 bytes at 4 lane; NVFP4: 2 x 8 at 16 lane).
+__host__ __device__ constexpr int tc_stage_bytes(int fmt) { return kGroupBytesW + (fmt == 0 ? 128 : 512); }
 
 struct TcParams {
   const uint8_t* w;
@@ -61,7 +65,7 @@ struct TcParams {
   float* ws;
   unsigned* counters;
   unsigned* err;
-  int M, N, K, KB, NT, tiles, S, kbs, units;
+  int M, N, K, KB, NT, tiles, S, gps, units;   // gps: 128-groups per split
 };
 
 // ------------------------------------------------------------------ tcgen05 wrappers
@@ -202,32 +206,57 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t phase, volatil
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+
 template <int FMT, int MPAD>
 struct TcShape {
-  static constexpr int kBBlock = MPAD * 128;                 // one 64-k activation box
-  static constexpr int kBStage = kKS * kBBlock;
-  static constexpr int kStageBytes = kBStage + kWStage + kSStage;
-  static constexpr int kStages = (kSmemBudget / kStageBytes) < kMaxStages
-                                     ? (kSmemBudget / kStageBytes) : kMaxStages;
-  static constexpr int kSmem = kStages * kStageBytes + 1024 /* barriers */ + 1024 /* align */;
+  static constexpr int kXStage = 2 * MPAD * 128;             // two 64-k activation boxes
+  static constexpr int kWRingBytes = kDeqWarps * kWRing * tc_stage_bytes(FMT);
+  static constexpr int kSmemUse = kXRing * kXStage + kWRingBytes + 1024 /* barriers */;
+  static constexpr int kSmem = (kSmemUse + 1024 /* align */ > kMinSmem) ? kSmemUse + 1024 : kMinSmem;
 };
+
+__device__ __forceinline__ void cpa16(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void cpa8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cpa_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The K range of a unit (tile, split) in 128-groups.
+__device__ __forceinline__ void unit_range(const TcParams& p, int unit, int& tile, int& split,
+                                           int& g_lo, int& g_hi) {
+  tile = unit / p.S;
+  split = unit - tile * p.S;
+  const int G = p.K >> 7;
+  g_lo = split * p.gps;
+  g_hi = min(G, g_lo + p.gps);
+}
 
 template <int FMT, int MPAD>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap xmap, const TcParams p) {
   using Sh = TcShape<FMT, MPAD>;
-  constexpr int NS = Sh::kStages;
+  constexpr int kSB = tc_stage_bytes(FMT);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* Bs = smem;                                   // NS x kKS x (MPAD x 128 B), SW128
-  uint8_t* Ws = Bs + NS * Sh::kBStage;                  // NS x 16 bands x kKS x 512 B
-  uint8_t* Ss = Ws + NS * kWStage;                      // NS x 16 bands x 256 B
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Ss + NS * kSStage);
-  uint64_t* full = bars;                                // NS
-  uint64_t* sfree = bars + NS;                          // NS
-  uint64_t* afull = bars + 2 * NS;                      // kASlots
-  uint64_t* afree = afull + kASlots;                    // kASlots
+  uint8_t* Xs = smem;                                    // kXRing x (2 boxes of MPAD x 128 B), SW128
+  uint8_t* Wr = Xs + kXRing * Sh::kXStage;               // dequant warps' weight rings
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Wr + Sh::kWRingBytes);
+  uint64_t* xfull = bars;                                // kXRing
+  uint64_t* xfree = bars + kXRing;                       // kXRing
+  uint64_t* afull = bars + 2 * kXRing;                   // kASlots
+  uint64_t* afree = afull + kASlots;                     // kASlots
   uint64_t* dfull = afree + kASlots;
   uint64_t* dfree = dfull + 1;
   uint64_t* drain = dfull + 2;
@@ -238,9 +267,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(full + i, 1);
-      mbar_init(sfree + i, kDeqWarps + 1);
+    for (int i = 0; i < kXRing; ++i) {
+      mbar_init(xfull + i, 1);
+      mbar_init(xfree + i, 1);
     }
     for (int i = 0; i < kASlots; ++i) {
       mbar_init(afull + i, kDeqWarps);
@@ -262,95 +291,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t sbytes_blk = FMT == 0 ? 16u : 64u;     // scale bytes per band per 64-block
 
   if (warp == kProducerWarp) {
-    // ---------------------------------------------------------------- producer (whole warp)
-    int last_use[kMaxStages];
-#pragma unroll
-    for (int i = 0; i < kMaxStages; ++i) last_use[i] = -1;
-    uint32_t st_it = 0;
+    // ---------------------------------------------------------------- activations (lane 0)
+    uint32_t it = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
-      const int tile = unit / p.S, split = unit - tile * p.S;
-      const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
-      const int nb0 = tile * 16;
-      const int nvalid = min(16, p.NT - nb0);
-      for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += kKS, ++st_it) {
-        const int s = st_it % NS;
-        const uint32_t u = st_it / NS;
-        const int nblk = min(kKS, kb_hi - kb0);
-        if (u > 0 && !warp_wait(sfree + s, (u - 1) & 1, abort_flag, p.err)) {
-          ok = false;
-          break;
+    if (lane == 0) {
+      for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
+        int tile, split, g_lo, g_hi;
+        unit_range(p, unit, tile, split, g_lo, g_hi);
+        for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
+          const int s = it % kXRing;
+          const uint32_t u = it / kXRing;
+          if (u > 0 && !tc_wait(xfree + s, (u - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(xfull + s, Sh::kXStage);
+          uint8_t* dst = Xs + s * Sh::kXStage;
+          tma_load_2d(dst, &xmap, gi * 128, 0, xfull + s);
+          tma_load_2d(dst + MPAD * 128, &xmap, gi * 128 + 64, 0, xfull + s);
         }
-        if (lane == 0)
-          mbar_arrive_expect_tx(full + s, nblk * Sh::kBBlock +
-                                              nvalid * nblk * (kTileBytes + sbytes_blk));
-        __syncwarp();
-        if (lane < nvalid) {
-          const size_t nb = (size_t)(nb0 + lane);
-          bulk_g2s(Ws + s * kWStage + lane * (kKS * kTileBytes), p.w + (nb * p.KB + kb0) * kTileBytes,
-                   nblk * kTileBytes, full + s);
-          const uint8_t* ssrc = FMT == 0 ? p.s + (nb * (p.K >> 7) + (kb0 >> 1)) * 32
-                                         : p.s + (nb * p.KB + kb0) * 64;
-          bulk_g2s(Ss + s * kSStage + lane * (kKS * 64), ssrc, nblk * sbytes_blk, full + s);
-        } else if (lane >= 16 && lane < 16 + nblk) {
-          const int j = lane - 16;
-          tma_load_2d(Bs + s * Sh::kBStage + j * Sh::kBBlock, &xmap, (kb0 + j) * 64, 0, full + s);
-        }
-        last_use[s] = (int)u;
       }
+      // drain: every issued copy has landed before the CTA may exit
+      const uint32_t issued = it;
+      for (uint32_t k = issued > kXRing ? issued - kXRing : 0; k < issued; ++k)
+        mbar_wait(xfull + k % kXRing, (k / kXRing) & 1, p.err);
     }
-    // drain: every issued copy has landed before the CTA may exit
-    if (lane == 0)
-      for (int s = 0; s < NS; ++s)
-        if (last_use[s] >= 0) mbar_wait(full + s, last_use[s] & 1, p.err);
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer (whole warp)
     constexpr uint32_t idesc = make_idesc(FMT == 0 ? 1 : 0, MPAD);
-    uint32_t st_it = 0, ab = 0, unit_i = 0;
+    uint32_t it = 0, unit_i = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
-      const int tile = unit / p.S, split = unit - tile * p.S;
-      const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
+      int tile, split, g_lo, g_hi;
+      unit_range(p, unit, tile, split, g_lo, g_hi);
       (void)tile;
       if (unit_i > 0) {
         if (!warp_wait(dfree, (unit_i - 1) & 1, abort_flag, p.err)) break;
         tc_fence_after();
       }
-      for (int kb0 = kb_lo; kb0 < kb_hi && ok; kb0 += kKS, ++st_it) {
-        const int s = st_it % NS;
-        const uint32_t u = st_it / NS;
-        const int nblk = min(kKS, kb_hi - kb0);
-        if (!warp_wait(full + s, u & 1, abort_flag, p.err)) {
+      for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
+        const int xs_ = it % kXRing, sl = it % kASlots;
+        if (!warp_wait(xfull + xs_, (it / kXRing) & 1, abort_flag, p.err) ||
+            !warp_wait(afull + sl, (it / kASlots) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
-        const uint64_t dbase = sw128_desc(smem_u32(Bs + s * Sh::kBStage));
-        for (int j = 0; j < nblk; ++j, ++ab) {
-          const int slot = ab % kASlots;
-          if (!warp_wait(afull + slot, (ab / kASlots) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t bj = dbase + (uint64_t)((j * Sh::kBBlock) >> 4);
-          const uint32_t a0 = tmem + kAColBase + slot * 64;
-          if (elect_one()) {
+        tc_fence_after();
+        const uint64_t b0 = sw128_desc(smem_u32(Xs + xs_ * Sh::kXStage));
+        const uint32_t a0 = tmem + kAColBase + sl * 128;
+        if (elect_one()) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < 2; ++h)
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                umma_ts(tmem + h * 64, a0 + h * 32 + k * 8, bj + (uint64_t)(k * 2), idesc,
-                        (kb0 + j > kb_lo || k > 0) ? 1u : 0u);
-            umma_commit(afree + slot);
-          }
-          __syncwarp();
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ts(tmem + h * 64, a0 + h * 64 + kk * 8,
+                      b0 + (uint64_t)(((kk >> 2) * MPAD * 128) >> 4) + (uint64_t)((kk & 3) * 2),
+                      idesc, (gi > g_lo || kk > 0) ? 1u : 0u);
+          umma_commit(afree + sl);
+          umma_commit(xfree + xs_);
         }
-        if (!ok) break;
-        if (elect_one()) umma_commit(sfree + s);
         __syncwarp();
       }
       if (ok) {
@@ -370,36 +372,94 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int band = h * 8 + 2 * q + bp;                // 16-row band of the 256-row tile
     const int g = lane >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q + 16 * bp) << 16;
-    uint32_t st_it = 0, ab = 0, unit_i = 0;
+    const uint64_t pol = policy_evict_first();
+    const int G = p.K >> 7;
+    constexpr int kSStep = FMT == 0 ? 32 : 128;          // one band's scale bytes per group
+
+    // copy cursor over this warp's groups: (unit, group) in the CTA's order
+    uint8_t* ring = Wr + warp * kWRing * kSB;
+    const uint32_t ring_s = smem_u32(ring) + lane * 16;
+    int c_unit = blockIdx.x, c_gi = 0, c_hi = 0, c_nb = 0;
+    const uint8_t* cw = nullptr;
+    const uint8_t* cs = nullptr;
+    auto c_start = [&]() {
+      if (c_unit < p.units) {
+        int tile, split, g_lo;
+        unit_range(p, c_unit, tile, split, g_lo, c_hi);
+        c_gi = g_lo;
+        c_nb = tile * 16 + band;
+        const int nb = min(c_nb, p.NT - 1);
+        cw = p.w + ((size_t)nb * p.KB + 2 * g_lo) * kTileBytes + lane * 16;
+        cs = FMT == 0 ? p.s + ((size_t)nb * G + g_lo) * 32 + g * 4
+                      : p.s + ((size_t)nb * p.KB + 2 * g_lo) * 64 + g * 8;
+      }
+    };
+    c_start();
+    uint32_t c_it = 0;
+    auto copy_next = [&]() {                            // one group -> stage c_it % kWRing
+      if (c_unit < p.units) {
+        if (c_nb < p.NT) {
+          const uint32_t d = ring_s + (c_it % kWRing) * kSB;
+          cpa16(d, cw, pol);
+          cpa16(d + kTileBytes, cw + kTileBytes, pol);
+          if (FMT == 0) {
+            cpa4(d + kGroupBytesW - lane * 12, cs);       // scale slot: lane * 4
+          } else {
+            cpa8(d + kGroupBytesW, cs);
+            cpa8(d + kGroupBytesW + 8, cs + 64);
+          }
+        }
+        cw += kGroupBytesW;
+        cs += kSStep;
+        if (++c_gi == c_hi) {
+          c_unit += gridDim.x;
+          c_start();
+        }
+      }
+      cpa_commit();
+      ++c_it;
+    };
+#pragma unroll
+    for (int k = 0; k < kWRing; ++k) copy_next();
+
+    uint32_t it = 0, unit_i = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
-      const int tile = unit / p.S, split = unit - tile * p.S;
-      const int kb_lo = split * p.kbs, kb_hi = min(p.KB, kb_lo + p.kbs);
-      for (int kb0 = kb_lo; kb0 < kb_hi && ok; kb0 += kKS, ++st_it) {
-        const int s = st_it % NS;
-        const uint32_t u = st_it / NS;
-        const int nblk = min(kKS, kb_hi - kb0);
-        if (!warp_wait(full + s, u & 1, abort_flag, p.err)) {
+      int tile, split, g_lo, g_hi;
+      unit_range(p, unit, tile, split, g_lo, g_hi);
+      const bool real_band = tile * 16 + band < p.NT;
+      for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
+        const int sl = it % kASlots;
+        const uint32_t ua = it / kASlots;
+        cpa_wait<kWRing - 1>();                          // this lane's bytes of group `it`
+        const uint8_t* st = ring + (it % kWRing) * kSB;
+        uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+        uint32_t sv0 = 0, sv1 = 0, sv2 = 0, sv3 = 0;
+        if (real_band) {
+          w0 = *reinterpret_cast<const uint4*>(st + lane * 16);
+          w1 = *reinterpret_cast<const uint4*>(st + kTileBytes + lane * 16);
+          if (FMT == 0) {
+            sv0 = *reinterpret_cast<const uint32_t*>(st + kGroupBytesW + lane * 4);
+          } else {
+            const uint4 sv = *reinterpret_cast<const uint4*>(st + kGroupBytesW + lane * 16);
+            sv0 = sv.x; sv1 = sv.y; sv2 = sv.z; sv3 = sv.w;
+          }
+        }
+        __syncwarp();
+        copy_next();                                     // refill the stage just read
+        if (ua > 0 && !warp_wait(afree + sl, (ua - 1) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
-        const uint8_t* wsrc = Ws + s * kWStage + band * (kKS * kTileBytes) + lane * 16;
-        const uint8_t* ssrc = Ss + s * kSStage + band * (kKS * 64);
-        for (int j = 0; j < nblk; ++j, ++ab) {
-          const int slot = ab % kASlots;
-          const uint32_t ua = ab / kASlots;
-          if (ua > 0 && !warp_wait(afree + slot, (ua - 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint4 wv = *reinterpret_cast<const uint4*>(wsrc + j * kTileBytes);
+        tc_fence_after();
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          const uint4 wv = blk ? w1 : w0;
           const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
           uint32_t r[16];
           if (FMT == 0) {
-            const uint32_t sp = *reinterpret_cast<const uint32_t*>(ssrc + (j >> 1) * 32 + g * 4);
-            const uint32_t s_lo = prmt(sp, sp, 0x1010u);  // (s_g, s_g)
-            const uint32_t s_hi = prmt(sp, sp, 0x3232u);  // (s_g8, s_g8)
+            const uint32_t s_lo = prmt(sv0, sv0, 0x1010u);  // (s_g, s_g)
+            const uint32_t s_hi = prmt(sv0, sv0, 0x3232u);  // (s_g8, s_g8)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               // register order of 16x256b: (row g, col 2t), (row g, col 2t+1),
@@ -410,8 +470,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               r[4 * k + 3] = hmul2_bf16(int4_pair_to_bf16x2(wd[k] >> 12), s_hi);
             }
           } else {
-            const uint2 sv = *reinterpret_cast<const uint2*>(ssrc + j * 64 + g * 8);
-            const uint32_t sw2[2] = {sv.x, sv.y};
+            const uint32_t sw2[2] = {blk ? sv2 : sv0, blk ? sv3 : sv1};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint32_t s2 =
@@ -423,15 +482,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               r[4 * k + 3] = hmul2_f16(e2m1x2_to_f16x2(wd[k] >> 24), s_hi);
             }
           }
-          tmem_st_16x256b_x4(tmem + lane_base + kAColBase + slot * 64 + h * 32, r);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(afull + slot);
+          tmem_st_16x256b_x4(tmem + lane_base + kAColBase + sl * 128 + h * 64 + blk * 32, r);
         }
-        if (!ok) break;
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(sfree + s);  // this warp's shared-memory reads are done
+        if (lane == 0) mbar_arrive(afull + sl);
       }
       if (!ok) break;
 
@@ -480,19 +536,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (*fix_word == static_cast<unsigned>(p.S - 1)) {
           __threadfence();
           if (n < p.N) {
-            for (int c = 0; c < kHalf; ++c) {
-              const int m = m0 + c;
-              if (m >= p.M) break;
-              float acc = 0.f;
-              for (int sp = 0; sp < p.S; ++sp) acc += __ldcg(p.ws + ((size_t)sp * p.M + m) * Npad + n);
-              if (FMT == 1) acc = acc * __ldg(p.row_mul + m) * gmul;
-              p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(acc);
+            // 8 columns at a time, every split's partial of them in flight at once
+#pragma unroll
+            for (int c0 = 0; c0 < kHalf; c0 += 8) {
+              float acc[8];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+              for (int sp = 0; sp < p.S; ++sp) {
+                const float* src = p.ws + ((size_t)sp * p.M + m0 + c0) * Npad + n;
+                float part[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) part[c] = m0 + c0 + c < p.M ? __ldcg(src + c * Npad) : 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[c] += part[c];
+              }
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int m = m0 + c0 + c;
+                if (m < p.M) {
+                  float val = acc[c];
+                  if (FMT == 1) val = val * __ldg(p.row_mul + m) * gmul;
+                  p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
+                }
+              }
             }
           }
           if (threadIdx.x == 0) p.counters[tile] = 0u;
         }
       }
     }
+    cpa_wait<0>();  // no copy in flight at exit
   }
 
   // ------------------------------------------------------------------ teardown
@@ -562,6 +635,7 @@ bool make_xmap(CUtensorMap* map, const void* x, int M, int K, int mpad, bool f16
   return r == CUDA_SUCCESS;
 }
 
+
 template <int FMT, int MPAD>
 cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, const float* row_mul,
                      cudaStream_t st) {
@@ -583,7 +657,7 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   p.NT = (a.N + 15) / 16;
   p.tiles = (a.N + kTcTileRows - 1) / kTcTileRows;
   p.S = pl.S;
-  p.kbs = pl.kbs;
+  p.gps = pl.kbs / 2;
   p.units = p.tiles * pl.S;
   static int smem_set[64] = {0};
   int dev = 0;
@@ -612,20 +686,22 @@ cudaError_t launch_fmt(const TcPlan& pl, const GemmArgs& a, const void* xsrc, co
 
 }  // namespace
 
+// Splits K so that the units (256-row tiles x K splits, whole 128-groups
+// each) fill the SMs: the cost is the number of groups the busiest CTA
+// processes, plus a penalty for the split-K fixup.
 TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
   TcPlan pl;
   pl.mpad = (M + 15) / 16 * 16;
   const int tiles = (N + kTcTileRows - 1) / kTcTileRows;
-  const int KB = K / 64;
   const int groups = K / 128;
   double best = 1e300;
   int best_s = 1;
   for (int S = 1; S <= 16 && S <= groups; ++S) {
-    const int kbs = 2 * ((groups + S - 1) / S);   // whole 128-groups per split
-    if ((S - 1) * kbs >= KB) continue;
+    const int gps = (groups + S - 1) / S;
+    if ((S - 1) * gps >= groups) continue;
     const int units = tiles * S;
     const int waves = (units + num_sms - 1) / num_sms;
-    const double cost = (double)waves * kbs + (S > 1 ? 4.0 : 0.0);
+    const double cost = (double)waves * gps + (S > 1 ? 2.0 : 0.0);
     if (cost < best - 1e-9) {
       best = cost;
       best_s = S;
@@ -642,7 +718,6 @@ TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
     case 48: smem = fmt == 0 ? TcShape<0, 48>::kSmem : TcShape<1, 48>::kSmem; break;
     default: smem = fmt == 0 ? TcShape<0, 64>::kSmem : TcShape<1, 64>::kSmem; break;
   }
-  if (smem < kMinSmem) smem = kMinSmem;
   pl.smem = smem;
   return pl;
 }
