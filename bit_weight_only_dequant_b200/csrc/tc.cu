@@ -495,40 +495,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!warp_wait(dfull, unit_i & 1, abort_flag, p.err)) break;
       tc_fence_after();
       constexpr int kHalf = MPAD / 2;                   // columns this warp reads
-      float v[kHalf];
-#pragma unroll
-      for (int c = 0; c < kHalf / 8; ++c)
-        tmem_ld_32x32b_x8(tmem + ((uint32_t)(32 * q) << 16) + h * 64 + bp * kHalf + c * 8, v + 8 * c);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dfree);
-
       const int n = tile * kTcTileRows + h * 128 + 32 * q + lane;
       const int m0 = bp * kHalf;
       float gmul = 1.f;
       if (FMT == 1) gmul = __ldg(p.g);
-      if (p.S == 1) {
+      const size_t Npad = (size_t)p.NT * 16;
+      // eight columns at a time (few live registers)
+#pragma unroll 1
+      for (int c0 = 0; c0 < kHalf; c0 += 8) {
+        float v[8];
+        tmem_ld_32x32b_x8(tmem + ((uint32_t)(32 * q) << 16) + h * 64 + m0 + c0, v);
+        tmem_wait_ld();
         if (n < p.N) {
 #pragma unroll
-          for (int c = 0; c < kHalf; ++c) {
-            const int m = m0 + c;
+          for (int c = 0; c < 8; ++c) {
+            const int m = m0 + c0 + c;
             if (m < p.M) {
-              float val = v[c];
-              if (FMT == 1) val = val * __ldg(p.row_mul + m) * gmul;
-              p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
+              if (p.S == 1) {
+                float val = v[c];
+                if (FMT == 1) val = val * __ldg(p.row_mul + m) * gmul;
+                p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
+              } else {
+                __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v[c]);
+              }
             }
           }
         }
-      } else {
-        const size_t Npad = (size_t)p.NT * 16;
-        if (n < p.N) {
-#pragma unroll
-          for (int c = 0; c < kHalf; ++c) {
-            const int m = m0 + c;
-            if (m < p.M) __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v[c]);
-          }
-        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dfree);
+
+      if (p.S > 1) {
         __threadfence();
         asm volatile("bar.sync 1, %0;" ::"n"(kDeqWarps * 32));
         if (threadIdx.x == 0) *fix_word = atomicAdd(p.counters + tile, 1u);
@@ -537,7 +535,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __threadfence();
           if (n < p.N) {
             // 8 columns at a time, every split's partial of them in flight at once
-#pragma unroll
+#pragma unroll 1
             for (int c0 = 0; c0 < kHalf; c0 += 8) {
               float acc[8];
 #pragma unroll
