@@ -94,11 +94,16 @@ int check_fmt_shape(int fmt, int N, int K) {
 
 // Row-count dispatch: the weight-streaming GEMV while the activations are a
 // thin n8 operand, the tcgen05 path once the tensor cores carry real work.
+// Row-count dispatch, from back-to-back timings of both paths on the decode
+// shapes (B200): the GEMV wins up to M = 8 everywhere and at M = 9..16 for
+// NVFP4 and for int4 with N >= 8192 (a 16-row GEMV tile per SM has enough
+// bands); the tensor-core path wins for narrower int4 layers at M >= 9 and
+// everywhere at M > 16.
 int choose_path(int fmt, int M, int N, int K) {
-  (void)fmt;
-  (void)N;
   (void)K;
-  return M <= 8 ? W4A16_PATH_GEMV : W4A16_PATH_TC;
+  if (M <= 8) return W4A16_PATH_GEMV;
+  if (M <= W4A16_GEMV_MAX_M && (fmt == W4A16_FMT_NVFP4_G16 || N >= 8192)) return W4A16_PATH_GEMV;
+  return W4A16_PATH_TC;
 }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA; }
@@ -204,6 +209,7 @@ int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16, co
   void* scratch = nullptr;
   if (path == W4A16_PATH_GEMV) {
     const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, d->num_sms);
+    if (pl.S == 0) return W4A16_ERR_SHAPE;
     const size_t nf = w4::gemv_workspace_floats(pl, M, N);
     if (nf > 0) {
       r = workspace(st, w4::gemv_counters(pl, N), nf, 0, &a.counters, &a.ws, &scratch);

@@ -589,6 +589,10 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   }
 }
 
+// Shared-memory bytes of the FP16 activation image of M rows and `groups`
+// 128-groups (one 16-byte pad per row).
+int image_bytes(int M, int groups) { return M * (groups * 256 + 16); }
+
 int warps_of(int fmt, int mt) {
   if (fmt == 0) return mt == 1 ? Cfg<0, 1>::kWarps : Cfg<0, 2>::kWarps;
   return mt == 1 ? Cfg<1, 1>::kWarps : Cfg<1, 2>::kWarps;
@@ -605,9 +609,11 @@ int header_of(int fmt, int mt) {
 // both powers of two) and the ring depth D.  Every warp's piece is padded to
 // a multiple of D groups (padding groups copy and add nothing) so that ring
 // slots stay compile-time constants across bands.  The cost is the largest
-// number of 64-blocks any warp processes (padding included), with small
-// penalties for cross-CTA split-K, per-round reductions and shallow rings;
-// the activation image and the rings must fit in shared memory together.
+// number of 64-blocks any warp processes (padding included) plus one per
+// round, 3 + S/2 for a cross-CTA split and a little for shallow rings; its
+// constants were fitted to a sweep of (S, wk, D) over the decode shapes at
+// M = 1, 4 and 8 on B200.  The activation image and the rings must fit in
+// shared memory together.
 GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
   GemvPlan pl;
   pl.mt = M <= 8 ? 1 : 2;
@@ -618,10 +624,12 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
   const int groups = K / 128;
   double best = 1e300;
   pl.S = 0;
-  for (int S = 1; S <= groups && S <= 32; ++S) {
+  static const int kSplits[] = {1, 2, 3, 4, 6, 8, 12, 16, 24, 32};
+  for (int S : kSplits) {
+    if (S > groups) break;
     const int gslice = (groups + S - 1) / S;
     if ((S - 1) * gslice >= groups) continue;  // an empty split
-    const int ximg = M * (gslice * 256 + 16);
+    const int ximg = image_bytes(M, gslice);
     const int dmax = min(kMaxDepth, (kMaxSmem - header - ximg) / (warps * sb));
     if (dmax < 2) continue;
     int ctas = num_sms / S;
@@ -636,8 +644,8 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
       for (int d = 2; d <= dmax; ++d) {
         if (d == 7) continue;                  // not instantiated
         const int padded = (piece + d - 1) / d * d;
-        const double cost = (double)rounds * (2.0 * padded + (wk > 1 ? 2.0 : 0.5)) +
-                            (S > 1 ? 3.0 : 0.0) + (d < 4 ? 1.5 * (4 - d) : 0.0);
+        const double cost = (double)rounds * (2.0 * padded + 1.0) +
+                            (S > 1 ? 3.0 + 0.5 * S : 0.0) + (d < 4 ? 0.5 * (4 - d) : 0.0);
         if (cost < best - 1e-9) {
           best = cost;
           pl.S = S;
@@ -648,6 +656,20 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
       }
     }
   }
+  if (pl.S == 0) {
+    // very long K: the smallest split whose activation slice fits
+    for (int S = 33; S <= groups && pl.S == 0; ++S) {
+      const int gslice = (groups + S - 1) / S;
+      if ((S - 1) * gslice >= groups) continue;
+      if (kMaxSmem - header - image_bytes(M, gslice) >= warps * 2 * sb) {
+        pl.S = S;
+        pl.wk = 1;
+        pl.depth = 2;
+        pl.ngp = (gslice + 1) / 2 * 2;
+      }
+    }
+    if (pl.S == 0) return pl;  // no plan: the caller reports W4A16_ERR_SHAPE
+  }
   pl.wn = warps / pl.wk;
   const int gslice = (groups + pl.S - 1) / pl.S;
   pl.kslice = gslice * 128;
@@ -655,7 +677,7 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
   if (ctas < 1) ctas = 1;
   if (ctas > NT) ctas = NT;
   pl.ctas_x = ctas;
-  pl.smem = header + warps * pl.depth * sb + M * ((pl.kslice / 64) * 128 + 16);
+  pl.smem = header + warps * pl.depth * sb + image_bytes(M, gslice);
   return pl;
 }
 

@@ -86,6 +86,7 @@ extern "C" int w4a16_gemm_noalloc(int fmt, int M, int N, int K, const void* x_bf
   if (r != W4A16_OK) return r;
 
   const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, d->num_sms);
+  if (pl.S == 0) return W4A16_ERR_SHAPE;
   const size_t counters = w4::gemv_counters(pl, N);
   const size_t floats = w4::gemv_workspace_floats(pl, M, N);
   const size_t counter_bytes = (counters * sizeof(unsigned) + 255) / 256 * 256;

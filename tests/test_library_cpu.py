@@ -158,4 +158,10 @@ def test_dispatcher_path_table():
         path = W.w4a16_gemm_path(0, M, 5120, 5120)
         assert path in (W.PATH_GEMV, W.PATH_TC)
     assert W.w4a16_gemm_path(0, 1, 17408, 5120) == W.PATH_GEMV
+    assert W.w4a16_gemm_path(0, 8, 5120, 6144) == W.PATH_GEMV
+    assert W.w4a16_gemm_path(0, 9, 5120, 6144) == W.PATH_TC      # narrow int4 layer
+    assert W.w4a16_gemm_path(0, 16, 34816, 5120) == W.PATH_GEMV  # wide int4 layer
+    assert W.w4a16_gemm_path(1, 16, 5120, 17408) == W.PATH_GEMV  # NVFP4
+    assert W.w4a16_gemm_path(0, 17, 34816, 5120) == W.PATH_TC
+    assert W.w4a16_gemm_path(0, 64, 34816, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 65, 5120, 5120) == W.ERR_SHAPE
