@@ -13,6 +13,7 @@ namespace {
 struct DeviceState {
   bool checked = false;
   bool ok = false;        // sm_100
+  int dev = 0;
   int num_sms = 0;
   unsigned* err = nullptr;  // device error word
 };
@@ -28,6 +29,41 @@ std::mutex g_mu;
 std::map<int, DeviceState> g_dev;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
+// Plans depend only on (format, M, N, K) and the SM count: computed once per
+// shape and device (a decode step calls the same few shapes every token).
+struct PlanKey {
+  int dev, fmt, M, N, K;
+  bool operator<(const PlanKey& o) const {
+    if (dev != o.dev) return dev < o.dev;
+    if (fmt != o.fmt) return fmt < o.fmt;
+    if (M != o.M) return M < o.M;
+    if (N != o.N) return N < o.N;
+    return K < o.K;
+  }
+};
+std::map<PlanKey, w4::GemvPlan> g_gemv_plans;
+std::map<PlanKey, w4::TcPlan> g_tc_plans;
+
+w4::GemvPlan cached_gemv_plan(int dev, int fmt, int M, int N, int K, int num_sms) {
+  const PlanKey key{dev, fmt, M, N, K};
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_gemv_plans.find(key);
+  if (it != g_gemv_plans.end()) return it->second;
+  const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, num_sms);
+  if (g_gemv_plans.size() < 4096) g_gemv_plans.emplace(key, pl);
+  return pl;
+}
+
+w4::TcPlan cached_tc_plan(int dev, int fmt, int M, int N, int K, int num_sms) {
+  const PlanKey key{dev, fmt, M, N, K};
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_tc_plans.find(key);
+  if (it != g_tc_plans.end()) return it->second;
+  const w4::TcPlan pl = w4::plan_tc(fmt, M, N, K, num_sms);
+  if (g_tc_plans.size() < 4096) g_tc_plans.emplace(key, pl);
+  return pl;
+}
+
 int device_state(DeviceState** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
@@ -37,6 +73,7 @@ int device_state(DeviceState** out) {
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return W4A16_ERR_CUDA;
     d.ok = prop.major == 10 && prop.minor == 0;
+    d.dev = dev;
     d.num_sms = prop.multiProcessorCount;
     if (d.ok) {
       if (cudaMalloc(&d.err, sizeof(unsigned)) != cudaSuccess) return W4A16_ERR_NOMEM;
@@ -208,7 +245,7 @@ int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16, co
   a.err = d->err;
   void* scratch = nullptr;
   if (path == W4A16_PATH_GEMV) {
-    const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, d->num_sms);
+    const w4::GemvPlan pl = cached_gemv_plan(d->dev, fmt, M, N, K, d->num_sms);
     if (pl.S == 0) return W4A16_ERR_SHAPE;
     const size_t nf = w4::gemv_workspace_floats(pl, M, N);
     if (nf > 0) {
@@ -217,7 +254,7 @@ int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16, co
     }
     return status_of(w4::launch_gemv(pl, a, st));
   }
-  const w4::TcPlan pl = w4::plan_tc(fmt, M, N, K, d->num_sms);
+  const w4::TcPlan pl = cached_tc_plan(d->dev, fmt, M, N, K, d->num_sms);
   const size_t nf = w4::tc_workspace_floats(pl, M, N);
   const size_t nb = w4::tc_x_f16_bytes(fmt, M, K);
   if (nf > 0 || nb > 0) {
