@@ -8,8 +8,7 @@
 // nibbles into multiply operands: at 7+ TB/s a B200 SM has about two
 // lane-instructions per weight.
 //
-// Structure (one CTA per SM; 32 warps for int4 at M <= 8, 24 for NVFP4,
-// 16 for M <= 16):
+// Structure (one CTA of 16 warps per SM):
 //  * A CTA owns one K-slice and a contiguous range of 16-row bands.  Its
 //    warps form a (Wn x Wk) grid: Wn bands in flight at a time, each band's
 //    slice cut into Wk group-aligned pieces, one per warp.  The Wk partial
@@ -20,10 +19,10 @@
 //    filled by cp.async: every lane copies, and later reads back, exactly its
 //    own 16 bytes of each tile (a warp's copies cover the whole tile), so no
 //    barrier guards the ring; only the lane's own cp.async groups are waited
-//    for.  The ring holds up to six groups per warp (about 190 KB per SM in
-//    flight) without spending registers, and runs on from one band's piece
-//    into the next.  The first copies are issued before the activations are
-//    staged and, under programmatic dependent launch, before the previous
+//    for.  The ring holds up to eight groups per warp (up to 144 KB per SM
+//    in flight) without spending registers, and runs on from one band's
+//    piece into the next.  The first copies are issued before the activations
+//    are staged and, under programmatic dependent launch, before the previous
 //    kernel on the stream has finished: only the activations depend on it.
 //  * The CTA copies its slice of the activations into shared memory as FP16,
 //    each row rescaled by a power of two so that its largest magnitude lies in
@@ -47,8 +46,7 @@ namespace {
 
 constexpr int kRowWords = 64;                                // per-row words (M <= 64)
 constexpr int kRowAuxOff = kRowWords * 4;
-constexpr int kZeroOff = 2 * kRowWords * 4;                  // 128 zero bytes
-constexpr int kRedOff = kZeroOff + 128;
+constexpr int kRedOff = 2 * kRowWords * 4;                   // per-lane partial sums
 constexpr int kMaxSmem = 232448;                             // 227 KB opt-in
 constexpr int kMaxDepth = 8;                                 // ring stages per warp
 constexpr int kGroupBytes = 2 * kTileBytes;                  // packed weights of one band-group
@@ -360,7 +358,6 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
   const uint8_t* ring = smem + C::kHeader + warp * D * kSB;       // this warp's stages
   uint8_t* xs = smem + C::kHeader + C::kWarps * D * kSB;          // activation image
   if (threadIdx.x < kRowWords) row_aux[threadIdx.x] = 0u;
-  if (threadIdx.x < 32) reinterpret_cast<uint32_t*>(smem + kZeroOff)[threadIdx.x] = 0u;
   pdl_launch_dependents();
 
   // work of this CTA and warp (no divisions: the host passes quotients and

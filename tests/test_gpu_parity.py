@@ -298,3 +298,61 @@ def test_golden_examples_on_gpu():
 
 def test_device_status_is_clean():
     assert W.w4a16_device_status() == W.OK
+
+
+# ---------------------------------------------------------------- chained launches
+# Every GEMV launch lets the next kernel on the stream start early
+# (programmatic dependent launch) and waits for the previous one only before
+# it reads the activations.  A chain whose layers feed each other, issued
+# back to back with no host synchronisation (eagerly and as a CUDA graph),
+# checks that each layer reads its input only after the previous layer wrote
+# it: every layer is compared with the oracle applied to the previous layer's
+# GPU output.
+
+
+def _chain_layers(fmt, dims, seed):
+    layers = []
+    for i, (K, N) in enumerate(zip(dims[:-1], dims[1:])):
+        p = synth.problem(fmt, seed + i, 1, N, K)
+        codes, scales, _ = to_device_problem(p)
+        pw, ps = W.pack_on_device(fmt, N, K, codes, scales)
+        layers.append((K, N, pw, ps, gscale_tensor(p["g"]), oracle_weights(p)))
+    return layers
+
+
+@pytest.mark.parametrize("fmt,M,path", [("int4", 1, W.PATH_GEMV), ("int4", 4, W.PATH_GEMV),
+                                        ("int4", 9, W.PATH_AUTO), ("nvfp4", 2, W.PATH_GEMV)])
+@pytest.mark.parametrize("graph", [False, True])
+def test_chained_layers_read_their_inputs_after_they_are_written(fmt, M, path, graph):
+    t = torch()
+    dims = [1024, 2048, 1536, 3072, 1024, 2048, 1024]
+    layers = _chain_layers(fmt, dims, 300 + M)
+    x0 = synth.problem(fmt, 399, M, 256, dims[0])["x"]
+    bufs = [t.from_numpy(np.ascontiguousarray(x0.view(np.int16))).cuda().view(t.bfloat16)]
+    for K, N, *_ in layers:
+        bufs.append(t.full((M, N), float("nan"), dtype=t.bfloat16, device="cuda"))
+    s = t.cuda.Stream()
+
+    def run():
+        for i, (K, N, pw, ps, g, _) in enumerate(layers):
+            W.gemm(fmt, bufs[i], pw, ps, N, global_scale=g, y=bufs[i + 1], path=path, stream=s)
+
+    with t.cuda.stream(s):
+        if graph:
+            run()                       # plans and workspace outside the capture
+            s.synchronize()
+            for b in bufs[1:]:
+                b.fill_(float("nan"))
+            gr = t.cuda.CUDAGraph()
+            with t.cuda.graph(gr, stream=s):
+                run()
+            gr.replay()
+        else:
+            run()
+    s.synchronize()
+    W.check(W.w4a16_device_status(s), "device status")
+    for i, (K, N, pw, ps, g, wref) in enumerate(layers):
+        x_in = bf16_bits(bufs[i])
+        y = bufs[i + 1].float().cpu().numpy().astype(np.float64)
+        assert not np.isnan(y).any(), (fmt, M, i)
+        assert_parity(y, x_in, wref, f"{fmt} M={M} layer {i}")
