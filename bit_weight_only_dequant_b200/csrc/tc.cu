@@ -1,4 +1,5 @@
-// Tensor-core path for speculative-verify row counts (M = 9 .. 64) on sm_100a.
+// Tensor-core path for speculative-verify and small-batch row counts
+// (M = 9 .. 256) on sm_100a.
 //
 // At M = 64 the matmul does 256 flops per packed weight byte, close to the
 // B200 ridge, so the multiply-adds belong on the 5th-generation tensor cores
@@ -23,12 +24,17 @@
 //    memory, B (activations, K-major SW128) from shared memory, fp32 D
 //    (128 lanes x Mpad columns) per 128-row half; 16 MMAs per group, issued
 //    by one elected lane of a converged warp.
-//  * epilogue: tcgen05.ld of D, BF16 stores (or fp32 split-K partials reduced
-//    in split order by the last CTA of the tile).
-// Tensor memory: D at columns [0, 128), three A slots of one group (2 halves
-// x 64 columns) at [128, 512).  Every mbarrier wait is bounded; a timeout
-// raises the device error word, the CTA drains its copies and MMAs and frees
-// tensor memory.
+//  * epilogue: tcgen05.ld of D, BF16 stores, or fp32 split-K partials that a
+//    second kernel (all SMs, programmatic dependent launch) sums in split
+//    order.
+// Tensor memory: D (two 128-row halves of Mpad columns), then A slots of one
+// group (2 halves x 64 columns) in the rest of the 512 columns.  Every
+// mbarrier wait is bounded; a timeout raises the device error word, the CTA
+// drains its copies and MMAs and frees tensor memory.
+//
+// M > 128 runs as launches of at most 128 activation rows (the MMA's N),
+// each streaming the whole weight matrix: beyond M = 128 the tensor cores,
+// not HBM, set the time.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -45,12 +51,10 @@ constexpr int kProducerWarp = kDeqWarps;
 constexpr int kMmaWarp = kDeqWarps + 1;
 constexpr int kTcTileRows = 256;              // 16 bands, two 128-row MMA tiles
 constexpr int kWRing = 4;                     // weight stages (groups) per dequant warp
-constexpr int kXRing = 4;                     // activation stages (groups)
-constexpr int kASlots = 3;                    // tensor-memory A slots of one group each
 constexpr int kTmemCols = 512;
-constexpr int kAColBase = 128;
 constexpr int kGroupBytesW = 2 * kTileBytes;  // one band's packed weights per 128-group
 constexpr int kMinSmem = 120 * 1024;          // keeps one CTA (and one TMEM owner) per SM
+constexpr int kMaxSmem = 227 * 1024;          // dynamic shared memory limit of one CTA
 
 // Weight ring stage: the group's two tiles (each lane's 16 bytes at 16 lane),
 // then the scales each lane needs (int4: 4 bytes at 4 lane; NVFP4: 2 x 8 at 16 lane).
@@ -62,8 +66,7 @@ struct TcParams {
   const float* g;
   const float* row_mul;    // NVFP4: per-row power-of-two activation scale
   __nv_bfloat16* y;
-  float* ws;
-  unsigned* counters;
+  float* ws;               // split-K partials [S][M][Npad] (S > 1)
   unsigned* err;
   int M, N, K, KB, NT, tiles, S, gps, units;   // gps: 128-groups per split
 };
@@ -101,6 +104,35 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, float* v) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, float* v);
+
+template <>
+__device__ __forceinline__ void tmem_ld_32x32b<8>(uint32_t taddr, float* v) {
+  tmem_ld_32x32b_x8(taddr, v);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_32x32b<16>(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld_32x32b<32>(uint32_t taddr, float* v) {
+  tmem_ld_32x32b<16>(taddr, v);
+  tmem_ld_32x32b<16>(taddr + 16, v + 16);
 }
 
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -207,12 +239,24 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t phase, volatil
 }
 
 
+// Per activation width MPAD (rows of x padded to 16, at most 128 per launch):
+// tensor memory holds D (two 128-row halves of MPAD fp32 columns, 64 apart up
+// to MPAD = 64) and then as many A slots of one group (2 halves x 64 columns)
+// as fit; the activation ring has four stages where they fit in shared memory.
 template <int FMT, int MPAD>
 struct TcShape {
+  static constexpr int kDStride = MPAD <= 64 ? 64 : 128;     // columns between the D halves
+  static constexpr int kAColBase = 2 * kDStride;
+  static constexpr int kASlots = (kTmemCols - kAColBase) / 128;
   static constexpr int kXStage = 2 * MPAD * 128;             // two 64-k activation boxes
   static constexpr int kWRingBytes = kDeqWarps * kWRing * tc_stage_bytes(FMT);
+  static constexpr int kXRing =                               // activation stages (groups)
+      4 * kXStage + kWRingBytes + 2048 <= kMaxSmem ? 4 : 3;
   static constexpr int kSmemUse = kXRing * kXStage + kWRingBytes + 1024 /* barriers */;
   static constexpr int kSmem = (kSmemUse + 1024 /* align */ > kMinSmem) ? kSmemUse + 1024 : kMinSmem;
+  static_assert(kSmem <= kMaxSmem, "stage rings exceed shared memory");
+  static_assert(kASlots >= 2 && kAColBase + kASlots * 128 <= kTmemCols, "tensor memory layout");
+  static_assert(MPAD % 16 == 0 && MPAD <= kTcMaxRows, "MMA N");
 };
 
 __device__ __forceinline__ void cpa16(uint32_t dst, const void* src, uint64_t pol) {
@@ -247,6 +291,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap xmap, const TcParams p) {
   using Sh = TcShape<FMT, MPAD>;
   constexpr int kSB = tc_stage_bytes(FMT);
+  constexpr int kXRing = Sh::kXRing, kASlots = Sh::kASlots, kAColBase = Sh::kAColBase;
+  constexpr int kDStride = Sh::kDStride;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -262,7 +308,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* drain = dfull + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile unsigned* fix_word = reinterpret_cast<volatile unsigned*>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -347,7 +392,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_ts(tmem + h * 64, a0 + h * 64 + kk * 8,
+              umma_ts(tmem + h * kDStride, a0 + h * 64 + kk * 8,
                       b0 + (uint64_t)(((kk >> 2) * MPAD * 128) >> 4) + (uint64_t)((kk & 3) * 2),
                       idesc, (gi > g_lo || kk > 0) ? 1u : 0u);
           umma_commit(afree + sl);
@@ -360,6 +405,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
       }
     }
+    // every MMA is issued: the split-K reduction grid may be scheduled
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // drain: all issued MMAs complete before tensor memory is released
     if (elect_one()) {
       umma_commit(drain);
@@ -495,20 +542,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!warp_wait(dfull, unit_i & 1, abort_flag, p.err)) break;
       tc_fence_after();
       constexpr int kHalf = MPAD / 2;                   // columns this warp reads
+      constexpr int kEC = kHalf % 32 == 0 ? 32 : kHalf % 16 == 0 ? 16 : 8;   // per tcgen05.ld
       const int n = tile * kTcTileRows + h * 128 + 32 * q + lane;
       const int m0 = bp * kHalf;
       float gmul = 1.f;
       if (FMT == 1) gmul = __ldg(p.g);
       const size_t Npad = (size_t)p.NT * 16;
-      // eight columns at a time (few live registers)
 #pragma unroll 1
-      for (int c0 = 0; c0 < kHalf; c0 += 8) {
-        float v[8];
-        tmem_ld_32x32b_x8(tmem + ((uint32_t)(32 * q) << 16) + h * 64 + m0 + c0, v);
+      for (int c0 = 0; c0 < kHalf; c0 += kEC) {
+        float v[kEC];
+        tmem_ld_32x32b<kEC>(tmem + ((uint32_t)(32 * q) << 16) + h * kDStride + m0 + c0, v);
         tmem_wait_ld();
         if (n < p.N) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < kEC; ++c) {
             const int m = m0 + c0 + c;
             if (m < p.M) {
               if (p.S == 1) {
@@ -525,43 +572,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dfree);
-
-      if (p.S > 1) {
-        __threadfence();
-        asm volatile("bar.sync 1, %0;" ::"n"(kDeqWarps * 32));
-        if (threadIdx.x == 0) *fix_word = atomicAdd(p.counters + tile, 1u);
-        asm volatile("bar.sync 1, %0;" ::"n"(kDeqWarps * 32));
-        if (*fix_word == static_cast<unsigned>(p.S - 1)) {
-          __threadfence();
-          if (n < p.N) {
-            // 8 columns at a time, every split's partial of them in flight at once
-#pragma unroll 1
-            for (int c0 = 0; c0 < kHalf; c0 += 8) {
-              float acc[8];
-#pragma unroll
-              for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-              for (int sp = 0; sp < p.S; ++sp) {
-                const float* src = p.ws + ((size_t)sp * p.M + m0 + c0) * Npad + n;
-                float part[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) part[c] = m0 + c0 + c < p.M ? __ldcg(src + c * Npad) : 0.f;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[c] += part[c];
-              }
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const int m = m0 + c0 + c;
-                if (m < p.M) {
-                  float val = acc[c];
-                  if (FMT == 1) val = val * __ldg(p.row_mul + m) * gmul;
-                  p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
-                }
-              }
-            }
-          }
-          if (threadIdx.x == 0) p.counters[tile] = 0u;
-        }
-      }
     }
     cpa_wait<0>();  // no copy in flight at exit
   }
@@ -602,6 +612,57 @@ __global__ void prep_x_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* _
   if (threadIdx.x == 0) row_mul[m] = ldexpf(1.f, e);
   for (int k = threadIdx.x; k < K; k += blockDim.x)
     xh[(size_t)m * K + k] = __float2half_rn(ldexpf(__bfloat162float(row[k]), -e));
+}
+
+// Split-K reduction: y[m][n] = BF16(sum over splits, in split order, of the
+// fp32 partials [S][M][Npad]), times the NVFP4 row multiplier and global
+// scale.  Four columns per thread; launched behind the main kernel with
+// programmatic dependent launch, so it waits for the partials on the device.
+template <int FMT>
+__global__ void __launch_bounds__(256)
+    tc_splitk_reduce(const float* __restrict__ ws, int S, int M, int N, int Npad,
+                     const float* __restrict__ row_mul, const float* __restrict__ g,
+                     __nv_bfloat16* __restrict__ y) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int m = blockIdx.y;
+  const int n0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (n0 >= N) return;
+  const size_t sstride = (size_t)M * Npad;
+  const float* src = ws + (size_t)m * Npad + n0;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  int sp = 0;
+  for (; sp + 4 <= S; sp += 4) {                 // four splits' loads in flight, added in order
+    float4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = __ldcg(reinterpret_cast<const float4*>(src + (sp + j) * sstride));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a[0] += v[j].x;
+      a[1] += v[j].y;
+      a[2] += v[j].z;
+      a[3] += v[j].w;
+    }
+  }
+  for (; sp < S; ++sp) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(src + sp * sstride));
+    a[0] += v.x;
+    a[1] += v.y;
+    a[2] += v.z;
+    a[3] += v.w;
+  }
+  float rm = 1.f, gm = 1.f;
+  if (FMT == 1) {
+    rm = __ldg(row_mul + m);
+    gm = __ldg(g);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (n0 + j < N) {
+      float val = a[j];
+      if (FMT == 1) val = val * rm * gm;
+      y[(size_t)m * N + n0 + j] = __float2bfloat16_rn(val);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -646,7 +707,6 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   p.row_mul = row_mul;
   p.y = static_cast<__nv_bfloat16*>(a.y);
   p.ws = a.ws;
-  p.counters = a.counters;
   p.err = a.err;
   p.M = a.M;
   p.N = a.N;
@@ -668,7 +728,21 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
     smem_set[dev] = pl.smem;
   }
   tc_kernel<FMT, MPAD><<<pl.grid, kTcThreads, pl.smem, st>>>(map, p);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || pl.S == 1) return e;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((a.N + 1023) / 1024), (unsigned)a.M, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_splitk_reduce<FMT>, static_cast<const float*>(a.ws), pl.S, a.M,
+                            a.N, p.NT * 16, row_mul, a.g, static_cast<__nv_bfloat16*>(a.y));
 }
 
 template <int FMT>
@@ -678,7 +752,11 @@ cudaError_t launch_fmt(const TcPlan& pl, const GemmArgs& a, const void* xsrc, co
     case 16: return launch_t<FMT, 16>(pl, a, xsrc, rm, st);
     case 32: return launch_t<FMT, 32>(pl, a, xsrc, rm, st);
     case 48: return launch_t<FMT, 48>(pl, a, xsrc, rm, st);
-    default: return launch_t<FMT, 64>(pl, a, xsrc, rm, st);
+    case 64: return launch_t<FMT, 64>(pl, a, xsrc, rm, st);
+    case 80: return launch_t<FMT, 80>(pl, a, xsrc, rm, st);
+    case 96: return launch_t<FMT, 96>(pl, a, xsrc, rm, st);
+    case 112: return launch_t<FMT, 112>(pl, a, xsrc, rm, st);
+    default: return launch_t<FMT, 128>(pl, a, xsrc, rm, st);
   }
 }
 
@@ -689,7 +767,9 @@ cudaError_t launch_fmt(const TcPlan& pl, const GemmArgs& a, const void* xsrc, co
 // processes, plus a penalty for the split-K fixup.
 TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
   TcPlan pl;
-  pl.mpad = (M + 15) / 16 * 16;
+  const int chunks = (M + kTcMaxRows - 1) / kTcMaxRows;
+  pl.rows = (M + chunks - 1) / chunks;
+  pl.mpad = (pl.rows + 15) / 16 * 16;
   const int tiles = (N + kTcTileRows - 1) / kTcTileRows;
   const int groups = K / 128;
   double best = 1e300;
@@ -714,30 +794,56 @@ TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
     case 16: smem = fmt == 0 ? TcShape<0, 16>::kSmem : TcShape<1, 16>::kSmem; break;
     case 32: smem = fmt == 0 ? TcShape<0, 32>::kSmem : TcShape<1, 32>::kSmem; break;
     case 48: smem = fmt == 0 ? TcShape<0, 48>::kSmem : TcShape<1, 48>::kSmem; break;
-    default: smem = fmt == 0 ? TcShape<0, 64>::kSmem : TcShape<1, 64>::kSmem; break;
+    case 64: smem = fmt == 0 ? TcShape<0, 64>::kSmem : TcShape<1, 64>::kSmem; break;
+    case 80: smem = fmt == 0 ? TcShape<0, 80>::kSmem : TcShape<1, 80>::kSmem; break;
+    case 96: smem = fmt == 0 ? TcShape<0, 96>::kSmem : TcShape<1, 96>::kSmem; break;
+    case 112: smem = fmt == 0 ? TcShape<0, 112>::kSmem : TcShape<1, 112>::kSmem; break;
+    default: smem = fmt == 0 ? TcShape<0, 128>::kSmem : TcShape<1, 128>::kSmem; break;
   }
   pl.smem = smem;
   return pl;
 }
 
 size_t tc_workspace_floats(const TcPlan& p, int M, int N) {
-  return p.S > 1 ? static_cast<size_t>(p.S) * M * ((N + 15) / 16 * 16) : 0;
+  const int rows = M < p.rows ? M : p.rows;   // chunks run one after another and share it
+  return p.S > 1 ? static_cast<size_t>(p.S) * rows * ((N + 15) / 16 * 16) : 0;
 }
 
-size_t tc_counters(const TcPlan& p, int N) { return p.S > 1 ? (N + 15) / 16 : 0; }
+size_t tc_counters(const TcPlan& p, int N) {
+  (void)p;
+  (void)N;
+  return 0;   // the split-K reduction is a separate kernel: no arrival counters
+}
 
 size_t tc_x_f16_bytes(int fmt, int M, int K) {
-  return fmt == 1 ? (size_t)M * K * 2 + 64 * sizeof(float) : 0;
+  return fmt == 1 ? (size_t)M * K * 2 + 256 * sizeof(float) : 0;
 }
 
+// NVFP4 first rescales all M rows into FP16 (one launch); then each chunk of
+// pl.rows activation rows is one launch that reads its slice of x and writes
+// its slice of y (plus, when K is split, one reduction launch).  Chunks are
+// stream-ordered, so they share the split-K partials.
 cudaError_t launch_tc(const TcPlan& pl, const GemmArgs& a, void* xf16_scratch, cudaStream_t st) {
-  if (a.fmt == 0) return launch_fmt<0>(pl, a, a.x, nullptr, st);
-  __half* xh = static_cast<__half*>(xf16_scratch);
-  float* rm = reinterpret_cast<float*>(static_cast<uint8_t*>(xf16_scratch) + (size_t)a.M * a.K * 2);
-  prep_x_f16_kernel<<<a.M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x), xh, rm, a.K);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_fmt<1>(pl, a, xh, rm, st);
+  const uint8_t* xsrc = static_cast<const uint8_t*>(a.x);
+  float* rm = nullptr;
+  if (a.fmt == 1) {
+    __half* xh = static_cast<__half*>(xf16_scratch);
+    rm = reinterpret_cast<float*>(static_cast<uint8_t*>(xf16_scratch) + (size_t)a.M * a.K * 2);
+    prep_x_f16_kernel<<<a.M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x), xh, rm, a.K);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    xsrc = reinterpret_cast<const uint8_t*>(xh);
+  }
+  for (int m0 = 0; m0 < a.M; m0 += pl.rows) {
+    GemmArgs c = a;
+    c.M = min(pl.rows, a.M - m0);
+    c.y = static_cast<uint8_t*>(a.y) + (size_t)m0 * a.N * 2;
+    const uint8_t* xc = xsrc + (size_t)m0 * a.K * 2;   // BF16 and FP16 rows are both 2K bytes
+    const cudaError_t e = a.fmt == 0 ? launch_fmt<0>(pl, c, xc, nullptr, st)
+                                     : launch_fmt<1>(pl, c, xc, rm + m0, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace w4

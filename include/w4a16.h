@@ -68,17 +68,19 @@ extern "C" {
 #define W4A16_ERR_SCRATCH (-8) /* w4a16_gemm_noalloc: the problem needs more than its fixed scratch */
 
 /* Limits of this version. */
-#define W4A16_MAX_M 64         /* decode / speculative-verify row counts */
+#define W4A16_MAX_M 256        /* decode, speculative verify and small prefill batches */
 
 /* Kernel paths (for w4a16_gemm_path / w4a16_gemm_ex). */
 #define W4A16_PATH_AUTO 0      /* row-count dispatch */
 #define W4A16_PATH_GEMV 1      /* weight-streaming split-K GEMV (mma.sync fragments), M <= 16 */
-#define W4A16_PATH_TC 2        /* tcgen05 tensor-core path (A in tensor memory), M <= 64 */
+#define W4A16_PATH_TC 2        /* tcgen05 tensor-core path (A in tensor memory), M <= 256 */
 #define W4A16_GEMV_MAX_M 16
 
 /*
- * Shape rules: 1 <= M <= 64; N >= 1 (any value; packed buffers are padded to
+ * Shape rules: 1 <= M <= 256; N >= 1 (any value; packed buffers are padded to
  * a multiple of 16 rows); K >= 128 and K a multiple of 128 (both formats).
+ * The tensor-core path runs M > 128 as two launches of about M/2 rows each
+ * (every launch streams the whole weight matrix once).
  */
 
 /* Bytes of the packed weight buffer: ceil(N/16)*16 * K / 2.  0 on bad args. */

@@ -140,7 +140,8 @@ def test_host_pack_rejects_out_of_range():
 def test_argument_validation_before_any_device_call():
     x = w = s = y = 1 << 20          # fake, aligned, never dereferenced
     assert W.w4a16_gemm(0, 0, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE       # M = 0
-    assert W.w4a16_gemm(0, 65, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE      # M > 64
+    assert W.w4a16_gemm(0, 257, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE     # M > 256
+    assert W.w4a16_gemm_ex(W.PATH_GEMV, 0, 17, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE
     assert W.w4a16_gemm(0, 1, 16, 100, x, w, s, None, y, 0) == W.ERR_SHAPE       # K % 128
     assert W.w4a16_gemm(0, 1, 0, 128, x, w, s, None, y, 0) == W.ERR_SHAPE        # N = 0
     assert W.w4a16_gemm(3, 1, 16, 128, x, w, s, None, y, 0) == W.ERR_ARG         # format
@@ -154,9 +155,10 @@ def test_argument_validation_before_any_device_call():
 
 
 def test_dispatcher_path_table():
-    for M in range(1, 65):
+    for M in range(1, W.MAX_M + 1):
         path = W.w4a16_gemm_path(0, M, 5120, 5120)
         assert path in (W.PATH_GEMV, W.PATH_TC)
+        assert M <= 16 or path == W.PATH_TC
     assert W.w4a16_gemm_path(0, 1, 17408, 5120) == W.PATH_GEMV
     assert W.w4a16_gemm_path(0, 8, 5120, 6144) == W.PATH_GEMV
     assert W.w4a16_gemm_path(0, 9, 5120, 6144) == W.PATH_TC      # narrow int4 layer
@@ -164,4 +166,6 @@ def test_dispatcher_path_table():
     assert W.w4a16_gemm_path(1, 16, 5120, 17408) == W.PATH_GEMV  # NVFP4
     assert W.w4a16_gemm_path(0, 17, 34816, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 64, 34816, 5120) == W.PATH_TC
-    assert W.w4a16_gemm_path(0, 65, 5120, 5120) == W.ERR_SHAPE
+    assert W.w4a16_gemm_path(0, 65, 5120, 5120) == W.PATH_TC
+    assert W.w4a16_gemm_path(1, 256, 17408, 5120) == W.PATH_TC
+    assert W.w4a16_gemm_path(0, 257, 5120, 5120) == W.ERR_SHAPE
