@@ -529,6 +529,7 @@ def run_native(args, rank, world, local_rank):
         cfg4 = [("nvfp4", n, K, N, Mv, 6) for Mv in (1, 9, 64) for n, K, N, _ in DECODE_SHAPES]
         cfg5 = [(fmt, n, K, N, Mv, 7) for fmt in ("int4", "nvfp4") for Mv in (128, 256)
                 for n, K, N, _ in DECODE_SHAPES]
+        cfg5 += [("int4", n, K, N, 2048, 8) for n, K, N, _ in DECODE_SHAPES]
         for fmt, n, K, N, Mv, s in target + cfg2 + cfg3 + cfg4 + cfg5:
             entries.append(sweep_entry(fmt, n, K, N, Mv, s, peaks, stream))
         extra["sweep"] = entries

@@ -40,16 +40,17 @@ cudaError_t launch_gemv(const GemvPlan& p, const GemmArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- tensor-core path (tcgen05)
 
-// Row chunking: M rows run as ceil(M / kTcMaxRows) launches of `rows` rows
-// each (the last one may be shorter), all with this one plan.
+// Row chunking: M rows run as ceil(M / kTcMaxRows) chunks of `rows` rows
+// each (the last one may be shorter), as units of one launch.
 constexpr int kTcMaxRows = 128;
 
 struct TcPlan {
-  int rows;      // activation rows per launch (M split evenly into <= kTcMaxRows)
+  int chunks;    // activation chunks
+  int rows;      // activation rows per chunk (M split evenly into <= kTcMaxRows)
   int mpad;      // rows padded to the MMA N (a multiple of 16, at most 128)
   int S;         // K splits
   int kbs;       // 64-blocks per split
-  int units;     // 256-row tiles x splits
+  int units;     // 256-row tiles x chunks x splits
   int grid;      // persistent CTAs
   int smem;      // dynamic shared memory bytes
 };

@@ -1,5 +1,5 @@
-// Tensor-core path for speculative-verify and small-batch row counts
-// (M = 9 .. 256) on sm_100a.
+// Tensor-core path for speculative-verify and prefill row counts
+// (M = 9 .. 8192) on sm_100a.
 //
 // At M = 64 the matmul does 256 flops per packed weight byte, close to the
 // B200 ridge, so the multiply-adds belong on the 5th-generation tensor cores
@@ -32,9 +32,10 @@
 // mbarrier wait is bounded; a timeout raises the device error word, the CTA
 // drains its copies and MMAs and frees tensor memory.
 //
-// M > 128 runs as launches of at most 128 activation rows (the MMA's N),
-// each streaming the whole weight matrix: beyond M = 128 the tensor cores,
-// not HBM, set the time.
+// M > 128 runs as chunks of at most 128 activation rows (the MMA's N); a unit
+// of work is (tile, chunk, K split), and the chunks of one tile are adjacent
+// units, so their weight reads mostly hit L2.  Beyond M = 128 the tensor
+// cores, not HBM, set the time.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -69,6 +70,7 @@ struct TcParams {
   float* ws;               // split-K partials [S][M][Npad] (S > 1)
   unsigned* err;
   int M, N, K, KB, NT, tiles, S, gps, units;   // gps: 128-groups per split
+  int chunks, rows;        // activation rows run as `chunks` slices of `rows`
 };
 
 // ------------------------------------------------------------------ tcgen05 wrappers
@@ -276,11 +278,16 @@ __device__ __forceinline__ void cpa_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// The K range of a unit (tile, split) in 128-groups.
-__device__ __forceinline__ void unit_range(const TcParams& p, int unit, int& tile, int& split,
-                                           int& g_lo, int& g_hi) {
-  tile = unit / p.S;
-  split = unit - tile * p.S;
+// A unit is (256-row tile, activation chunk, K split); units of one tile are
+// adjacent, so CTAs working at the same time share its weights in L2.
+// Returns the tile, the chunk, the split and its K range in 128-groups.
+__device__ __forceinline__ void unit_range(const TcParams& p, int unit, int& tile, int& chunk,
+                                           int& split, int& g_lo, int& g_hi) {
+  const int per_tile = p.chunks * p.S;
+  tile = unit / per_tile;
+  const int r = unit - tile * per_tile;
+  chunk = r / p.S;
+  split = r - chunk * p.S;
   const int G = p.K >> 7;
   g_lo = split * p.gps;
   g_hi = min(G, g_lo + p.gps);
@@ -343,8 +350,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     if (lane == 0) {
       for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
-        int tile, split, g_lo, g_hi;
-        unit_range(p, unit, tile, split, g_lo, g_hi);
+        int tile, chunk, split, g_lo, g_hi;
+        unit_range(p, unit, tile, chunk, split, g_lo, g_hi);
+        const int xrow = chunk * p.rows;
         for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
           const int s = it % kXRing;
           const uint32_t u = it / kXRing;
@@ -354,8 +362,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           mbar_arrive_expect_tx(xfull + s, Sh::kXStage);
           uint8_t* dst = Xs + s * Sh::kXStage;
-          tma_load_2d(dst, &xmap, gi * 128, 0, xfull + s);
-          tma_load_2d(dst + MPAD * 128, &xmap, gi * 128 + 64, 0, xfull + s);
+          tma_load_2d(dst, &xmap, gi * 128, xrow, xfull + s);
+          tma_load_2d(dst + MPAD * 128, &xmap, gi * 128 + 64, xrow, xfull + s);
         }
       }
       // drain: every issued copy has landed before the CTA may exit
@@ -370,9 +378,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t it = 0, unit_i = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
-      int tile, split, g_lo, g_hi;
-      unit_range(p, unit, tile, split, g_lo, g_hi);
+      int tile, chunk, split, g_lo, g_hi;
+      unit_range(p, unit, tile, chunk, split, g_lo, g_hi);
       (void)tile;
+      (void)chunk;
       if (unit_i > 0) {
         if (!warp_wait(dfree, (unit_i - 1) & 1, abort_flag, p.err)) break;
         tc_fence_after();
@@ -431,8 +440,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint8_t* cs = nullptr;
     auto c_start = [&]() {
       if (c_unit < p.units) {
-        int tile, split, g_lo;
-        unit_range(p, c_unit, tile, split, g_lo, c_hi);
+        int tile, chunk, split, g_lo;
+        unit_range(p, c_unit, tile, chunk, split, g_lo, c_hi);
         c_gi = g_lo;
         c_nb = tile * 16 + band;
         const int nb = min(c_nb, p.NT - 1);
@@ -472,8 +481,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t it = 0, unit_i = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
-      int tile, split, g_lo, g_hi;
-      unit_range(p, unit, tile, split, g_lo, g_hi);
+      int tile, chunk, split, g_lo, g_hi;
+      unit_range(p, unit, tile, chunk, split, g_lo, g_hi);
       const bool real_band = tile * 16 + band < p.NT;
       for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
         const int sl = it % kASlots;
@@ -544,7 +553,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr int kHalf = MPAD / 2;                   // columns this warp reads
       constexpr int kEC = kHalf % 32 == 0 ? 32 : kHalf % 16 == 0 ? 16 : 8;   // per tcgen05.ld
       const int n = tile * kTcTileRows + h * 128 + 32 * q + lane;
-      const int m0 = bp * kHalf;
+      const int m0 = bp * kHalf;                        // local row of the chunk
+      const int xrow = chunk * p.rows;
+      const int mlim = min(p.rows, p.M - xrow);          // rows of this chunk
       float gmul = 1.f;
       if (FMT == 1) gmul = __ldg(p.g);
       const size_t Npad = (size_t)p.NT * 16;
@@ -554,18 +565,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld_32x32b<kEC>(tmem + ((uint32_t)(32 * q) << 16) + h * kDStride + m0 + c0, v);
         tmem_wait_ld();
         if (n < p.N) {
+          const int mb = xrow + m0 + c0;                 // first row of this batch
+          if (p.S == 1) {
+            __nv_bfloat16* yp = p.y + (size_t)mb * p.N + n;
 #pragma unroll
-          for (int c = 0; c < kEC; ++c) {
-            const int m = m0 + c0 + c;
-            if (m < p.M) {
-              if (p.S == 1) {
+            for (int c = 0; c < kEC; ++c, yp += p.N) {
+              if (m0 + c0 + c < mlim) {
                 float val = v[c];
-                if (FMT == 1) val = val * __ldg(p.row_mul + m) * gmul;
-                p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(val);
-              } else {
-                __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, v[c]);
+                if (FMT == 1) val = val * __ldg(p.row_mul + mb + c) * gmul;
+                *yp = __float2bfloat16_rn(val);
               }
             }
+          } else {
+            float* wp = p.ws + ((size_t)split * p.M + mb) * Npad + n;
+#pragma unroll
+            for (int c = 0; c < kEC; ++c, wp += Npad)
+              if (m0 + c0 + c < mlim) __stcg(wp, v[c]);
           }
         }
       }
@@ -716,7 +731,9 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   p.tiles = (a.N + kTcTileRows - 1) / kTcTileRows;
   p.S = pl.S;
   p.gps = pl.kbs / 2;
-  p.units = p.tiles * pl.S;
+  p.chunks = pl.chunks;
+  p.rows = pl.rows;
+  p.units = p.tiles * pl.chunks * pl.S;
   static int smem_set[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -762,24 +779,30 @@ cudaError_t launch_fmt(const TcPlan& pl, const GemmArgs& a, const void* xsrc, co
 
 }  // namespace
 
-// Splits K so that the units (256-row tiles x K splits, whole 128-groups
-// each) fill the SMs: the cost is the number of groups the busiest CTA
-// processes, plus a penalty for the split-K fixup.
+// Splits K so that the units (256-row tiles x row chunks x K splits, whole
+// 128-groups each) fill the SMs.  Estimated time in microseconds, from
+// per-group and per-unit timings of the kernel on B200 (clock64 timelines):
+// the busiest CTA's waves x (its groups x t_group + t_unit), t_unit being the
+// epilogue and pipeline refill of a unit, plus, with split K, the reduction
+// launch and its traffic (the partials written and read once more).
 TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
   TcPlan pl;
-  const int chunks = (M + kTcMaxRows - 1) / kTcMaxRows;
-  pl.rows = (M + chunks - 1) / chunks;
+  pl.chunks = (M + kTcMaxRows - 1) / kTcMaxRows;
+  pl.rows = (M + pl.chunks - 1) / pl.chunks;
   pl.mpad = (pl.rows + 15) / 16 * 16;
   const int tiles = (N + kTcTileRows - 1) / kTcTileRows;
   const int groups = K / 128;
+  const double t_group = 0.75 + 0.0017 * pl.mpad;   // us per 128-group of a 256-row tile
+  const double t_unit = 0.5 + 0.035 * pl.mpad;      // us per unit: epilogue, refill
+  const double part_mb = (double)M * ((N + 15) / 16 * 16) * 4 / 1e6;   // one split's partials
   double best = 1e300;
   int best_s = 1;
   for (int S = 1; S <= 16 && S <= groups; ++S) {
     const int gps = (groups + S - 1) / S;
     if ((S - 1) * gps >= groups) continue;
-    const int units = tiles * S;
+    const int units = tiles * pl.chunks * S;
     const int waves = (units + num_sms - 1) / num_sms;
-    const double cost = (double)waves * gps + (S > 1 ? 2.0 : 0.0);
+    const double cost = waves * (gps * t_group + t_unit) + (S > 1 ? 2.0 + S * part_mb / 3.0 : 0.0);
     if (cost < best - 1e-9) {
       best = cost;
       best_s = S;
@@ -787,7 +810,7 @@ TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
   }
   pl.S = best_s;
   pl.kbs = 2 * ((groups + pl.S - 1) / pl.S);
-  pl.units = tiles * pl.S;
+  pl.units = tiles * pl.chunks * pl.S;
   pl.grid = pl.units < num_sms ? pl.units : num_sms;
   int smem = 0;
   switch (pl.mpad) {
@@ -805,8 +828,7 @@ TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
 }
 
 size_t tc_workspace_floats(const TcPlan& p, int M, int N) {
-  const int rows = M < p.rows ? M : p.rows;   // chunks run one after another and share it
-  return p.S > 1 ? static_cast<size_t>(p.S) * rows * ((N + 15) / 16 * 16) : 0;
+  return p.S > 1 ? static_cast<size_t>(p.S) * M * ((N + 15) / 16 * 16) : 0;
 }
 
 size_t tc_counters(const TcPlan& p, int N) {
@@ -816,34 +838,20 @@ size_t tc_counters(const TcPlan& p, int N) {
 }
 
 size_t tc_x_f16_bytes(int fmt, int M, int K) {
-  return fmt == 1 ? (size_t)M * K * 2 + 256 * sizeof(float) : 0;
+  return fmt == 1 ? (size_t)M * K * 2 + (size_t)M * sizeof(float) : 0;
 }
 
-// NVFP4 first rescales all M rows into FP16 (one launch); then each chunk of
-// pl.rows activation rows is one launch that reads its slice of x and writes
-// its slice of y (plus, when K is split, one reduction launch).  Chunks are
-// stream-ordered, so they share the split-K partials.
+// NVFP4 first rescales all M rows into FP16 (one launch); then one launch of
+// the tensor-core kernel covers every chunk of rows (plus, when K is split,
+// one reduction launch).
 cudaError_t launch_tc(const TcPlan& pl, const GemmArgs& a, void* xf16_scratch, cudaStream_t st) {
-  const uint8_t* xsrc = static_cast<const uint8_t*>(a.x);
-  float* rm = nullptr;
-  if (a.fmt == 1) {
-    __half* xh = static_cast<__half*>(xf16_scratch);
-    rm = reinterpret_cast<float*>(static_cast<uint8_t*>(xf16_scratch) + (size_t)a.M * a.K * 2);
-    prep_x_f16_kernel<<<a.M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x), xh, rm, a.K);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    xsrc = reinterpret_cast<const uint8_t*>(xh);
-  }
-  for (int m0 = 0; m0 < a.M; m0 += pl.rows) {
-    GemmArgs c = a;
-    c.M = min(pl.rows, a.M - m0);
-    c.y = static_cast<uint8_t*>(a.y) + (size_t)m0 * a.N * 2;
-    const uint8_t* xc = xsrc + (size_t)m0 * a.K * 2;   // BF16 and FP16 rows are both 2K bytes
-    const cudaError_t e = a.fmt == 0 ? launch_fmt<0>(pl, c, xc, nullptr, st)
-                                     : launch_fmt<1>(pl, c, xc, rm + m0, st);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  if (a.fmt == 0) return launch_fmt<0>(pl, a, a.x, nullptr, st);
+  __half* xh = static_cast<__half*>(xf16_scratch);
+  float* rm = reinterpret_cast<float*>(static_cast<uint8_t*>(xf16_scratch) + (size_t)a.M * a.K * 2);
+  prep_x_f16_kernel<<<a.M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x), xh, rm, a.K);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_fmt<1>(pl, a, xh, rm, st);
 }
 
 }  // namespace w4

@@ -24,7 +24,7 @@ OK = 0
 ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_DEVICE, ERR_CUDA, ERR_TIMEOUT, ERR_NOMEM = -1, -2, -3, -4, -5, -6, -7
 ERR_SCRATCH = -8
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
-MAX_M = 256
+MAX_M = 8192
 
 _lib = None
 

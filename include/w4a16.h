@@ -68,19 +68,20 @@ extern "C" {
 #define W4A16_ERR_SCRATCH (-8) /* w4a16_gemm_noalloc: the problem needs more than its fixed scratch */
 
 /* Limits of this version. */
-#define W4A16_MAX_M 256        /* decode, speculative verify and small prefill batches */
+#define W4A16_MAX_M 8192       /* decode, speculative verify and prefill chunks */
 
 /* Kernel paths (for w4a16_gemm_path / w4a16_gemm_ex). */
 #define W4A16_PATH_AUTO 0      /* row-count dispatch */
 #define W4A16_PATH_GEMV 1      /* weight-streaming split-K GEMV (mma.sync fragments), M <= 16 */
-#define W4A16_PATH_TC 2        /* tcgen05 tensor-core path (A in tensor memory), M <= 256 */
+#define W4A16_PATH_TC 2        /* tcgen05 tensor-core path (A in tensor memory), M <= 8192 */
 #define W4A16_GEMV_MAX_M 16
 
 /*
- * Shape rules: 1 <= M <= 256; N >= 1 (any value; packed buffers are padded to
- * a multiple of 16 rows); K >= 128 and K a multiple of 128 (both formats).
- * The tensor-core path runs M > 128 as two launches of about M/2 rows each
- * (every launch streams the whole weight matrix once).
+ * Shape rules: 1 <= M <= 8192; N >= 1 (any value; packed buffers are padded
+ * to a multiple of 16 rows); K >= 128 and K a multiple of 128 (both formats).
+ * The tensor-core path splits M > 128 into ceil(M / 128) chunks of equal row
+ * counts inside one launch (beyond M = 128 the tensor cores, not HBM, set the
+ * time).
  */
 
 /* Bytes of the packed weight buffer: ceil(N/16)*16 * K / 2.  0 on bad args. */
@@ -129,7 +130,7 @@ int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packe
  *   global_scale: NVFP4: device pointer to one fp32 g; INT4: must be NULL.
  *   y_bf16:   device, [M][N] BF16 row-major; must not overlap any input.
  * Picks the kernel by row count (W4A16_PATH_AUTO): the split-K GEMV for
- * M <= 8, and for 9 <= M <= 16 when the format is NVFP4 or N >= 8192; the
+ * M <= 8, and for 9 <= M <= 16 when the format is NVFP4 or N >= 16384; the
  * tensor-core path otherwise.  w4a16_gemm_path() reports the choice.
  */
 int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,

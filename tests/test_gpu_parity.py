@@ -143,7 +143,8 @@ def test_gemm_parity_small(fmt, M, N, K, seed):
 
 ROW_COUNTS = [(W.PATH_GEMV, M) for M in (1, 2, 3, 4, 5, 7, 8, 9, 12, 15, 16)] + \
              [(W.PATH_TC, M) for M in (1, 2, 8, 9, 15, 16, 17, 24, 31, 32, 33, 48, 63, 64,
-                                       65, 80, 96, 111, 112, 127, 128, 129, 160, 200, 255, 256)]
+                                       65, 80, 96, 111, 112, 127, 128, 129, 160, 200, 255, 256,
+                                       383, 385, 1000, 4096, 8192)]
 
 
 @pytest.mark.parametrize("path,M", ROW_COUNTS)
@@ -158,7 +159,8 @@ def test_gemm_parity_every_row_count(path, M):
 @pytest.mark.parametrize("path,M", [(W.PATH_GEMV, 1), (W.PATH_GEMV, 8), (W.PATH_GEMV, 9),
                                     (W.PATH_GEMV, 16), (W.PATH_TC, 1), (W.PATH_TC, 9),
                                     (W.PATH_TC, 33), (W.PATH_TC, 64), (W.PATH_TC, 80),
-                                    (W.PATH_TC, 128), (W.PATH_TC, 129), (W.PATH_TC, 256)])
+                                    (W.PATH_TC, 128), (W.PATH_TC, 129), (W.PATH_TC, 256),
+                                    (W.PATH_TC, 1000)])
 def test_gemm_parity_every_row_count_nvfp4(path, M):
     fmt, N, K = "nvfp4", 208, 1280
     p = synth.problem(fmt, 200 + M, M, N, K)
@@ -174,7 +176,8 @@ FULL = ([("int4", name, 1, SEEDS[name]) for name in SHAPES] +
         [("int4", name, M, 5) for name in ("qkv", "o", "gate_up", "down") for M in (2, 4, 9, 16, 64)] +
         [("nvfp4", name, M, 6) for name in ("qkv", "o", "gate_up", "down") for M in (1, 9, 64)] +
         [("int4", name, M, 7) for name in ("gate_up", "down") for M in (128, 200, 256)] +
-        [("nvfp4", name, M, 7) for name in ("o", "gate_up") for M in (96, 256)])
+        [("nvfp4", name, M, 7) for name in ("o", "gate_up") for M in (96, 256)] +
+        [("int4", "gate_up", 1024, 8), ("nvfp4", "down", 640, 8)])
 
 
 @pytest.mark.parametrize("fmt,name,M,seed", FULL)

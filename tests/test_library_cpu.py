@@ -140,7 +140,7 @@ def test_host_pack_rejects_out_of_range():
 def test_argument_validation_before_any_device_call():
     x = w = s = y = 1 << 20          # fake, aligned, never dereferenced
     assert W.w4a16_gemm(0, 0, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE       # M = 0
-    assert W.w4a16_gemm(0, 257, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE     # M > 256
+    assert W.w4a16_gemm(0, 8193, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE    # M > 8192
     assert W.w4a16_gemm_ex(W.PATH_GEMV, 0, 17, 16, 128, x, w, s, None, y, 0) == W.ERR_SHAPE
     assert W.w4a16_gemm(0, 1, 16, 100, x, w, s, None, y, 0) == W.ERR_SHAPE       # K % 128
     assert W.w4a16_gemm(0, 1, 0, 128, x, w, s, None, y, 0) == W.ERR_SHAPE        # N = 0
@@ -162,10 +162,12 @@ def test_dispatcher_path_table():
     assert W.w4a16_gemm_path(0, 1, 17408, 5120) == W.PATH_GEMV
     assert W.w4a16_gemm_path(0, 8, 5120, 6144) == W.PATH_GEMV
     assert W.w4a16_gemm_path(0, 9, 5120, 6144) == W.PATH_TC      # narrow int4 layer
+    assert W.w4a16_gemm_path(0, 16, 8192, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 16, 34816, 5120) == W.PATH_GEMV  # wide int4 layer
     assert W.w4a16_gemm_path(1, 16, 5120, 17408) == W.PATH_GEMV  # NVFP4
     assert W.w4a16_gemm_path(0, 17, 34816, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 64, 34816, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 65, 5120, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(1, 256, 17408, 5120) == W.PATH_TC
-    assert W.w4a16_gemm_path(0, 257, 5120, 5120) == W.ERR_SHAPE
+    assert W.w4a16_gemm_path(0, 8192, 5120, 5120) == W.PATH_TC
+    assert W.w4a16_gemm_path(0, 8193, 5120, 5120) == W.ERR_SHAPE
