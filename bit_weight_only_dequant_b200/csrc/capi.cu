@@ -132,14 +132,15 @@ int check_fmt_shape(int fmt, int N, int K) {
 // Row-count dispatch: the weight-streaming GEMV while the activations are a
 // thin n8 operand, the tcgen05 path once the tensor cores carry real work.
 // The crossovers come from back-to-back timings of both paths on the decode
-// shapes (B200): the GEMV wins up to M = 8 everywhere and at M = 9..16 for
-// NVFP4 and for the widest int4 layer (N >= 16384: enough 16-row bands per
-// SM); the tensor-core path wins for the other int4 layers at M >= 9 and
-// everywhere at M > 16.
+// shapes (B200), the same for both formats: the GEMV wins up to M = 8
+// everywhere and at M = 9..16 for the widest layer (N >= 16384: enough
+// 16-row bands per SM); the tensor-core path wins for the other layers at
+// M >= 9 and everywhere at M > 16.
 int choose_path(int fmt, int M, int N, int K) {
+  (void)fmt;
   (void)K;
   if (M <= 8) return W4A16_PATH_GEMV;
-  if (M <= W4A16_GEMV_MAX_M && (fmt == W4A16_FMT_NVFP4_G16 || N >= 16384)) return W4A16_PATH_GEMV;
+  if (M <= W4A16_GEMV_MAX_M && N >= 16384) return W4A16_PATH_GEMV;
   return W4A16_PATH_TC;
 }
 

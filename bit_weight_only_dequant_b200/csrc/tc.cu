@@ -602,13 +602,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // Per-row power-of-two rescaling of the activations into FP16 (NVFP4 path):
-// row_mul[m] = 2^e with max|x[m]| * 2^-e in [2^14, 2^15).
-__global__ void prep_x_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* __restrict__ xh,
-                                  float* __restrict__ row_mul, int K) {
+// row_mul[m] = 2^e with max|x[m]| * 2^-e in [2^14, 2^15).  One CTA per row,
+// eight BF16 values per 16-byte load; the second pass re-reads the row from
+// cache.  K is a multiple of 128, so rows are 16-byte aligned.
+__global__ void __launch_bounds__(256) prep_x_f16_kernel(const __nv_bfloat16* __restrict__ x,
+                                                         __half* __restrict__ xh,
+                                                         float* __restrict__ row_mul, int K) {
   const int m = blockIdx.x;
-  const __nv_bfloat16* row = x + (size_t)m * K;
+  const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)m * K);
+  uint4* out = reinterpret_cast<uint4*>(xh + (size_t)m * K);
+  const int n8 = K >> 3;
   float mx = 0.f;
-  for (int k = threadIdx.x; k < K; k += blockDim.x) mx = fmaxf(mx, fabsf(__bfloat162float(row[k])));
+  for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+    const uint4 v = __ldg(row + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[j] << 16)));
+      mx = fmaxf(mx, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+    }
+  }
   __shared__ float red[32];
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -625,8 +638,23 @@ __global__ void prep_x_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* _
   int e = 0;
   if (mx > 0.f && isfinite(mx)) e = ilogbf(mx) - 14;
   if (threadIdx.x == 0) row_mul[m] = ldexpf(1.f, e);
-  for (int k = threadIdx.x; k < K; k += blockDim.x)
-    xh[(size_t)m * K + k] = __float2half_rn(ldexpf(__bfloat162float(row[k]), -e));
+  // x * 2^-e is one exact scaling: a single multiply when 2^-e is a normal
+  // float, ldexpf otherwise (rows whose largest magnitude is below 2^-112)
+  const bool direct = e >= -126 && e <= 126;
+  const float sc = direct ? __int_as_float((127 - e) << 23) : 0.f;
+  for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+    const uint4 v = __ldg(row + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(w[j] << 16), hi = __uint_as_float(w[j] & 0xFFFF0000u);
+      const __half hl = __float2half_rn(direct ? lo * sc : ldexpf(lo, -e));
+      const __half hh = __float2half_rn(direct ? hi * sc : ldexpf(hi, -e));
+      o[j] = (uint32_t)__half_as_ushort(hl) | ((uint32_t)__half_as_ushort(hh) << 16);
+    }
+    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
 }
 
 // Split-K reduction: y[m][n] = BF16(sum over splits, in split order, of the

@@ -130,8 +130,8 @@ int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packe
  *   global_scale: NVFP4: device pointer to one fp32 g; INT4: must be NULL.
  *   y_bf16:   device, [M][N] BF16 row-major; must not overlap any input.
  * Picks the kernel by row count (W4A16_PATH_AUTO): the split-K GEMV for
- * M <= 8, and for 9 <= M <= 16 when the format is NVFP4 or N >= 16384; the
- * tensor-core path otherwise.  w4a16_gemm_path() reports the choice.
+ * M <= 8, and for 9 <= M <= 16 when N >= 16384; the tensor-core path
+ * otherwise.  w4a16_gemm_path() reports the choice.
  */
 int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
                const void* packed_scales, const float* global_scale, void* y_bf16, void* stream);

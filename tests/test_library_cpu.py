@@ -164,7 +164,8 @@ def test_dispatcher_path_table():
     assert W.w4a16_gemm_path(0, 9, 5120, 6144) == W.PATH_TC      # narrow int4 layer
     assert W.w4a16_gemm_path(0, 16, 8192, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 16, 34816, 5120) == W.PATH_GEMV  # wide int4 layer
-    assert W.w4a16_gemm_path(1, 16, 5120, 17408) == W.PATH_GEMV  # NVFP4
+    assert W.w4a16_gemm_path(1, 16, 5120, 17408) == W.PATH_TC    # NVFP4, narrow layer
+    assert W.w4a16_gemm_path(1, 16, 34816, 5120) == W.PATH_GEMV  # NVFP4, wide layer
     assert W.w4a16_gemm_path(0, 17, 34816, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 64, 34816, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 65, 5120, 5120) == W.PATH_TC
