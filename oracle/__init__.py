@@ -11,7 +11,8 @@ What it computes (plain definitions, no blocking, no fusion):
   BF16 from an exact binary64 value.
 * ``w4a16``: dequantisation of the two checkpoint formats into BF16 weights
   (one rounding of the exact product), then y = x . W_deq^T accumulated in
-  fp64, plus the per-element tolerance bound sum_k |W_deq[n][k] * x[m][k]|.
+  fp64, plus the per-element tolerance bound sum_k |W_deq[n][k] * x[m][k]|;
+  and the fused gate/up layer h = SiLU(gate) * up with its tolerance.
 
 It works from the *logical* tensors (int8 q or uint8 codes, [N][K]; scales per
 output column and K-group) and never from the library's packed layout, so it
@@ -25,6 +26,9 @@ from .w4a16 import (  # noqa: F401
     gemm_ref,
     abs_bound,
     within_tolerance,
+    silu,
+    gate_up_silu_ref,
+    gate_up_silu_allowed,
     TOL_REL,
     TOL_ABS,
 )

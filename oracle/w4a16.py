@@ -24,6 +24,13 @@ speed is set by the bytes of weights streamed per token.
 
 Accuracy contract: per element |y - y_ref| <= 2**-7 * sum_k |W_deq[n][k] *
 x[m][k]| + 1e-3, and exported dequantised weights bit-exact.
+
+Fused gate/up projection (the MLP of every layer, named on the pages only as
+"MLP" linears: model card "Qwen3.8 27B - NVFP4 for veloGB10", section
+"Specifications"; guide "Qwen3.8-27B on DGX Spark (GB10)", section "What
+Spark-native means").  Reading, the plainest one for this model family: the
+packed [2I][K] weight holds the gate rows first and the up rows second, and
+the layer's output is h = SiLU(gate) * up with SiLU(z) = z / (1 + e^-z).
 """
 
 from __future__ import annotations
@@ -105,3 +112,54 @@ def within_tolerance(y: np.ndarray, y_ref: np.ndarray, bound: np.ndarray):
     allowed = TOL_REL * bound + TOL_ABS
     err = np.abs(np.asarray(y, dtype=np.float64) - y_ref)
     return err <= allowed, err / allowed
+
+
+# ---------------------------------------------------------------- fused gate/up + SiLU
+
+SILU_LIPSCHITZ = 1.1   # max over z of |d/dz (z * sigmoid(z))| is 1.0998...
+
+
+def silu(z: np.ndarray) -> np.ndarray:
+    """SiLU(z) = z * sigmoid(z) = z / (1 + exp(-z)), binary64, elementwise.
+
+    exp(-z) overflows to +inf for z < -709; z / inf is then -0.0, the limit.
+    """
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def gate_up_silu_ref(x_bits: np.ndarray, w_bits: np.ndarray):
+    """h[m][i] = SiLU(gate[m][i]) * up[m][i] in binary64 (unrounded).
+
+    w_bits: BF16 [2I][K], gate rows [0, I), up rows [I, 2I).  gate and up are
+    the exact products of gemm_ref.  Returns (h, gate, up), float64 [M][I].
+    """
+    N = w_bits.shape[0]
+    if N % 2:
+        raise ValueError("the fused gate/up weight has an even number of rows")
+    I = N // 2
+    y = gemm_ref(x_bits, w_bits)
+    gate, up = y[:, :I], y[:, I:]
+    return silu(gate) * up, gate, up
+
+
+def gate_up_silu_allowed(x_bits: np.ndarray, w_bits: np.ndarray, gate: np.ndarray,
+                         up: np.ndarray) -> np.ndarray:
+    """Allowed |h - h_ref| per element for the fused output.
+
+    Each of gate and up may carry the matmul's own error e = 2^-7 * sum_k
+    |W_deq x| + 1e-3.  SiLU is 1.1-Lipschitz, so |SiLU(g') u' - SiLU(g) u| <=
+    (|SiLU(g)| + 1.1 e_g) e_u + 1.1 e_g |u|; the BF16 rounding of the output
+    and the fp32 evaluation of SiLU add at most 2^-7 |h| (RNE onto BF16 alone
+    is 2^-8 relative), and 1e-3 absolute covers the rest.
+    """
+    N = w_bits.shape[0]
+    I = N // 2
+    b = abs_bound(x_bits, w_bits)
+    e_g = TOL_REL * b[:, :I] + TOL_ABS
+    e_u = TOL_REL * b[:, I:] + TOL_ABS
+    sg = silu(gate)
+    h = sg * up
+    return ((np.abs(sg) + SILU_LIPSCHITZ * e_g) * e_u + SILU_LIPSCHITZ * e_g * np.abs(up)
+            + TOL_REL * np.abs(h) + TOL_ABS)

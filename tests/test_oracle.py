@@ -363,3 +363,70 @@ def test_pins_catch_planted_mistakes():
     assert "sign" in _pin_suite(offset_sign, oracle.gemm_ref)
     assert "matmul" in _pin_suite(oracle.dequant_int4_g128, transposed)
     assert "matmul" in _pin_suite(oracle.dequant_int4_g128, dropped_term)
+
+
+# ---------------------------------------------------------------- fused gate/up + SiLU
+
+
+def test_silu_closed_forms():
+    import math
+    s = oracle.silu(np.array([0.0, 1.0, -1.0, 2.0, 50.0, -50.0, -800.0, 800.0]))
+    # sigmoid(1) = e / (1 + e), sigmoid(2) = e^2 / (1 + e^2): textbook values
+    assert s[0] == 0.0
+    assert abs(s[1] - 0.7310585786300049) <= 1e-16
+    assert abs(s[2] - (-0.2689414213699951)) <= 1e-16
+    assert abs(s[3] - 2 * math.e ** 2 / (1 + math.e ** 2)) <= 1e-15   # a few ulps
+    assert s[4] == 50.0                                  # sigmoid(50) rounds to 1
+    assert abs(s[5]) < 1e-19 and s[5] < 0                # -50 * e^-50
+    assert s[6] == 0.0 and np.signbit(s[6])              # the limit, no NaN from inf / inf
+    assert s[7] == 800.0
+    # SiLU(z) - SiLU(-z) = z: sigmoid(z) + sigmoid(-z) = 1
+    z = np.linspace(-30, 30, 121)
+    assert np.allclose(oracle.silu(z) - oracle.silu(-z), z, rtol=0, atol=1e-13)
+
+
+def _silu_brute(x_bits, w_bits):
+    """h by pure-Python loops from the formats' bit fields and math.exp."""
+    import math
+    M, K = x_bits.shape
+    N = w_bits.shape[0]
+    I = N // 2
+    ex = _exact_y(x_bits, w_bits)
+    out = []
+    for m in range(M):
+        row = []
+        for i in range(I):
+            g, u = float(ex[m][i]), float(ex[m][I + i])
+            row.append(g / (1.0 + math.exp(-g)) * u if g > -700 else 0.0 * u)
+        out.append(row)
+    return out
+
+
+@pytest.mark.parametrize("fmt,M,I,K,seed", [("int4", 2, 3, 128, 31), ("nvfp4", 3, 2, 256, 32)])
+def test_gate_up_silu_brute_force(fmt, M, I, K, seed):
+    p = synth.problem(fmt, seed, M, 2 * I, K)
+    w = (oracle.dequant_int4_g128(p["codes"], p["scales"]) if fmt == "int4"
+         else oracle.dequant_nvfp4(p["codes"], p["scales"], p["g"]))
+    h, gate, up = oracle.gate_up_silu_ref(p["x"], w)
+    assert h.shape == (M, I) and gate.shape == (M, I) and up.shape == (M, I)
+    ref = _silu_brute(p["x"], w)
+    for m in range(M):
+        for i in range(I):
+            assert abs(h[m, i] - ref[m][i]) <= 1e-12 * max(1.0, abs(ref[m][i]))
+
+
+def test_gate_up_silu_layout_and_tolerance():
+    p = synth.problem("int4", 33, 4, 2 * 24, 384)
+    w = oracle.dequant_int4_g128(p["codes"], p["scales"])
+    h, gate, up = oracle.gate_up_silu_ref(p["x"], w)
+    y = oracle.gemm_ref(p["x"], w)
+    # gate rows first, up rows second (not interleaved, not swapped)
+    assert np.array_equal(gate, y[:, :24]) and np.array_equal(up, y[:, 24:])
+    allowed = oracle.gate_up_silu_allowed(p["x"], w, gate, up)
+    assert np.all(allowed > 0)
+    # the exact value and its BF16 rounding pass
+    hb = formats.bf16_to_f64(formats.f64_to_bf16_rne(h))
+    assert np.all(np.abs(hb - h) <= allowed)
+    # plausible mistakes fail: halves swapped, SiLU on the wrong half, SiLU left out
+    for wrong in (oracle.silu(up) * gate, gate * up, oracle.silu(gate) * gate):
+        assert np.any(np.abs(wrong - h) > allowed)
