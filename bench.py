@@ -330,6 +330,41 @@ def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
             "frac_of_8TBps": round(b / us / 1e3 / 8000.0, 4)}
 
 
+def gate_up_entry(fmt, M, seed, peaks, stream, reps=24):
+    """The fused gate/up layer h = SiLU(gate) * up at the decode gate/up shape
+    (K = 5120, I = 17408: the 34816-row weight), back to back like the sweep.
+    Algorithmic bytes: the weight and scales, x, and h (M x I BF16)."""
+    import torch
+    from bit_weight_only_dequant_b200 import w4a16 as W
+    f = W.FMTS[fmt]
+    K, N = 5120, 34816
+    I = N // 2
+    wbytes = W.w4a16_packed_weight_bytes(f, N, K) + W.w4a16_packed_scale_bytes(f, N, K)
+    ws = make_weights(fmt, seed, N, K, copies_for(wbytes))
+    x = make_x(fmt, seed, M, K)
+    h = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
+    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
+    path = W.w4a16_gemm_path(f, M, N, K)
+
+    def launch(r, ws=ws):
+        pw, ps = ws[r % len(ws)]
+        W.check(W.w4a16_gemm_gate_up_silu(f, M, I, K, x, pw, ps, g, h, stream.cuda_stream),
+                "gate_up_silu")
+
+    with torch.cuda.stream(stream):
+        for r in range(3):
+            launch(r)
+    torch.cuda.synchronize()
+    us = time_back_to_back(launch, reps, stream) * 1e3
+    b = alg_bytes(fmt, M, N, K) - 2 * M * N + 2 * M * I
+    fl = flops(M, N, K)
+    t_roof = max(b / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+    del ws
+    torch.cuda.empty_cache()
+    return {"fmt": fmt, "M": M, "K": K, "I": I, "path": int(path), "us": round(us, 3),
+            "GBps": round(b / us / 1e3, 1), "frac_roofline": round(t_roof * 1e6 / us, 4)}
+
+
 def whole_stack(Ms, peaks, stream, reps=3):
     """64 layers x (QKV, O, gate/up, down) + the 5120->248320 output projection,
     int4 g128, weights of layer l drawn with seed 7+l and the output projection
@@ -533,6 +568,10 @@ def run_native(args, rank, world, local_rank):
         for fmt, n, K, N, Mv, s in target + cfg2 + cfg3 + cfg4 + cfg5:
             entries.append(sweep_entry(fmt, n, K, N, Mv, s, peaks, stream))
         extra["sweep"] = entries
+        extra["gate_up_silu"] = [gate_up_entry(fmt, Mv, 3, peaks, stream)
+                                 for fmt, Mv in (("int4", 1), ("int4", 4), ("int4", 9),
+                                                 ("int4", 16), ("int4", 64), ("int4", 256),
+                                                 ("nvfp4", 1), ("nvfp4", 64))]
     if world == 1 and not args.no_stack:
         extra["whole_stack"] = whole_stack((1, 16, 64), peaks, stream)
 

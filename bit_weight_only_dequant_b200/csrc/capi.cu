@@ -32,9 +32,10 @@ std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 // Plans depend only on (format, M, N, K) and the SM count: computed once per
 // shape and device (a decode step calls the same few shapes every token).
 struct PlanKey {
-  int dev, fmt, M, N, K;
+  int dev, fmt, M, N, K, fuse;
   bool operator<(const PlanKey& o) const {
     if (dev != o.dev) return dev < o.dev;
+    if (fuse != o.fuse) return fuse < o.fuse;
     if (fmt != o.fmt) return fmt < o.fmt;
     if (M != o.M) return M < o.M;
     if (N != o.N) return N < o.N;
@@ -44,22 +45,22 @@ struct PlanKey {
 std::map<PlanKey, w4::GemvPlan> g_gemv_plans;
 std::map<PlanKey, w4::TcPlan> g_tc_plans;
 
-w4::GemvPlan cached_gemv_plan(int dev, int fmt, int M, int N, int K, int num_sms) {
-  const PlanKey key{dev, fmt, M, N, K};
+w4::GemvPlan cached_gemv_plan(int dev, int fmt, int M, int N, int K, int num_sms, int fuse) {
+  const PlanKey key{dev, fmt, M, N, K, fuse};
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_gemv_plans.find(key);
   if (it != g_gemv_plans.end()) return it->second;
-  const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, num_sms);
+  const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, num_sms, fuse);
   if (g_gemv_plans.size() < 4096) g_gemv_plans.emplace(key, pl);
   return pl;
 }
 
-w4::TcPlan cached_tc_plan(int dev, int fmt, int M, int N, int K, int num_sms) {
-  const PlanKey key{dev, fmt, M, N, K};
+w4::TcPlan cached_tc_plan(int dev, int fmt, int M, int N, int K, int num_sms, int fuse) {
+  const PlanKey key{dev, fmt, M, N, K, fuse};
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_tc_plans.find(key);
   if (it != g_tc_plans.end()) return it->second;
-  const w4::TcPlan pl = w4::plan_tc(fmt, M, N, K, num_sms);
+  const w4::TcPlan pl = w4::plan_tc(fmt, M, N, K, num_sms, fuse);
   if (g_tc_plans.size() < 4096) g_tc_plans.emplace(key, pl);
   return pl;
 }
@@ -146,6 +147,62 @@ int choose_path(int fmt, int M, int N, int K) {
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA; }
 
+// The matmul (fuse = 0) or the fused gate/up layer (fuse = 1, N = 2I rows,
+// y = [M][I]) on the chosen path.
+int run_gemm(int path, int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
+             const void* packed_scales, const float* global_scale, void* y_bf16, void* stream,
+             int fuse) {
+  int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (M < 1 || M > W4A16_MAX_M) return W4A16_ERR_SHAPE;
+  if (path != W4A16_PATH_AUTO && path != W4A16_PATH_GEMV && path != W4A16_PATH_TC)
+    return W4A16_ERR_ARG;
+  if (!x_bf16 || !packed_w || !packed_scales || !y_bf16) return W4A16_ERR_ARG;
+  if ((fmt == W4A16_FMT_NVFP4_G16) != (global_scale != nullptr)) return W4A16_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(packed_w) || !aligned16(packed_scales) ||
+      !aligned16(y_bf16))
+    return W4A16_ERR_ALIGN;
+  if (path == W4A16_PATH_AUTO) path = choose_path(fmt, M, N, K);
+  if (path == W4A16_PATH_GEMV && M > W4A16_GEMV_MAX_M) return W4A16_ERR_SHAPE;
+  DeviceState* d = nullptr;
+  if ((r = device_state(&d)) != W4A16_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  w4::GemmArgs a;
+  a.fmt = fmt;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.x = x_bf16;
+  a.w = packed_w;
+  a.s = packed_scales;
+  a.g = global_scale;
+  a.y = y_bf16;
+  a.ws = nullptr;
+  a.counters = nullptr;
+  a.err = d->err;
+  a.fuse = fuse;
+  void* scratch = nullptr;
+  if (path == W4A16_PATH_GEMV) {
+    const w4::GemvPlan pl = cached_gemv_plan(d->dev, fmt, M, N, K, d->num_sms, fuse);
+    if (pl.S == 0) return W4A16_ERR_SHAPE;
+    const size_t nf = w4::gemv_workspace_floats(pl, M, N);
+    if (nf > 0) {
+      r = workspace(st, w4::gemv_counters(pl, N), nf, 0, &a.counters, &a.ws, &scratch);
+      if (r != W4A16_OK) return r;
+    }
+    return status_of(w4::launch_gemv(pl, a, st));
+  }
+  const w4::TcPlan pl = cached_tc_plan(d->dev, fmt, M, N, K, d->num_sms, fuse);
+  const size_t nf = w4::tc_workspace_floats(pl, M, N);
+  const size_t nb = w4::tc_x_f16_bytes(fmt, M, K);
+  if (nf > 0 || nb > 0) {
+    r = workspace(st, w4::tc_counters(pl, N), nf, nb, &a.counters, &a.ws, &scratch);
+    if (r != W4A16_OK) return r;
+  }
+  return status_of(w4::launch_tc(pl, a, scratch, st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -215,54 +272,23 @@ int w4a16_gemm_path(int fmt, int M, int N, int K) {
 int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
                   const void* packed_scales, const float* global_scale, void* y_bf16,
                   void* stream) {
-  int r = check_fmt_shape(fmt, N, K);
-  if (r != W4A16_OK) return r;
-  if (M < 1 || M > W4A16_MAX_M) return W4A16_ERR_SHAPE;
-  if (path != W4A16_PATH_AUTO && path != W4A16_PATH_GEMV && path != W4A16_PATH_TC)
-    return W4A16_ERR_ARG;
-  if (!x_bf16 || !packed_w || !packed_scales || !y_bf16) return W4A16_ERR_ARG;
-  if ((fmt == W4A16_FMT_NVFP4_G16) != (global_scale != nullptr)) return W4A16_ERR_ARG;
-  if (!aligned16(x_bf16) || !aligned16(packed_w) || !aligned16(packed_scales) ||
-      !aligned16(y_bf16))
-    return W4A16_ERR_ALIGN;
-  if (path == W4A16_PATH_AUTO) path = choose_path(fmt, M, N, K);
-  if (path == W4A16_PATH_GEMV && M > W4A16_GEMV_MAX_M) return W4A16_ERR_SHAPE;
-  DeviceState* d = nullptr;
-  if ((r = device_state(&d)) != W4A16_OK) return r;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return run_gemm(path, fmt, M, N, K, x_bf16, packed_w, packed_scales, global_scale, y_bf16,
+                  stream, 0);
+}
 
-  w4::GemmArgs a;
-  a.fmt = fmt;
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.x = x_bf16;
-  a.w = packed_w;
-  a.s = packed_scales;
-  a.g = global_scale;
-  a.y = y_bf16;
-  a.ws = nullptr;
-  a.counters = nullptr;
-  a.err = d->err;
-  void* scratch = nullptr;
-  if (path == W4A16_PATH_GEMV) {
-    const w4::GemvPlan pl = cached_gemv_plan(d->dev, fmt, M, N, K, d->num_sms);
-    if (pl.S == 0) return W4A16_ERR_SHAPE;
-    const size_t nf = w4::gemv_workspace_floats(pl, M, N);
-    if (nf > 0) {
-      r = workspace(st, w4::gemv_counters(pl, N), nf, 0, &a.counters, &a.ws, &scratch);
-      if (r != W4A16_OK) return r;
-    }
-    return status_of(w4::launch_gemv(pl, a, st));
-  }
-  const w4::TcPlan pl = cached_tc_plan(d->dev, fmt, M, N, K, d->num_sms);
-  const size_t nf = w4::tc_workspace_floats(pl, M, N);
-  const size_t nb = w4::tc_x_f16_bytes(fmt, M, K);
-  if (nf > 0 || nb > 0) {
-    r = workspace(st, w4::tc_counters(pl, N), nf, nb, &a.counters, &a.ws, &scratch);
-    if (r != W4A16_OK) return r;
-  }
-  return status_of(w4::launch_tc(pl, a, scratch, st));
+int w4a16_gemm_gate_up_silu_ex(int path, int fmt, int M, int I, int K, const void* x_bf16,
+                               const void* packed_w, const void* packed_scales,
+                               const float* global_scale, void* h_bf16, void* stream) {
+  if (I < 16 || I % 16 != 0 || I > (1 << 29)) return W4A16_ERR_SHAPE;
+  return run_gemm(path, fmt, M, 2 * I, K, x_bf16, packed_w, packed_scales, global_scale, h_bf16,
+                  stream, 1);
+}
+
+int w4a16_gemm_gate_up_silu(int fmt, int M, int I, int K, const void* x_bf16,
+                            const void* packed_w, const void* packed_scales,
+                            const float* global_scale, void* h_bf16, void* stream) {
+  return w4a16_gemm_gate_up_silu_ex(W4A16_PATH_AUTO, fmt, M, I, K, x_bf16, packed_w,
+                                    packed_scales, global_scale, h_bf16, stream);
 }
 
 int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,

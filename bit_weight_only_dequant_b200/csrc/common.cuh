@@ -184,3 +184,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 }  // namespace w4
+
+
+// SiLU(z) = z * sigmoid(z) = z / (1 + e^-z) in fp32 for the fused gate/up
+// epilogues: the hardware exponential and a correctly rounded reciprocal
+// (relative error a few 1e-6, far inside the layer's tolerance).  e^-z
+// overflows to +inf for z below about -88, and z * (1 / inf) is -0, the limit.
+__device__ __forceinline__ float silu_f32(float z) { return z * __frcp_rn(1.f + __expf(-z)); }

@@ -60,10 +60,10 @@ __host__ __device__ constexpr int stage_bytes(int fmt) { return kGroupBytes + (f
 // rematerialises the conversion constants in the loop, and the ring, not the
 // warp count, keeps the bytes in flight (measured: 16 warps are ~20% faster
 // at M = 1).
-template <int FMT, int MT>
+template <int FMT, int MT, bool FUSE = false>
 struct Cfg {
   static constexpr int kWarps = 16;
-  static constexpr int kRedBytes = kWarps * 32 * 4 * MT * 4;  // per-lane partial sums
+  static constexpr int kRedBytes = kWarps * 32 * 4 * MT * 4 * (FUSE ? 2 : 1);  // per-lane partial sums
   static constexpr int kHeader = (kRedOff + kRedBytes + 127) / 128 * 128;
   static constexpr int kCache = 4;                              // staging chunks in registers
 };
@@ -81,7 +81,12 @@ struct Params {
   int bq, br;                                      // bands per CTA: bq, plus one for the first br
   int wn, wn_log2, wk_log2;                        // warp grid: wn bands x 2^wk_log2 pieces
   int ngp;                                         // groups per piece, padded to the ring depth
+  // fused gate/up layer: bands index the I gate rows; the up band of gate
+  // band b lies up_w (weights) and up_s (scales) bytes further; y is [M][I]
+  int I;
+  size_t up_w, up_s;
 };
+
 
 // Programmatic dependent launch: let the next kernel on the stream start its
 // prologue, and wait for the previous one before touching data it may write.
@@ -293,12 +298,14 @@ __device__ __forceinline__ void block_nvfp4(uint4 wv, uint2 sv, const uint8_t* c
   }
 }
 
-template <int FMT, int MT>
+template <int FMT, int MT, bool FUSE>
 __device__ __forceinline__ void band_epilogue(const Params& p, int band, int split, int lane,
-                                              const float* row_mul, const float (*vals)[4]) {
+                                              const float* row_mul, const float (*vals)[4],
+                                              const float (*vals_u)[4]) {
   const int g = lane >> 2, t = lane & 3;
   const float gmul = FMT == 1 ? __ldg(p.g) : 1.f;
   const int n0 = band * 16 + g;
+  const int cols = FUSE ? p.I : p.N;             // output columns (row stride of y)
   if (p.S == 1) {
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
@@ -306,19 +313,27 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
       for (int i = 0; i < 4; ++i) {
         const int m = mt * 8 + 2 * t + (i & 1);
         const int n = n0 + 8 * (i >> 1);
-        if (m < p.M && n < p.N)
-          p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(vals[mt][i] * row_mul[m] * gmul);
+        if (m < p.M && n < cols) {
+          float v = vals[mt][i] * row_mul[m] * gmul;
+          if (FUSE) v = silu_f32(v) * (vals_u[mt][i] * row_mul[m] * gmul);
+          p.y[(size_t)m * cols + n] = __float2bfloat16_rn(v);
+        }
       }
     return;
   }
-  const size_t Npad = (size_t)p.NT * 16;
+  // partials [S][M][Npad]: fused, gate row n and up row I + n
+  const size_t Npad = FUSE ? (size_t)2 * p.I : (size_t)p.NT * 16;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int m = mt * 8 + 2 * t + (i & 1);
       const int n = n0 + 8 * (i >> 1);
-      if (m < p.M) __stcg(p.ws + ((size_t)split * p.M + m) * Npad + n, vals[mt][i] * row_mul[m]);
+      if (m < p.M) {
+        float* dst = p.ws + ((size_t)split * p.M + m) * Npad + n;
+        __stcg(dst, vals[mt][i] * row_mul[m]);
+        if (FUSE) __stcg(dst + p.I, vals_u[mt][i] * row_mul[m]);
+      }
     }
   __threadfence();
   __syncwarp();
@@ -333,20 +348,27 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
     for (int i = 0; i < 4; ++i) {
       const int m = mt * 8 + 2 * t + (i & 1);
       const int n = n0 + 8 * (i >> 1);
-      if (m < p.M && n < p.N) {
-        float v = 0.f;
-        for (int sp = 0; sp < p.S; ++sp) v += __ldcg(p.ws + ((size_t)sp * p.M + m) * Npad + n);
-        p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(v * gmul);
+      if (m < p.M && n < cols) {
+        float v = 0.f, u = 0.f;
+        for (int sp = 0; sp < p.S; ++sp) {
+          const float* src = p.ws + ((size_t)sp * p.M + m) * Npad + n;
+          v += __ldcg(src);
+          if (FUSE) u += __ldcg(src + p.I);
+        }
+        v *= gmul;
+        if (FUSE) v = silu_f32(v) * (u * gmul);
+        p.y[(size_t)m * cols + n] = __float2bfloat16_rn(v);
       }
     }
   if (lane == 0) p.counters[band] = 0u;
 }
 
 
-template <int FMT, int MT, int D>
-__global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(const Params p) {
-  using C = Cfg<FMT, MT>;
-  constexpr int kSB = stage_bytes(FMT);
+template <int FMT, int MT, int D, bool FUSE>
+__global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kernel(const Params p) {
+  using C = Cfg<FMT, MT, FUSE>;
+  constexpr int kSB1 = stage_bytes(FMT);       // one band's group
+  constexpr int kSB = kSB1 * (FUSE ? 2 : 1);   // fused: the gate band's group, then the up band's
   constexpr int kSStep = FMT == 0 ? 32 : 128;  // scale bytes of one band per 128-group
   extern __shared__ __align__(128) uint8_t smem[];
   float* row_mul = reinterpret_cast<float*>(smem);
@@ -405,6 +427,18 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
         cpa8(d + kGroupBytes, cs + k * kSStep);
         cpa8(d + kGroupBytes + 8, cs + k * kSStep + 64);
       }
+      if (FUSE) {
+        const uint8_t* uw = cw + p.up_w + k * kGroupBytes;
+        const uint8_t* us = cs + p.up_s + k * kSStep;
+        cpa16(d + kSB1, uw, pol);
+        cpa16(d + kSB1 + kTileBytes, uw + kTileBytes, pol);
+        if (FMT == 0) {
+          cpa4(d + kSB1 + kGroupBytes - lane * 12, us);
+        } else {
+          cpa8(d + kSB1 + kGroupBytes, us);
+          cpa8(d + kSB1 + kGroupBytes + 8, us + 64);
+        }
+      }
     }
     cpa_commit();
   };
@@ -447,11 +481,11 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
   const uint8_t* slot0 = ring + lane * 16;
 
   for (int r = 0; r < rounds; ++r) {
-    float acc[MT][4];
+    float acc[MT][4], acc_u[MT][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[mt][i] = 0.f;
+      for (int i = 0; i < 4; ++i) acc[mt][i] = acc_u[mt][i] = 0.f;
     const bool active = r < my_rounds;
     const int band = band_lo + wi + r * p.wn;
     if (active) {
@@ -481,6 +515,24 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) xg[mt] += 128;
               block_nvfp4<MT>(cur.w1, cur.s1, xg, acc);
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) xg[mt] -= 128;
+            }
+            if (FUSE) {                 // the up band's group, same activations
+              const uint8_t* su = st + kSB1;
+              GroupWords up;
+              up.w0 = *reinterpret_cast<const uint4*>(su);
+              up.w1 = *reinterpret_cast<const uint4*>(su + kTileBytes);
+              if (FMT == 0) {
+                up.s0.x = *reinterpret_cast<const uint32_t*>(su + kGroupBytes - lane * 12);
+                group_int4<MT>(up, xg, acc_u);
+              } else {
+                const uint4 sv = *reinterpret_cast<const uint4*>(su + kGroupBytes);
+                block_nvfp4<MT>(up.w0, make_uint2(sv.x, sv.y), xg, acc_u);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) xg[mt] += 128;
+                block_nvfp4<MT>(up.w1, make_uint2(sv.z, sv.w), xg, acc_u);
+              }
             }
           }
           copy_item(k);               // refill the slot just read
@@ -489,37 +541,44 @@ __global__ void __launch_bounds__(Cfg<FMT, MT>::kWarps * 32, 1) gemv_kernel(cons
       }
     }
     if (p.wk_log2 == 0) {
-      if (active) band_epilogue<FMT, MT>(p, band, split, lane, row_mul, acc);
+      if (active) band_epilogue<FMT, MT, FUSE>(p, band, split, lane, row_mul, acc, acc_u);
       continue;
     }
     // add the wk pieces of each band in piece order
-    float* mine = red + (warp * 32 + lane) * 4 * MT;
+    constexpr int kLaneFloats = 4 * MT * (FUSE ? 2 : 1);
+    float* mine = red + (warp * 32 + lane) * kLaneFloats;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) mine[mt * 4 + i] = active ? acc[mt][i] : 0.f;
+      for (int i = 0; i < 4; ++i) {
+        mine[mt * 4 + i] = active ? acc[mt][i] : 0.f;
+        if (FUSE) mine[4 * MT + mt * 4 + i] = active ? acc_u[mt][i] : 0.f;
+      }
     __syncthreads();
     if (wj == 0 && active) {
-      float sum[MT][4];
+      float sum[MT][4], sum_u[MT][4];
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) sum[mt][i] = 0.f;
+        for (int i = 0; i < 4; ++i) sum[mt][i] = sum_u[mt][i] = 0.f;
       for (int pc = 0; pc < (1 << p.wk_log2); ++pc) {
-        const float* o = red + ((pc * p.wn + wi) * 32 + lane) * 4 * MT;
+        const float* o = red + ((pc * p.wn + wi) * 32 + lane) * kLaneFloats;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) sum[mt][i] += o[mt * 4 + i];
+          for (int i = 0; i < 4; ++i) {
+            sum[mt][i] += o[mt * 4 + i];
+            if (FUSE) sum_u[mt][i] += o[4 * MT + mt * 4 + i];
+          }
       }
-      band_epilogue<FMT, MT>(p, band, split, lane, row_mul, sum);
+      band_epilogue<FMT, MT, FUSE>(p, band, split, lane, row_mul, sum, sum_u);
     }
     __syncthreads();
   }
   cpa_wait<0>();  // nothing is in flight at exit
 }
 
-template <int FMT, int MT, int D>
+template <int FMT, int MT, int D, bool FUSE>
 cudaError_t launch_d(const Params& p, const GemvPlan& pl, cudaStream_t st) {
   // raise the dynamic shared memory limit once per device (kept out of the
   // steady state so launches can be captured in CUDA graphs)
@@ -528,14 +587,14 @@ cudaError_t launch_d(const Params& p, const GemvPlan& pl, cudaStream_t st) {
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!smem_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MT, D>,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MT, D, FUSE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return e;
     smem_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.ctas_x, pl.S);
-  cfg.blockDim = dim3(Cfg<FMT, MT>::kWarps * 32);
+  cfg.blockDim = dim3(Cfg<FMT, MT, FUSE>::kWarps * 32);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -543,7 +602,7 @@ cudaError_t launch_d(const Params& p, const GemvPlan& pl, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<FMT, MT, D>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<FMT, MT, D, FUSE>, p);
 }
 
 int ilog2(int v) {
@@ -552,7 +611,7 @@ int ilog2(int v) {
   return l;
 }
 
-template <int FMT, int MT>
+template <int FMT, int MT, bool FUSE>
 cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   Params p;
   p.x = static_cast<const __nv_bfloat16*>(a.x);
@@ -566,7 +625,11 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
-  p.NT = (a.N + 15) / 16;
+  p.I = a.N / 2;
+  p.NT = FUSE ? p.I / 16 : (a.N + 15) / 16;    // fused: bands of gate rows
+  const size_t KB = (size_t)a.K / 64;
+  p.up_w = (size_t)(p.I / 16) * KB * kTileBytes;
+  p.up_s = FMT == 0 ? (size_t)(p.I / 16) * (a.K / 128) * 32 : (size_t)(p.I / 16) * KB * 64;
   p.S = pl.S;
   p.kslice = pl.kslice;
   p.bq = p.NT / pl.ctas_x;
@@ -576,13 +639,21 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   p.wn_log2 = ilog2(pl.wn);
   p.wk_log2 = ilog2(pl.wk);
   p.ngp = pl.ngp;
-  switch (pl.depth) {
-    case 2: return launch_d<FMT, MT, 2>(p, pl, st);
-    case 3: return launch_d<FMT, MT, 3>(p, pl, st);
-    case 4: return launch_d<FMT, MT, 4>(p, pl, st);
-    case 5: return launch_d<FMT, MT, 5>(p, pl, st);
-    case 6: return launch_d<FMT, MT, 6>(p, pl, st);
-    default: return launch_d<FMT, MT, 8>(p, pl, st);
+  if constexpr (FUSE) {                         // stages are twice as large: D <= 4
+    switch (pl.depth) {
+      case 2: return launch_d<FMT, MT, 2, FUSE>(p, pl, st);
+      case 3: return launch_d<FMT, MT, 3, FUSE>(p, pl, st);
+      default: return launch_d<FMT, MT, 4, FUSE>(p, pl, st);
+    }
+  } else {
+    switch (pl.depth) {
+      case 2: return launch_d<FMT, MT, 2, FUSE>(p, pl, st);
+      case 3: return launch_d<FMT, MT, 3, FUSE>(p, pl, st);
+      case 4: return launch_d<FMT, MT, 4, FUSE>(p, pl, st);
+      case 5: return launch_d<FMT, MT, 5, FUSE>(p, pl, st);
+      case 6: return launch_d<FMT, MT, 6, FUSE>(p, pl, st);
+      default: return launch_d<FMT, MT, 8, FUSE>(p, pl, st);
+    }
   }
 }
 
@@ -595,7 +666,11 @@ int warps_of(int fmt, int mt) {
   return mt == 1 ? Cfg<1, 1>::kWarps : Cfg<1, 2>::kWarps;
 }
 
-int header_of(int fmt, int mt) {
+int header_of(int fmt, int mt, int fuse) {
+  if (fuse) {
+    if (fmt == 0) return mt == 1 ? Cfg<0, 1, true>::kHeader : Cfg<0, 2, true>::kHeader;
+    return mt == 1 ? Cfg<1, 1, true>::kHeader : Cfg<1, 2, true>::kHeader;
+  }
   if (fmt == 0) return mt == 1 ? Cfg<0, 1>::kHeader : Cfg<0, 2>::kHeader;
   return mt == 1 ? Cfg<1, 1>::kHeader : Cfg<1, 2>::kHeader;
 }
@@ -611,13 +686,15 @@ int header_of(int fmt, int mt) {
 // constants were fitted to a sweep of (S, wk, D) over the decode shapes at
 // M = 1, 4 and 8 on B200.  The activation image and the rings must fit in
 // shared memory together.
-GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
+GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms, int fuse) {
   GemvPlan pl;
   pl.mt = M <= 8 ? 1 : 2;
   const int warps = warps_of(fmt, pl.mt);
-  const int header = header_of(fmt, pl.mt);
-  const int sb = stage_bytes(fmt);
-  const int NT = (N + 15) / 16;
+  const int header = header_of(fmt, pl.mt, fuse);
+  const int sb = stage_bytes(fmt) * (fuse ? 2 : 1);   // fused: gate and up group per stage
+  const int NT = fuse ? N / 32 : (N + 15) / 16;       // fused: bands of the I gate rows
+  const int depth_cap = fuse ? 4 : kMaxDepth;
+  const double per_group = fuse ? 4.0 : 2.0;          // two bands' bytes per fused group
   const int groups = K / 128;
   double best = 1e300;
   pl.S = 0;
@@ -627,7 +704,7 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
     const int gslice = (groups + S - 1) / S;
     if ((S - 1) * gslice >= groups) continue;  // an empty split
     const int ximg = image_bytes(M, gslice);
-    const int dmax = min(kMaxDepth, (kMaxSmem - header - ximg) / (warps * sb));
+    const int dmax = min(depth_cap, (kMaxSmem - header - ximg) / (warps * sb));
     if (dmax < 2) continue;
     int ctas = num_sms / S;
     if (ctas < 1) ctas = 1;
@@ -641,7 +718,7 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms) {
       for (int d = 2; d <= dmax; ++d) {
         if (d == 7) continue;                  // not instantiated
         const int padded = (piece + d - 1) / d * d;
-        const double cost = (double)rounds * (2.0 * padded + 1.0) +
+        const double cost = (double)rounds * (per_group * padded + 1.0) +
                             (S > 1 ? 3.0 + 0.5 * S : 0.0) + (d < 4 ? 0.5 * (4 - d) : 0.0);
         if (cost < best - 1e-9) {
           best = cost;
@@ -685,8 +762,12 @@ size_t gemv_workspace_floats(const GemvPlan& p, int M, int N) {
 size_t gemv_counters(const GemvPlan& p, int N) { return p.S > 1 ? (N + 15) / 16 : 0; }
 
 cudaError_t launch_gemv(const GemvPlan& p, const GemmArgs& a, cudaStream_t st) {
-  if (a.fmt == 0) return p.mt == 1 ? launch_t<0, 1>(p, a, st) : launch_t<0, 2>(p, a, st);
-  return p.mt == 1 ? launch_t<1, 1>(p, a, st) : launch_t<1, 2>(p, a, st);
+  if (a.fuse) {
+    if (a.fmt == 0) return p.mt == 1 ? launch_t<0, 1, true>(p, a, st) : launch_t<0, 2, true>(p, a, st);
+    return p.mt == 1 ? launch_t<1, 1, true>(p, a, st) : launch_t<1, 2, true>(p, a, st);
+  }
+  if (a.fmt == 0) return p.mt == 1 ? launch_t<0, 1, false>(p, a, st) : launch_t<0, 2, false>(p, a, st);
+  return p.mt == 1 ? launch_t<1, 1, false>(p, a, st) : launch_t<1, 2, false>(p, a, st);
 }
 
 }  // namespace w4

@@ -17,6 +17,8 @@ struct GemmArgs {
   float* ws;            // split-K partials (fp32), may be null when no split is used
   unsigned* counters;   // per 16-row band arrival counters (zero between calls)
   unsigned* err;        // device error word
+  int fuse = 0;         // 1: fused gate/up layer, N = 2I weight rows (gate first),
+                        //    y = [M][I] holds SiLU(gate) * up
 };
 
 // ---------------------------------------------------------------- GEMV (M <= 16)
@@ -32,7 +34,7 @@ struct GemvPlan {
   int smem;      // dynamic shared memory bytes
 };
 
-GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms);
+GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms, int fuse = 0);
 // Bytes of fp32 workspace and number of counters the plan needs.
 size_t gemv_workspace_floats(const GemvPlan& p, int M, int N);
 size_t gemv_counters(const GemvPlan& p, int N);
@@ -55,7 +57,7 @@ struct TcPlan {
   int smem;      // dynamic shared memory bytes
 };
 
-TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms);
+TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms, int fuse = 0);
 size_t tc_workspace_floats(const TcPlan& p, int M, int N);
 size_t tc_counters(const TcPlan& p, int N);
 size_t tc_x_f16_bytes(int fmt, int M, int K);   // NVFP4: FP16 copy of x + row multipliers

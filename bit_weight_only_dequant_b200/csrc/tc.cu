@@ -71,7 +71,9 @@ struct TcParams {
   unsigned* err;
   int M, N, K, KB, NT, tiles, S, gps, units;   // gps: 128-groups per split
   int chunks, rows;        // activation rows run as `chunks` slices of `rows`
+  int fuse, I;             // fused gate/up: I output rows, gate bands [0, I/16), up after
 };
+
 
 // ------------------------------------------------------------------ tcgen05 wrappers
 
@@ -110,6 +112,17 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, float* v) {
 
 template <int NC>
 __device__ __forceinline__ void tmem_ld_32x32b(uint32_t taddr, float* v);
+
+template <>
+__device__ __forceinline__ void tmem_ld_32x32b<4>(uint32_t taddr, float* v) {
+  uint32_t r[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
 
 template <>
 __device__ __forceinline__ void tmem_ld_32x32b<8>(uint32_t taddr, float* v) {
@@ -436,6 +449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* ring = Wr + warp * kWRing * kSB;
     const uint32_t ring_s = smem_u32(ring) + lane * 16;
     int c_unit = blockIdx.x, c_gi = 0, c_hi = 0, c_nb = 0;
+    bool c_valid = false;
     const uint8_t* cw = nullptr;
     const uint8_t* cs = nullptr;
     auto c_start = [&]() {
@@ -443,7 +457,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int tile, chunk, split, g_lo;
         unit_range(p, c_unit, tile, chunk, split, g_lo, c_hi);
         c_gi = g_lo;
-        c_nb = tile * 16 + band;
+        // weight band: tile x 16 bands, or (fused) 8 gate bands in half 0
+        // and the matching up bands, I/16 further, in half 1
+        c_nb = p.fuse ? (h ? p.I >> 4 : 0) + tile * 8 + (band & 7) : tile * 16 + band;
+        c_valid = p.fuse ? tile * 8 + (band & 7) < (p.I >> 4) : c_nb < p.NT;
         const int nb = min(c_nb, p.NT - 1);
         cw = p.w + ((size_t)nb * p.KB + 2 * g_lo) * kTileBytes + lane * 16;
         cs = FMT == 0 ? p.s + ((size_t)nb * G + g_lo) * 32 + g * 4
@@ -454,7 +471,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t c_it = 0;
     auto copy_next = [&]() {                            // one group -> stage c_it % kWRing
       if (c_unit < p.units) {
-        if (c_nb < p.NT) {
+        if (c_valid) {
           const uint32_t d = ring_s + (c_it % kWRing) * kSB;
           cpa16(d, cw, pol);
           cpa16(d + kTileBytes, cw + kTileBytes, pol);
@@ -483,7 +500,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
       int tile, chunk, split, g_lo, g_hi;
       unit_range(p, unit, tile, chunk, split, g_lo, g_hi);
-      const bool real_band = tile * 16 + band < p.NT;
+      const bool real_band = p.fuse ? tile * 8 + (band & 7) < (p.I >> 4) : tile * 16 + band < p.NT;
       for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
         const int sl = it % kASlots;
         const uint32_t ua = it / kASlots;
@@ -552,35 +569,71 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       constexpr int kHalf = MPAD / 2;                   // columns this warp reads
       constexpr int kEC = kHalf % 32 == 0 ? 32 : kHalf % 16 == 0 ? 16 : 8;   // per tcgen05.ld
-      const int n = tile * kTcTileRows + h * 128 + 32 * q + lane;
+      // weight row of this lane; fused: gate row i in half 0, up row I + i in half 1
+      const int i_out = tile * (p.fuse ? 128 : kTcTileRows) + (p.fuse ? 0 : h * 128) + 32 * q + lane;
+      const int n = p.fuse ? (h ? p.I : 0) + i_out : i_out;
+      const bool n_ok = p.fuse ? i_out < p.I : n < p.N;
       const int m0 = bp * kHalf;                        // local row of the chunk
       const int xrow = chunk * p.rows;
       const int mlim = min(p.rows, p.M - xrow);          // rows of this chunk
       float gmul = 1.f;
       if (FMT == 1) gmul = __ldg(p.g);
       const size_t Npad = (size_t)p.NT * 16;
+      if (p.fuse && p.S == 1) {
+        // fused, not split: every warp reads gate (half 0) and up (half 1) for
+        // its 32 lanes, which hold the same output row i, over a quarter of
+        // the columns, and writes BF16(SiLU(gate) * up)
+        constexpr int kQ = MPAD / 4;
+        constexpr int kEQ = kQ % 32 == 0 ? 32 : kQ % 16 == 0 ? 16 : kQ % 8 == 0 ? 8 : 4;
+        const int mq = (2 * bp + h) * kQ;
+        const int i_row = tile * 128 + 32 * q + lane;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kHalf; c0 += kEC) {
-        float v[kEC];
-        tmem_ld_32x32b<kEC>(tmem + ((uint32_t)(32 * q) << 16) + h * kDStride + m0 + c0, v);
-        tmem_wait_ld();
-        if (n < p.N) {
-          const int mb = xrow + m0 + c0;                 // first row of this batch
-          if (p.S == 1) {
-            __nv_bfloat16* yp = p.y + (size_t)mb * p.N + n;
+        for (int c0 = 0; c0 < kQ; c0 += kEQ) {
+          float v[kEQ], u[kEQ];
+          tmem_ld_32x32b<kEQ>(tmem + ((uint32_t)(32 * q) << 16) + mq + c0, v);
+          tmem_ld_32x32b<kEQ>(tmem + ((uint32_t)(32 * q) << 16) + kDStride + mq + c0, u);
+          tmem_wait_ld();
+          if (i_row < p.I) {
+            const int mb = xrow + mq + c0;
+            __nv_bfloat16* hp = p.y + (size_t)mb * p.I + i_row;
 #pragma unroll
-            for (int c = 0; c < kEC; ++c, yp += p.N) {
-              if (m0 + c0 + c < mlim) {
-                float val = v[c];
-                if (FMT == 1) val = val * __ldg(p.row_mul + mb + c) * gmul;
-                *yp = __float2bfloat16_rn(val);
+            for (int c = 0; c < kEQ; ++c, hp += p.I) {
+              if (mq + c0 + c < mlim) {
+                float gv = v[c], uv = u[c];
+                if (FMT == 1) {
+                  const float rm = __ldg(p.row_mul + mb + c);
+                  gv = gv * rm * gmul;
+                  uv = uv * rm * gmul;
+                }
+                *hp = __float2bfloat16_rn(silu_f32(gv) * uv);
               }
             }
-          } else {
-            float* wp = p.ws + ((size_t)split * p.M + mb) * Npad + n;
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < kHalf; c0 += kEC) {
+          float v[kEC];
+          tmem_ld_32x32b<kEC>(tmem + ((uint32_t)(32 * q) << 16) + h * kDStride + m0 + c0, v);
+          tmem_wait_ld();
+          if (n_ok) {
+            const int mb = xrow + m0 + c0;                 // first row of this batch
+            if (p.S == 1) {
+              __nv_bfloat16* yp = p.y + (size_t)mb * p.N + n;
 #pragma unroll
-            for (int c = 0; c < kEC; ++c, wp += Npad)
-              if (m0 + c0 + c < mlim) __stcg(wp, v[c]);
+              for (int c = 0; c < kEC; ++c, yp += p.N) {
+                if (m0 + c0 + c < mlim) {
+                  float val = v[c];
+                  if (FMT == 1) val = val * __ldg(p.row_mul + mb + c) * gmul;
+                  *yp = __float2bfloat16_rn(val);
+                }
+              }
+            } else {
+              float* wp = p.ws + ((size_t)split * p.M + mb) * Npad + n;
+#pragma unroll
+              for (int c = 0; c < kEC; ++c, wp += Npad)
+                if (m0 + c0 + c < mlim) __stcg(wp, v[c]);
+            }
           }
         }
       }
@@ -661,18 +714,9 @@ __global__ void __launch_bounds__(256) prep_x_f16_kernel(const __nv_bfloat16* __
 // fp32 partials [S][M][Npad]), times the NVFP4 row multiplier and global
 // scale.  Four columns per thread; launched behind the main kernel with
 // programmatic dependent launch, so it waits for the partials on the device.
-template <int FMT>
-__global__ void __launch_bounds__(256)
-    tc_splitk_reduce(const float* __restrict__ ws, int S, int M, int N, int Npad,
-                     const float* __restrict__ row_mul, const float* __restrict__ g,
-                     __nv_bfloat16* __restrict__ y) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int m = blockIdx.y;
-  const int n0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
-  if (n0 >= N) return;
-  const size_t sstride = (size_t)M * Npad;
-  const float* src = ws + (size_t)m * Npad + n0;
-  float a[4] = {0.f, 0.f, 0.f, 0.f};
+// Sum over splits, in split order, of four consecutive partials at `src`.
+__device__ __forceinline__ void sum_splits4(const float* src, size_t sstride, int S, float* a) {
+  a[0] = a[1] = a[2] = a[3] = 0.f;
   int sp = 0;
   for (; sp + 4 <= S; sp += 4) {                 // four splits' loads in flight, added in order
     float4 v[4];
@@ -693,6 +737,23 @@ __global__ void __launch_bounds__(256)
     a[2] += v.z;
     a[3] += v.w;
   }
+}
+
+// Fused gate/up: `cols` = I output columns, gate partials at n, up at I + n,
+// y[m][n] = BF16(SiLU(gate) * up).
+template <int FMT, bool FUSE>
+__global__ void __launch_bounds__(256)
+    tc_splitk_reduce(const float* __restrict__ ws, int S, int M, int cols, int Npad,
+                     const float* __restrict__ row_mul, const float* __restrict__ g,
+                     __nv_bfloat16* __restrict__ y) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int m = blockIdx.y;
+  const int n0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (n0 >= cols) return;
+  const size_t sstride = (size_t)M * Npad;
+  float a[4], u[4];
+  sum_splits4(ws + (size_t)m * Npad + n0, sstride, S, a);
+  if (FUSE) sum_splits4(ws + (size_t)m * Npad + cols + n0, sstride, S, u);
   float rm = 1.f, gm = 1.f;
   if (FMT == 1) {
     rm = __ldg(row_mul + m);
@@ -700,10 +761,15 @@ __global__ void __launch_bounds__(256)
   }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    if (n0 + j < N) {
+    if (n0 + j < cols) {
       float val = a[j];
       if (FMT == 1) val = val * rm * gm;
-      y[(size_t)m * N + n0 + j] = __float2bfloat16_rn(val);
+      if (FUSE) {
+        float uv = u[j];
+        if (FMT == 1) uv = uv * rm * gm;
+        val = silu_f32(val) * uv;
+      }
+      y[(size_t)m * cols + n0 + j] = __float2bfloat16_rn(val);
     }
   }
 }
@@ -756,7 +822,9 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   p.K = a.K;
   p.KB = a.K / 64;
   p.NT = (a.N + 15) / 16;
-  p.tiles = (a.N + kTcTileRows - 1) / kTcTileRows;
+  p.fuse = a.fuse;
+  p.I = a.N / 2;
+  p.tiles = a.fuse ? (p.I + 127) / 128 : (a.N + kTcTileRows - 1) / kTcTileRows;
   p.S = pl.S;
   p.gps = pl.kbs / 2;
   p.chunks = pl.chunks;
@@ -776,8 +844,9 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || pl.S == 1) return e;
 
+  const int cols = a.fuse ? a.N / 2 : a.N;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((a.N + 1023) / 1024), (unsigned)a.M, 1);
+  cfg.gridDim = dim3((unsigned)((cols + 1023) / 1024), (unsigned)a.M, 1);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -786,8 +855,13 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_splitk_reduce<FMT>, static_cast<const float*>(a.ws), pl.S, a.M,
-                            a.N, p.NT * 16, row_mul, a.g, static_cast<__nv_bfloat16*>(a.y));
+  const float* ws = a.ws;
+  __nv_bfloat16* y = static_cast<__nv_bfloat16*>(a.y);
+  if (a.fuse)
+    return cudaLaunchKernelEx(&cfg, tc_splitk_reduce<FMT, true>, ws, pl.S, a.M, cols, p.NT * 16,
+                              row_mul, a.g, y);
+  return cudaLaunchKernelEx(&cfg, tc_splitk_reduce<FMT, false>, ws, pl.S, a.M, cols, p.NT * 16,
+                            row_mul, a.g, y);
 }
 
 template <int FMT>
@@ -813,12 +887,12 @@ cudaError_t launch_fmt(const TcPlan& pl, const GemmArgs& a, const void* xsrc, co
 // the busiest CTA's waves x (its groups x t_group + t_unit), t_unit being the
 // epilogue and pipeline refill of a unit, plus, with split K, the reduction
 // launch and its traffic (the partials written and read once more).
-TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms) {
+TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms, int fuse) {
   TcPlan pl;
   pl.chunks = (M + kTcMaxRows - 1) / kTcMaxRows;
   pl.rows = (M + pl.chunks - 1) / pl.chunks;
   pl.mpad = (pl.rows + 15) / 16 * 16;
-  const int tiles = (N + kTcTileRows - 1) / kTcTileRows;
+  const int tiles = fuse ? (N / 2 + 127) / 128 : (N + kTcTileRows - 1) / kTcTileRows;
   const int groups = K / 128;
   const double t_group = 0.75 + 0.0017 * pl.mpad;   // us per 128-group of a 256-row tile
   const double t_unit = 0.5 + 0.035 * pl.mpad;      // us per unit: epilogue, refill

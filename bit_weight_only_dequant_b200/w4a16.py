@@ -40,6 +40,8 @@ _SIGS = {
     "w4a16_gemm": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_ex": (_i, [_i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_path": (_i, [_i, _i, _i, _i]),
+    "w4a16_gemm_gate_up_silu": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_gemm_gate_up_silu_ex": (_i, [_i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_device_status": (_i, [_vp]),
     "w4a16_status_string": (ctypes.c_char_p, [_i]),
@@ -141,6 +143,20 @@ def w4a16_gemm_noalloc(fmt, M, N, K, x, packed_w, packed_scales, global_scale, y
                                     _ptr(global_scale), _ptr(y), _stream(stream))
 
 
+def w4a16_gemm_gate_up_silu(fmt, M, I, K, x, packed_w, packed_scales, global_scale, h,
+                            stream=None):
+    return lib().w4a16_gemm_gate_up_silu(fmt, M, I, K, _ptr(x), _ptr(packed_w),
+                                         _ptr(packed_scales), _ptr(global_scale), _ptr(h),
+                                         _stream(stream))
+
+
+def w4a16_gemm_gate_up_silu_ex(path, fmt, M, I, K, x, packed_w, packed_scales, global_scale, h,
+                               stream=None):
+    return lib().w4a16_gemm_gate_up_silu_ex(path, fmt, M, I, K, _ptr(x), _ptr(packed_w),
+                                            _ptr(packed_scales), _ptr(global_scale), _ptr(h),
+                                            _stream(stream))
+
+
 def w4a16_gemm_path(fmt, M, N, K):
     return lib().w4a16_gemm_path(fmt, M, N, K)
 
@@ -177,6 +193,19 @@ def gemm(fmt: str, x, packed_w, packed_scales, N: int, global_scale=None, y=None
     check(w4a16_gemm_ex(path, FMTS[fmt], M, N, K, x, packed_w, packed_scales, global_scale, y,
                         stream), "w4a16_gemm")
     return y
+
+
+def gate_up_silu(fmt: str, x, packed_w, packed_scales, I: int, global_scale=None, h=None,
+                 path=PATH_AUTO, stream=None):
+    """h = SiLU(x . W_gate^T) * (x . W_up^T) for a BF16 CUDA tensor x [M][K] and
+    the packed [2I][K] gate/up weight; returns h (BF16 [M][I])."""
+    import torch
+    M, K = x.shape
+    if h is None:
+        h = torch.empty((M, I), dtype=torch.bfloat16, device=x.device)
+    check(w4a16_gemm_gate_up_silu_ex(path, FMTS[fmt], M, I, K, x, packed_w, packed_scales,
+                                     global_scale, h, stream), "w4a16_gemm_gate_up_silu")
+    return h
 
 
 def dequant(fmt: str, N: int, K: int, packed_w, packed_scales, global_scale=None, out=None,

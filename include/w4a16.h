@@ -143,6 +143,29 @@ int w4a16_gemm_ex(int path, int fmt, int M, int N, int K, const void* x_bf16,
                   void* y_bf16, void* stream);
 
 /*
+ * The fused gate/up layer of the MLP: h[M][I] = BF16(SiLU(gate) * up) with
+ *   gate = x . W_deq[0:I]^T,  up = x . W_deq[I:2I]^T,  SiLU(z) = z / (1 + e^-z),
+ * gate and up kept in fp32 until the product (one kernel, or two when K is
+ * split across CTAs on the tensor-core path: the reduction applies SiLU).
+ * Reading of the pages' MLP linears (model card "Qwen3.8 27B - NVFP4 for
+ * veloGB10", section "Specifications"): the [2I][K] weight holds the gate
+ * rows first and the up rows second.
+ *   packed_w, packed_scales: that [2I][K] weight packed as for w4a16_gemm
+ *     with N = 2I.  I >= 16 and a multiple of 16 (else W4A16_ERR_SHAPE).
+ *   x_bf16, global_scale: as for w4a16_gemm.
+ *   h_bf16: device, [M][I] BF16 row-major; must not overlap any input.
+ * Same row limits and dispatch as w4a16_gemm with N = 2I.
+ */
+int w4a16_gemm_gate_up_silu(int fmt, int M, int I, int K, const void* x_bf16,
+                            const void* packed_w, const void* packed_scales,
+                            const float* global_scale, void* h_bf16, void* stream);
+
+/* Same as w4a16_gemm_gate_up_silu with an explicit path (W4A16_PATH_*). */
+int w4a16_gemm_gate_up_silu_ex(int path, int fmt, int M, int I, int K, const void* x_bf16,
+                               const void* packed_w, const void* packed_scales,
+                               const float* global_scale, void* h_bf16, void* stream);
+
+/*
  * The split-K GEMV (M <= W4A16_GEMV_MAX_M) for callers that cannot allocate
  * device memory: code that issues the matmul while its stream is being
  * captured into a CUDA graph, where cudaMalloc is not allowed, and

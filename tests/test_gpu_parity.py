@@ -195,6 +195,90 @@ def test_gemm_parity_full_shapes_sampled(fmt, name, M, seed):
     t.cuda.empty_cache()
 
 
+# ---------------------------------------------------------------- fused gate/up + SiLU
+
+
+def _assert_gate_up_parity(h_gpu, x_bits, w_bits, what=""):
+    h_ref, gate, up = oracle.gate_up_silu_ref(x_bits, w_bits)
+    allowed = oracle.gate_up_silu_allowed(x_bits, w_bits, gate, up)
+    err = np.abs(h_gpu - h_ref)
+    if not np.all(err <= allowed):
+        bad = np.argwhere(err > allowed)[:5]
+        detail = [(int(m), int(i), float(h_gpu[m, i]), float(h_ref[m, i]), float(allowed[m, i]))
+                  for m, i in bad]
+        raise AssertionError(f"{what}: {int((err > allowed).sum())} elements out of tolerance, "
+                             f"e.g. {detail}")
+
+
+def _run_gate_up(fmt, p, I, path=W.PATH_AUTO):
+    t = torch()
+    codes, scales, x = to_device_problem(p)
+    pw, ps = W.pack_on_device(fmt, 2 * I, p["K"], codes, scales)
+    h = W.gate_up_silu(fmt, x.view(t.bfloat16), pw, ps, I, global_scale=gscale_tensor(p["g"]),
+                       path=path)
+    t.cuda.synchronize()
+    W.check(W.w4a16_device_status(), "device status")
+    return h.float().cpu().numpy().astype(np.float64)
+
+
+GATE_UP = [  # fmt, M, I, K, path
+    ("int4", 1, 48, 640, W.PATH_GEMV), ("int4", 4, 400, 1536, W.PATH_GEMV),
+    ("int4", 8, 144, 17408, W.PATH_GEMV),          # long K: split across CTAs
+    ("int4", 16, 64, 2048, W.PATH_GEMV), ("nvfp4", 3, 208, 1280, W.PATH_GEMV),
+    ("nvfp4", 12, 96, 4096, W.PATH_GEMV), ("nvfp4", 1, 16, 17408, W.PATH_GEMV),
+    ("int4", 9, 48, 640, W.PATH_TC), ("int4", 64, 400, 1536, W.PATH_TC),
+    ("int4", 17, 144, 17408, W.PATH_TC),           # split K: SiLU in the reduction
+    ("int4", 1, 16, 128, W.PATH_TC), ("int4", 200, 272, 1024, W.PATH_TC),
+    ("nvfp4", 33, 208, 1280, W.PATH_TC), ("nvfp4", 128, 160, 2048, W.PATH_TC),
+    ("nvfp4", 40, 48, 12288, W.PATH_TC), ("int4", 1000, 144, 384, W.PATH_TC),
+    ("int4", 5, 32, 512, W.PATH_AUTO), ("nvfp4", 70, 64, 512, W.PATH_AUTO),
+]
+
+
+@pytest.mark.parametrize("fmt,M,I,K,path", GATE_UP)
+def test_gate_up_silu_parity(fmt, M, I, K, path):
+    p = synth.problem(fmt, 300 + M + I, M, 2 * I, K)
+    h = _run_gate_up(fmt, p, I, path)
+    _assert_gate_up_parity(h, p["x"], oracle_weights(p), f"{fmt} M={M} I={I} K={K} path={path}")
+
+
+@pytest.mark.parametrize("fmt,M", [("int4", 1), ("int4", 9), ("int4", 64), ("nvfp4", 1),
+                                   ("nvfp4", 64), ("int4", 256)])
+def test_gate_up_silu_full_shape_sampled(fmt, M):
+    K, N = SHAPES["gate_up"]
+    I = N // 2
+    t = torch()
+    seed = SEEDS["gate_up"]
+    p = synth.device_problem(fmt, seed, M, N, K)
+    pw, ps = W.pack_on_device(fmt, N, K, p["codes"], p["scales"])
+    h = W.gate_up_silu(fmt, p["x"].view(t.bfloat16), pw, ps, I, global_scale=gscale_tensor(p["g"]))
+    t.cuda.synchronize()
+    cols = np.unique(np.concatenate([[0, 15, 16, 127, 128, I - 1],
+                                     np.random.default_rng(M).integers(0, I, 40)]))
+    ph = synth.problem(fmt, seed, M, N, K, rows=np.concatenate([cols, I + cols]))
+    hs = h[:, t.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
+    _assert_gate_up_parity(hs, ph["x"], oracle_weights(ph), f"{fmt} gate_up M={M}")
+    del p, pw, ps, h
+    t.cuda.empty_cache()
+
+
+def test_gate_up_silu_matches_the_unfused_pair():
+    # the fused layer against SiLU / product applied on the host to the two
+    # halves of the plain matmul: both within tolerance of each other
+    t = torch()
+    fmt, M, I, K = "int4", 6, 272, 1024
+    p = synth.problem(fmt, 77, M, 2 * I, K)
+    codes, scales, x = to_device_problem(p)
+    pw, ps = W.pack_on_device(fmt, 2 * I, K, codes, scales)
+    xb = x.view(t.bfloat16)
+    y = W.gemm(fmt, xb, pw, ps, 2 * I).float().cpu().numpy().astype(np.float64)
+    h = W.gate_up_silu(fmt, xb, pw, ps, I).float().cpu().numpy().astype(np.float64)
+    w = oracle_weights(p)
+    _, gate, up = oracle.gate_up_silu_ref(p["x"], w)
+    allowed = oracle.gate_up_silu_allowed(p["x"], w, gate, up)
+    assert np.all(np.abs(h - oracle.silu(y[:, :I]) * y[:, I:]) <= 2 * allowed)
+
+
 # ---------------------------------------------------------------- invariants and edge cases
 
 

@@ -154,6 +154,20 @@ def test_argument_validation_before_any_device_call():
     assert W.w4a16_pack(0, 16, 100, x, s, w, s, 0) == W.ERR_SHAPE
 
 
+def test_gate_up_silu_argument_validation():
+    x = w = s = h = 1 << 20          # fake, aligned, never dereferenced
+    assert W.w4a16_gemm_gate_up_silu(0, 1, 24, 128, x, w, s, None, h, 0) == W.ERR_SHAPE   # I % 16
+    assert W.w4a16_gemm_gate_up_silu(0, 1, 0, 128, x, w, s, None, h, 0) == W.ERR_SHAPE    # I = 0
+    assert W.w4a16_gemm_gate_up_silu(0, 0, 16, 128, x, w, s, None, h, 0) == W.ERR_SHAPE   # M = 0
+    assert W.w4a16_gemm_gate_up_silu(0, 8193, 16, 128, x, w, s, None, h, 0) == W.ERR_SHAPE
+    assert W.w4a16_gemm_gate_up_silu(0, 1, 16, 100, x, w, s, None, h, 0) == W.ERR_SHAPE   # K % 128
+    assert W.w4a16_gemm_gate_up_silu(5, 1, 16, 128, x, w, s, None, h, 0) == W.ERR_ARG     # format
+    assert W.w4a16_gemm_gate_up_silu(1, 1, 16, 128, x, w, s, None, h, 0) == W.ERR_ARG     # no g
+    assert W.w4a16_gemm_gate_up_silu(0, 1, 16, 128, x, w, s, None, h + 4, 0) == W.ERR_ALIGN
+    assert W.w4a16_gemm_gate_up_silu_ex(9, 0, 1, 16, 128, x, w, s, None, h, 0) == W.ERR_ARG
+    assert W.w4a16_gemm_gate_up_silu_ex(W.PATH_GEMV, 0, 17, 16, 128, x, w, s, None, h, 0) == W.ERR_SHAPE
+
+
 def test_dispatcher_path_table():
     for M in range(1, W.MAX_M + 1):
         path = W.w4a16_gemm_path(0, M, 5120, 5120)
