@@ -43,7 +43,10 @@ L2_BYTES = 126 * 1024 * 1024
 
 
 def alg_bytes(fmt, M, N, K):
-    w = N * K * (0.5 + (2 / 128 if fmt == "int4" else 1 / 16)) + (4 if fmt == "nvfp4" else 0)
+    if fmt == "fp8":                                  # a byte per weight, one fp32 scale
+        w = N * K + 4
+    else:
+        w = N * K * (0.5 + (2 / 128 if fmt == "int4" else 1 / 16)) + (4 if fmt == "nvfp4" else 0)
     return w + 2 * M * K + 2 * M * N
 
 
@@ -304,7 +307,7 @@ def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
     ws = make_weights(fmt, seed, N, K, copies)
     x = make_x(fmt, seed, M, K)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
+    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt != "int4" else None
     path = W.w4a16_gemm_path(f, M, N, K)
 
     def launch(r, ws=ws):
@@ -343,7 +346,7 @@ def gate_up_entry(fmt, M, seed, peaks, stream, reps=24):
     ws = make_weights(fmt, seed, N, K, copies_for(wbytes))
     x = make_x(fmt, seed, M, K)
     h = torch.empty((M, I), dtype=torch.bfloat16, device="cuda")
-    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
+    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt != "int4" else None
     path = W.w4a16_gemm_path(f, M, N, K)
 
     def launch(r, ws=ws):
@@ -565,6 +568,8 @@ def run_native(args, rank, world, local_rank):
         cfg5 = [(fmt, n, K, N, Mv, 7) for fmt in ("int4", "nvfp4") for Mv in (128, 256)
                 for n, K, N, _ in DECODE_SHAPES]
         cfg5 += [("int4", n, K, N, 2048, 8) for n, K, N, _ in DECODE_SHAPES]
+        # FP8-E4M3 weights (W8A16) on the attention linears
+        cfg5 += [("fp8", n, K, N, Mv, 9) for Mv in (1, 9, 64) for n, K, N, _ in DECODE_SHAPES[:2]]
         for fmt, n, K, N, Mv, s in target + cfg2 + cfg3 + cfg4 + cfg5:
             entries.append(sweep_entry(fmt, n, K, N, Mv, s, peaks, stream))
         extra["sweep"] = entries
@@ -613,7 +618,7 @@ def run_case(spec: str, launches: int):
     (pw, ps), = make_weights(fmt, 3, N, K, 1)
     x = make_x(fmt, 3, M, K)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
+    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt != "int4" else None
     for _ in range(launches):
         W.check(W.w4a16_gemm_ex(path, f, M, N, K, x, pw, ps, g, y), "gemm")
     torch.cuda.synchronize()

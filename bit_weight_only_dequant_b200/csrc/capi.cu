@@ -122,8 +122,12 @@ int workspace(cudaStream_t st, size_t counters, size_t floats, size_t bytes, uns
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool has_global_scale(int fmt) { return fmt != W4A16_FMT_INT4_G128; }
+bool has_packed_scales(int fmt) { return fmt != W4A16_FMT_FP8_E4M3; }
+
 int check_fmt_shape(int fmt, int N, int K) {
-  if (fmt != W4A16_FMT_INT4_G128 && fmt != W4A16_FMT_NVFP4_G16) return W4A16_ERR_ARG;
+  if (fmt != W4A16_FMT_INT4_G128 && fmt != W4A16_FMT_NVFP4_G16 && fmt != W4A16_FMT_FP8_E4M3)
+    return W4A16_ERR_ARG;
   if (N < 1 || K < 128 || K % 128 != 0) return W4A16_ERR_SHAPE;
   // packed tensors are addressed with 32-bit tile/scale indices in places
   if ((long long)((N + 15) / 16) * (K / 64) >= (1ll << 31) / 64) return W4A16_ERR_SHAPE;
@@ -157,10 +161,11 @@ int run_gemm(int path, int fmt, int M, int N, int K, const void* x_bf16, const v
   if (M < 1 || M > W4A16_MAX_M) return W4A16_ERR_SHAPE;
   if (path != W4A16_PATH_AUTO && path != W4A16_PATH_GEMV && path != W4A16_PATH_TC)
     return W4A16_ERR_ARG;
-  if (!x_bf16 || !packed_w || !packed_scales || !y_bf16) return W4A16_ERR_ARG;
-  if ((fmt == W4A16_FMT_NVFP4_G16) != (global_scale != nullptr)) return W4A16_ERR_ARG;
-  if (!aligned16(x_bf16) || !aligned16(packed_w) || !aligned16(packed_scales) ||
-      !aligned16(y_bf16))
+  if (!x_bf16 || !packed_w || !y_bf16) return W4A16_ERR_ARG;
+  if (has_packed_scales(fmt) && !packed_scales) return W4A16_ERR_ARG;
+  if (has_global_scale(fmt) != (global_scale != nullptr)) return W4A16_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(packed_w) || !aligned16(y_bf16) ||
+      (has_packed_scales(fmt) && !aligned16(packed_scales)))
     return W4A16_ERR_ALIGN;
   if (path == W4A16_PATH_AUTO) path = choose_path(fmt, M, N, K);
   if (path == W4A16_PATH_GEMV && M > W4A16_GEMV_MAX_M) return W4A16_ERR_SHAPE;
@@ -209,7 +214,7 @@ extern "C" {
 
 size_t w4a16_packed_weight_bytes(int fmt, int N, int K) {
   if (check_fmt_shape(fmt, N, K) != W4A16_OK) return 0;
-  return (size_t)w4::weight_bytes(N, K);
+  return (size_t)w4::weight_bytes(fmt, N, K);
 }
 
 size_t w4a16_packed_scale_bytes(int fmt, int N, int K) {
@@ -221,7 +226,8 @@ int w4a16_pack_host(int fmt, int N, int K, const void* codes, const void* scales
                     void* packed_scales) {
   const int r = check_fmt_shape(fmt, N, K);
   if (r != W4A16_OK) return r;
-  if (!codes || !scales || !packed_w || !packed_scales) return W4A16_ERR_ARG;
+  if (!codes || !packed_w || (has_packed_scales(fmt) && (!scales || !packed_scales)))
+    return W4A16_ERR_ARG;
   return w4::pack_host(fmt, N, K, codes, scales, packed_w, packed_scales) == 0 ? W4A16_OK
                                                                                : W4A16_ERR_ARG;
 }
@@ -230,7 +236,8 @@ int w4a16_unpack_host(int fmt, int N, int K, const void* packed_w, const void* p
                       void* codes, void* scales) {
   const int r = check_fmt_shape(fmt, N, K);
   if (r != W4A16_OK) return r;
-  if (!codes || !scales || !packed_w || !packed_scales) return W4A16_ERR_ARG;
+  if (!codes || !packed_w || (has_packed_scales(fmt) && (!scales || !packed_scales)))
+    return W4A16_ERR_ARG;
   return w4::unpack_host(fmt, N, K, packed_w, packed_scales, codes, scales) == 0 ? W4A16_OK
                                                                                  : W4A16_ERR_ARG;
 }
@@ -239,8 +246,10 @@ int w4a16_pack(int fmt, int N, int K, const void* codes, const void* scales, voi
                void* packed_scales, void* stream) {
   int r = check_fmt_shape(fmt, N, K);
   if (r != W4A16_OK) return r;
-  if (!codes || !scales || !packed_w || !packed_scales) return W4A16_ERR_ARG;
-  if (!aligned16(codes) || !aligned16(scales) || !aligned16(packed_w) || !aligned16(packed_scales))
+  if (!codes || !packed_w || (has_packed_scales(fmt) && (!scales || !packed_scales)))
+    return W4A16_ERR_ARG;
+  if (!aligned16(codes) || !aligned16(packed_w) ||
+      (has_packed_scales(fmt) && (!aligned16(scales) || !aligned16(packed_scales))))
     return W4A16_ERR_ALIGN;
   DeviceState* d = nullptr;
   if ((r = device_state(&d)) != W4A16_OK) return r;
@@ -252,9 +261,10 @@ int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packe
                   const float* global_scale, void* w_bf16, void* stream) {
   int r = check_fmt_shape(fmt, N, K);
   if (r != W4A16_OK) return r;
-  if (!packed_w || !packed_scales || !w_bf16) return W4A16_ERR_ARG;
-  if ((fmt == W4A16_FMT_NVFP4_G16) != (global_scale != nullptr)) return W4A16_ERR_ARG;
-  if (!aligned16(packed_w) || !aligned16(packed_scales) || !aligned16(w_bf16))
+  if (!packed_w || !w_bf16 || (has_packed_scales(fmt) && !packed_scales)) return W4A16_ERR_ARG;
+  if (has_global_scale(fmt) != (global_scale != nullptr)) return W4A16_ERR_ARG;
+  if (!aligned16(packed_w) || !aligned16(w_bf16) ||
+      (has_packed_scales(fmt) && !aligned16(packed_scales)))
     return W4A16_ERR_ALIGN;
   DeviceState* d = nullptr;
   if ((r = device_state(&d)) != W4A16_OK) return r;

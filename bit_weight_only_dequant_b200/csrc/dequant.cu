@@ -9,6 +9,9 @@
 //   and rounded once: fp64 -> fp32 toward zero with a sticky bit (round to
 //   odd, 16 spare bits) followed by fp32 -> bf16 to nearest even gives the
 //   correctly rounded BF16 value, subnormal range included.
+// FP8-E4M3 (weight-only FP8 of the attention linears, guide "Qwen3.8-27B on
+//   DGX Spark (GB10)", section "What Spark-native means"): W = RNE_bf16(e4m3
+//   * g) with one fp32 g per tensor, rounded the same way.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -93,14 +96,52 @@ __global__ void dequant_kernel(int N, int K, const uint8_t* __restrict__ w,
   }
 }
 
+__global__ void dequant_fp8_kernel(int N, int K, const uint8_t* __restrict__ w,
+                                   const float* __restrict__ gptr, __nv_bfloat16* __restrict__ out) {
+  const int KT = K >> 5;
+  const long long NT = (N + 15) / 16;
+  const long long total = NT * KT * 32;
+  const float g = __ldg(gptr);
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int lane = (int)(idx & 31);
+    const long long tile = idx >> 5;
+    const long long nt = tile / KT;
+    const int kt = (int)(tile - nt * KT);
+    const int gq = lane >> 2, t = lane & 3;
+    const uint4 wv = *reinterpret_cast<const uint4*>(w + tile * kTileBytes + lane * 16);
+    const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int hrow = 0; hrow < 2; ++hrow) {
+      const long long n = nt * 16 + gq + 8 * hrow;
+      if (n >= N) continue;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int k0 = kt * 32 + j * 16 + 4 * t;
+        __nv_bfloat16 o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pair = hrow + 2 * (e >> 1), second = e & 1;
+          const uint32_t b = (wd[2 * j + (pair >> 1)] >> (8 * (2 * (pair & 1) + second))) & 0xFFu;
+          o[e] = round_product_bf16(e4m3_value(b), g);
+        }
+        *reinterpret_cast<uint2*>(out + n * (long long)K + k0) = *reinterpret_cast<uint2*>(o);
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_dequant(int fmt, int N, int K, const void* w, const void* s, const float* g,
                            void* out, cudaStream_t st) {
-  const long long total = (long long)((N + 15) / 16) * (K / 64) * 32;
+  const long long total = (long long)((N + 15) / 16) * (K / 64) * 32 * (fmt == kFmtFp8 ? 2 : 1);
   long long blocks = (total + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  if (fmt == 0)
+  if (fmt == kFmtFp8)
+    dequant_fp8_kernel<<<(unsigned)blocks, 256, 0, st>>>(N, K, (const uint8_t*)w, g,
+                                                         (__nv_bfloat16*)out);
+  else if (fmt == 0)
     dequant_kernel<0><<<(unsigned)blocks, 256, 0, st>>>(N, K, (const uint8_t*)w, (const uint8_t*)s,
                                                          g, (__nv_bfloat16*)out);
   else

@@ -49,11 +49,16 @@ constexpr int kRowAuxOff = kRowWords * 4;
 constexpr int kRedOff = 2 * kRowWords * 4;                   // per-lane partial sums
 constexpr int kMaxSmem = 232448;                             // 227 KB opt-in
 constexpr int kMaxDepth = 8;                                 // ring stages per warp
-constexpr int kGroupBytes = 2 * kTileBytes;                  // packed weights of one band-group
+constexpr int kGroupBytes = 2 * kTileBytes;                  // packed 4-bit weights of one band-group
+
+// Packed weights of one band's 128-group: two 512-byte tiles at 4 bits, four at 8.
+__host__ __device__ constexpr int group_bytes(int fmt) { return fmt == kFmtFp8 ? 4 * kTileBytes : kGroupBytes; }
 
 // Shared-memory bytes of one ring stage: the group's two tiles, then the
 // scales each lane needs (int4: 4 bytes, NVFP4: 2 x 8 bytes per lane).
-__host__ __device__ constexpr int stage_bytes(int fmt) { return kGroupBytes + (fmt == 0 ? 128 : 512); }
+__host__ __device__ constexpr int stage_bytes(int fmt) {
+  return fmt == kFmtFp8 ? group_bytes(fmt) : kGroupBytes + (fmt == 0 ? 128 : 512);
+}
 
 // Warps per CTA: a power of two (the warp grid is split with shifts).  16
 // warps leave 128 registers a thread; with 64 (32 warps) the compiler
@@ -298,12 +303,42 @@ __device__ __forceinline__ void block_nvfp4(uint4 wv, uint2 sv, const uint8_t* c
   }
 }
 
+// One 128-group of one band, FP8-E4M3 (per-tensor scale, applied in the
+// epilogue): st is this lane's 16 bytes of the group's first tile; the four
+// tiles are 512 bytes apart, two per 64-block, two k16 sub-blocks per tile.
+template <int MT>
+__device__ __forceinline__ void group_fp8(const uint8_t* st, const uint8_t* const* xg,
+                                          float (*acc)[4]) {
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk) {
+    const uint4 t0 = *reinterpret_cast<const uint4*>(st + (2 * blk) * kTileBytes);
+    const uint4 t1 = *reinterpret_cast<const uint4*>(st + (2 * blk + 1) * kTileBytes);
+    const uint32_t wd[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+    uint32_t a[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {     // k16 sub-block j of the 64-block: words 2j (P0, P1), 2j+1 (P2, P3)
+      a[j][0] = e4m3x2_to_f16x2(static_cast<uint16_t>(wd[2 * j]));
+      a[j][1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wd[2 * j] >> 16));
+      a[j][2] = e4m3x2_to_f16x2(static_cast<uint16_t>(wd[2 * j + 1]));
+      a[j][3] = e4m3x2_to_f16x2(static_cast<uint16_t>(wd[2 * j + 1] >> 16));
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const uint4* xb = reinterpret_cast<const uint4*>(xg[mt] + blk * 128);
+      const uint4 v0 = xb[0], v1 = xb[1];
+      const uint32_t bx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) mma_f16_16816(acc[mt], a[j], bx[2 * j], bx[2 * j + 1]);
+    }
+  }
+}
+
 template <int FMT, int MT, bool FUSE>
 __device__ __forceinline__ void band_epilogue(const Params& p, int band, int split, int lane,
                                               const float* row_mul, const float (*vals)[4],
                                               const float (*vals_u)[4]) {
   const int g = lane >> 2, t = lane & 3;
-  const float gmul = FMT == 1 ? __ldg(p.g) : 1.f;
+  const float gmul = FMT != 0 ? __ldg(p.g) : 1.f;   // NVFP4 and FP8: per-tensor scale
   const int n0 = band * 16 + g;
   const int cols = FUSE ? p.I : p.N;             // output columns (row stride of y)
   if (p.S == 1) {
@@ -369,7 +404,9 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
   using C = Cfg<FMT, MT, FUSE>;
   constexpr int kSB1 = stage_bytes(FMT);       // one band's group
   constexpr int kSB = kSB1 * (FUSE ? 2 : 1);   // fused: the gate band's group, then the up band's
-  constexpr int kSStep = FMT == 0 ? 32 : 128;  // scale bytes of one band per 128-group
+  constexpr int kSStep = FMT == 0 ? 32 : FMT == 1 ? 128 : 0;  // scale bytes of a band per 128-group
+  constexpr int kGB = group_bytes(FMT);         // weight bytes of a band per 128-group
+  constexpr int kTPG = kGB / kTileBytes;        // tiles per group
   extern __shared__ __align__(128) uint8_t smem[];
   float* row_mul = reinterpret_cast<float*>(smem);
   unsigned* row_aux = reinterpret_cast<unsigned*>(smem + kRowAuxOff);
@@ -405,13 +442,16 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
   // two bands (pieces are padded to whole blocks), so its groups sit at fixed
   // offsets from one pointer; padding groups copy nothing.
   const int b0 = min(band_lo + wi, p.NT - 1);
-  const uint8_t* cw = p.w + ((size_t)b0 * KB + 2 * gk0) * kTileBytes + lane * 16;
-  const uint8_t* cs = FMT == 0 ? p.s + ((size_t)b0 * (p.K >> 7) + gk0) * 32 + g * 4
-                               : p.s + ((size_t)b0 * KB + 2 * gk0) * 64 + g * 8;
+  const size_t tpb = (size_t)KB * (kTPG / 2);  // tiles per band
+  const uint8_t* cw = p.w + ((size_t)b0 * tpb + kTPG * gk0) * kTileBytes + lane * 16;
+  const uint8_t* cs = FMT == 0   ? p.s + ((size_t)b0 * (p.K >> 7) + gk0) * 32 + g * 4
+                      : FMT == 1 ? p.s + ((size_t)b0 * KB + 2 * gk0) * 64 + g * 8
+                                 : p.s;   // FP8: no packed scales
   // from the last block of a piece to the first block of the next band's piece
-  const int wjump = p.wn * KB * kTileBytes - (ngp - D) * kGroupBytes;
-  const int sjump = FMT == 0 ? p.wn * (p.K >> 7) * 32 - (ngp - D) * 32
-                             : p.wn * KB * 64 - (ngp - D) * 128;
+  const int wjump = p.wn * (int)tpb * kTileBytes - (ngp - D) * kGB;
+  const int sjump = FMT == 0   ? p.wn * (p.K >> 7) * 32 - (ngp - D) * 32
+                    : FMT == 1 ? p.wn * KB * 64 - (ngp - D) * 128
+                               : 0;
   const int nbp = ngp / D;                     // blocks per piece
   int c_blocks = my_rounds * nbp;              // blocks still to copy
   int c_bb = 0;                                // block index of the cursor within its piece
@@ -419,22 +459,22 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
   auto copy_item = [&](int k) {                // group k of the cursor block -> slot k
     if (c_blocks > 0 && c_bb * D + k < ng) {
       const uint32_t d = ring_s + k * kSB;
-      cpa16(d, cw + k * kGroupBytes, pol);
-      cpa16(d + kTileBytes, cw + k * kGroupBytes + kTileBytes, pol);
+#pragma unroll
+      for (int i = 0; i < kTPG; ++i) cpa16(d + i * kTileBytes, cw + k * kGB + i * kTileBytes, pol);
       if (FMT == 0) {
         cpa4(d + kGroupBytes - lane * 12, cs + k * kSStep);   // scale slot: lane * 4
-      } else {
+      } else if (FMT == 1) {
         cpa8(d + kGroupBytes, cs + k * kSStep);
         cpa8(d + kGroupBytes + 8, cs + k * kSStep + 64);
       }
       if (FUSE) {
-        const uint8_t* uw = cw + p.up_w + k * kGroupBytes;
+        const uint8_t* uw = cw + p.up_w + k * kGB;
         const uint8_t* us = cs + p.up_s + k * kSStep;
-        cpa16(d + kSB1, uw, pol);
-        cpa16(d + kSB1 + kTileBytes, uw + kTileBytes, pol);
+#pragma unroll
+        for (int i = 0; i < kTPG; ++i) cpa16(d + kSB1 + i * kTileBytes, uw + i * kTileBytes, pol);
         if (FMT == 0) {
           cpa4(d + kSB1 + kGroupBytes - lane * 12, us);
-        } else {
+        } else if (FMT == 1) {
           cpa8(d + kSB1 + kGroupBytes, us);
           cpa8(d + kSB1 + kGroupBytes + 8, us + 64);
         }
@@ -450,7 +490,7 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
         cw += wjump;
         cs += sjump;
       } else {
-        cw += D * kGroupBytes;
+        cw += D * kGB;
         cs += D * kSStep;
       }
     }
@@ -504,7 +544,10 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
             const uint8_t* xg[MT];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) xg[mt] = xb[mt] + k * 256;
-            if (FMT == 0) {
+            if (FMT == kFmtFp8) {
+              group_fp8<MT>(st, xg, acc);
+              if (FUSE) group_fp8<MT>(st + kSB1, xg, acc_u);
+            } else if (FMT == 0) {
               cur.s0.x = *reinterpret_cast<const uint32_t*>(st + kGroupBytes - lane * 12);
               group_int4<MT>(cur, xg, acc);
             } else {
@@ -518,7 +561,7 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) xg[mt] -= 128;
             }
-            if (FUSE) {                 // the up band's group, same activations
+            if (FUSE && FMT != kFmtFp8) {   // the up band's group, same activations
               const uint8_t* su = st + kSB1;
               GroupWords up;
               up.w0 = *reinterpret_cast<const uint4*>(su);
@@ -628,8 +671,9 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   p.I = a.N / 2;
   p.NT = FUSE ? p.I / 16 : (a.N + 15) / 16;    // fused: bands of gate rows
   const size_t KB = (size_t)a.K / 64;
-  p.up_w = (size_t)(p.I / 16) * KB * kTileBytes;
-  p.up_s = FMT == 0 ? (size_t)(p.I / 16) * (a.K / 128) * 32 : (size_t)(p.I / 16) * KB * 64;
+  p.up_w = (size_t)(p.I / 16) * KB * (FMT == kFmtFp8 ? 2 : 1) * kTileBytes;
+  p.up_s = FMT == 0 ? (size_t)(p.I / 16) * (a.K / 128) * 32
+           : FMT == 1 ? (size_t)(p.I / 16) * KB * 64 : 0;
   p.S = pl.S;
   p.kslice = pl.kslice;
   p.bq = p.NT / pl.ctas_x;
@@ -639,7 +683,7 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   p.wn_log2 = ilog2(pl.wn);
   p.wk_log2 = ilog2(pl.wk);
   p.ngp = pl.ngp;
-  if constexpr (FUSE) {                         // stages are twice as large: D <= 4
+  if constexpr (FUSE || FMT == kFmtFp8) {       // stages two or four times as large: D <= 4
     switch (pl.depth) {
       case 2: return launch_d<FMT, MT, 2, FUSE>(p, pl, st);
       case 3: return launch_d<FMT, MT, 3, FUSE>(p, pl, st);
@@ -667,12 +711,9 @@ int warps_of(int fmt, int mt) {
 }
 
 int header_of(int fmt, int mt, int fuse) {
-  if (fuse) {
-    if (fmt == 0) return mt == 1 ? Cfg<0, 1, true>::kHeader : Cfg<0, 2, true>::kHeader;
-    return mt == 1 ? Cfg<1, 1, true>::kHeader : Cfg<1, 2, true>::kHeader;
-  }
-  if (fmt == 0) return mt == 1 ? Cfg<0, 1>::kHeader : Cfg<0, 2>::kHeader;
-  return mt == 1 ? Cfg<1, 1>::kHeader : Cfg<1, 2>::kHeader;
+  (void)fmt;   // the header depends on the row tiles and fusion only
+  if (fuse) return mt == 1 ? Cfg<0, 1, true>::kHeader : Cfg<0, 2, true>::kHeader;
+  return mt == 1 ? Cfg<0, 1>::kHeader : Cfg<0, 2>::kHeader;
 }
 
 }  // namespace
@@ -693,8 +734,9 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms, int fuse) {
   const int header = header_of(fmt, pl.mt, fuse);
   const int sb = stage_bytes(fmt) * (fuse ? 2 : 1);   // fused: gate and up group per stage
   const int NT = fuse ? N / 32 : (N + 15) / 16;       // fused: bands of the I gate rows
-  const int depth_cap = fuse ? 4 : kMaxDepth;
-  const double per_group = fuse ? 4.0 : 2.0;          // two bands' bytes per fused group
+  const int depth_cap = (fuse || fmt == kFmtFp8) ? 4 : kMaxDepth;
+  // cost per group in units of one 4-bit band-group (1 KB): x2 fused, x2 FP8
+  const double per_group = 2.0 * (fuse ? 2 : 1) * (fmt == kFmtFp8 ? 2 : 1);
   const int groups = K / 128;
   double best = 1e300;
   pl.S = 0;
@@ -762,6 +804,10 @@ size_t gemv_workspace_floats(const GemvPlan& p, int M, int N) {
 size_t gemv_counters(const GemvPlan& p, int N) { return p.S > 1 ? (N + 15) / 16 : 0; }
 
 cudaError_t launch_gemv(const GemvPlan& p, const GemmArgs& a, cudaStream_t st) {
+  if (a.fmt == kFmtFp8) {
+    if (a.fuse) return p.mt == 1 ? launch_t<2, 1, true>(p, a, st) : launch_t<2, 2, true>(p, a, st);
+    return p.mt == 1 ? launch_t<2, 1, false>(p, a, st) : launch_t<2, 2, false>(p, a, st);
+  }
   if (a.fuse) {
     if (a.fmt == 0) return p.mt == 1 ? launch_t<0, 1, true>(p, a, st) : launch_t<0, 2, true>(p, a, st);
     return p.mt == 1 ? launch_t<1, 1, true>(p, a, st) : launch_t<1, 2, true>(p, a, st);

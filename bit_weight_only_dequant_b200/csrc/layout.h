@@ -24,6 +24,14 @@
 //   INT4 nibble = q + 8 (offset binary); NVFP4 nibble = e2m1 code.
 //   Rows n >= N (padding up to a multiple of 16) hold value 0 and scale 0.
 //
+// FP8-E4M3 (one byte per weight, one fp32 scale per tensor, no packed
+// scales): the same pairs, a byte per element, so a 512-byte tile covers 16
+// rows x 32 k.  Tile (nt, kt), kt = k / 32, at ((nt * K/32) + kt) * 512; lane
+// L = 4g + t owns the 16 bytes at 16 L: for k16 sub-block j (0, 1) of the
+// tile, word 2j holds P0 (bytes 0, 1) and P1 (bytes 2, 3), word 2j + 1 holds
+// P2 and P3, first element in the lower byte: the operand order of the
+// hardware e4m3x2 -> f16x2 conversion.  A 128-group of a band is four tiles.
+//
 // Scales:
 //   INT4: per (nt, group gi = k / 128), 32 bytes at (nt * (K/128) + gi) * 32;
 //         BF16 of row nt*16 + g + 8h at byte 4g + 2h (h = 0, 1), so lane
@@ -50,13 +58,30 @@ constexpr int kInt4Group = 128;
 constexpr int kNvfp4Group = 16;
 constexpr int kInt4ScaleBlockBytes = 32;   // per (nt, 128-group)
 constexpr int kNvfp4ScaleBlockBytes = 64;  // per (nt, k64 block)
+constexpr int kFmtFp8 = 2;                 // FP8-E4M3 weights, per-tensor fp32 scale
 
 W4_HD int64_t padded_rows(int64_t N) { return (N + 15) / 16 * 16; }
 
-W4_HD int64_t weight_bytes(int64_t N, int64_t K) { return padded_rows(N) * K / 2; }
+W4_HD int64_t weight_bytes(int fmt, int64_t N, int64_t K) {
+  return fmt == kFmtFp8 ? padded_rows(N) * K : padded_rows(N) * K / 2;
+}
 
 W4_HD int64_t scale_bytes(int fmt, int64_t N, int64_t K) {
+  if (fmt == kFmtFp8) return 0;
   return fmt == 0 ? padded_rows(N) * (K / kInt4Group) * 2 : padded_rows(N) * (K / kNvfp4Group);
+}
+
+// Byte offset of element (n, k) in packed FP8-E4M3 weights.
+W4_HD int64_t fp8_pos(int64_t n, int64_t k, int64_t K) {
+  const int64_t nt = n >> 4, kt = k >> 5;
+  const int r = (int)(n & 15), kk = (int)(k & 31);
+  const int g = r & 7, hi_row = r >> 3;
+  const int j = kk >> 4, kin = kk & 15;
+  const int t = kin >> 2, e = kin & 3;
+  const int pair = hi_row + 2 * (e >> 1);        // P0..P3
+  const int second = e & 1;
+  const int word = 2 * j + (pair >> 1);
+  return ((nt * (K >> 5) + kt) * 512) + (4 * g + t) * 16 + word * 4 + 2 * (pair & 1) + second;
 }
 
 // Position of element (n, k) in the packed weights: byte offset and nibble

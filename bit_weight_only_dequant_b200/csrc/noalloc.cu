@@ -70,14 +70,16 @@ int noalloc_setup(NoAllocDevice** out) {
 extern "C" int w4a16_gemm_noalloc(int fmt, int M, int N, int K, const void* x_bf16,
                                   const void* packed_w, const void* packed_scales,
                                   const float* global_scale, void* y_bf16, void* stream) {
-  if (fmt != W4A16_FMT_INT4_G128 && fmt != W4A16_FMT_NVFP4_G16) return W4A16_ERR_ARG;
+  if (fmt != W4A16_FMT_INT4_G128 && fmt != W4A16_FMT_NVFP4_G16 && fmt != W4A16_FMT_FP8_E4M3)
+    return W4A16_ERR_ARG;
   if (N < 1 || K < 128 || K % 128 != 0) return W4A16_ERR_SHAPE;
   if ((long long)((N + 15) / 16) * (K / 64) >= (1ll << 31) / 64) return W4A16_ERR_SHAPE;
   if (M < 1 || M > W4A16_GEMV_MAX_M) return W4A16_ERR_SHAPE;
-  if (!x_bf16 || !packed_w || !packed_scales || !y_bf16) return W4A16_ERR_ARG;
-  if ((fmt == W4A16_FMT_NVFP4_G16) != (global_scale != nullptr)) return W4A16_ERR_ARG;
+  const bool scaled = fmt != W4A16_FMT_FP8_E4M3;   // FP8 has no packed scales
+  if (!x_bf16 || !packed_w || !y_bf16 || (scaled && !packed_scales)) return W4A16_ERR_ARG;
+  if ((fmt != W4A16_FMT_INT4_G128) != (global_scale != nullptr)) return W4A16_ERR_ARG;
   const uintptr_t mis = reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(packed_w) |
-                        reinterpret_cast<uintptr_t>(packed_scales) |
+                        (scaled ? reinterpret_cast<uintptr_t>(packed_scales) : 0) |
                         reinterpret_cast<uintptr_t>(y_bf16);
   if (mis & 15u) return W4A16_ERR_ALIGN;
 

@@ -15,8 +15,18 @@ int pack_host(int fmt, int N, int K, const void* codes_v, const void* scales_v, 
   const int64_t Np = padded_rows(N);
   uint8_t* w = static_cast<uint8_t*>(w_v);
   uint8_t* s = static_cast<uint8_t*>(s_v);
-  // padding rows: value 0 (int4 nibble 8, e2m1 code 0), scale 0
-  memset(w, 0, (size_t)weight_bytes(N, K));
+  // padding rows: value 0 (int4 nibble 8, e2m1 / e4m3 code 0), scale 0
+  memset(w, 0, (size_t)weight_bytes(fmt, N, K));
+  if (fmt == kFmtFp8) {
+    const uint8_t* c = static_cast<const uint8_t*>(codes_v);
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t k = 0; k < K; ++k) {
+        const uint8_t b = c[n * K + k];
+        if ((b & 0x7Fu) == 0x7Fu) return -1;  // E4M3 NaN
+        w[fp8_pos(n, k, K)] = b;
+      }
+    return 0;
+  }
   memset(s, 0, (size_t)scale_bytes(fmt, N, K));
   if (fmt == 0) {
     const int8_t* q = static_cast<const int8_t*>(codes_v);
@@ -63,6 +73,12 @@ int unpack_host(int fmt, int N, int K, const void* w_v, const void* s_v, void* c
                 void* scales_v) {
   const uint8_t* w = static_cast<const uint8_t*>(w_v);
   const uint8_t* s = static_cast<const uint8_t*>(s_v);
+  if (fmt == kFmtFp8) {
+    for (int64_t n = 0; n < N; ++n)
+      for (int64_t k = 0; k < K; ++k)
+        static_cast<uint8_t*>(codes_v)[n * K + k] = w[fp8_pos(n, k, K)];
+    return 0;
+  }
   for (int64_t n = 0; n < N; ++n)
     for (int64_t k = 0; k < K; ++k) {
       const NibblePos pos = weight_pos(fmt, n, k, K);
@@ -133,6 +149,40 @@ __global__ void pack_weights_kernel(int N, int K, const uint8_t* __restrict__ co
   }
 }
 
+// FP8: one thread per (32-k tile, lane), 16 codes of its two rows.
+__global__ void pack_fp8_kernel(int N, int K, const uint8_t* __restrict__ codes,
+                                uint8_t* __restrict__ w) {
+  const int KT = K >> 5;
+  const long long total = (long long)((N + 15) / 16) * KT * 32;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int lane = (int)(idx & 31);
+    const long long tile = idx >> 5;
+    const long long nt = tile / KT;
+    const int kt = (int)(tile - nt * KT);
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+      for (int hrow = 0; hrow < 2; ++hrow) {
+        const long long n = nt * 16 + g + 8 * hrow;
+        const int k0 = kt * 32 + j * 16 + 4 * t;
+        const uint32_t four =
+            n < N ? *reinterpret_cast<const uint32_t*>(codes + n * (long long)K + k0) : 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pair = hrow + 2 * (e >> 1), second = e & 1;
+          const int byte = 2 * (pair & 1) + second;
+          wd[2 * j + (pair >> 1)] |= ((four >> (8 * e)) & 0xFFu) << (8 * byte);
+        }
+      }
+    }
+    *reinterpret_cast<uint4*>(w + tile * kTileBytes + lane * 16) =
+        make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  }
+}
+
 template <int FMT>
 __global__ void pack_scales_kernel(int N, int K, const uint8_t* __restrict__ scales,
                                    uint8_t* __restrict__ s) {
@@ -156,6 +206,12 @@ __global__ void pack_scales_kernel(int N, int K, const uint8_t* __restrict__ sca
 
 cudaError_t launch_pack(int fmt, int N, int K, const void* codes, const void* scales, void* w,
                         void* s, cudaStream_t st) {
+  if (fmt == kFmtFp8) {
+    const long long ft = (long long)((N + 15) / 16) * (K / 32) * 32;
+    const unsigned bf = (unsigned)((ft + 255) / 256 < 148 * 32 ? (ft + 255) / 256 : 148 * 32);
+    pack_fp8_kernel<<<bf, 256, 0, st>>>(N, K, (const uint8_t*)codes, (uint8_t*)w);
+    return cudaGetLastError();
+  }
   const long long wt = (long long)((N + 15) / 16) * (K / 64) * 32;
   const long long sc = (long long)((N + 15) / 16 * 16) * (fmt == 0 ? K / 128 : K / 16);
   const unsigned bw = (unsigned)((wt + 255) / 256 < 148 * 32 ? (wt + 255) / 256 : 148 * 32);

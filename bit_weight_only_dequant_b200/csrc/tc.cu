@@ -59,7 +59,11 @@ constexpr int kMaxSmem = 227 * 1024;          // dynamic shared memory limit of 
 
 // Weight ring stage: the group's two tiles (each lane's 16 bytes at 16 lane),
 // then the scales each lane needs (int4: 4 bytes at 4 lane; NVFP4: 2 x 8 at 16 lane).
-__host__ __device__ constexpr int tc_stage_bytes(int fmt) { return kGroupBytesW + (fmt == 0 ? 128 : 512); }
+// FP8-E4M3: four 512-byte tiles per band-group, no packed scales.
+__host__ __device__ constexpr int tc_group_bytes(int fmt) { return fmt == kFmtFp8 ? 4 * kTileBytes : kGroupBytesW; }
+__host__ __device__ constexpr int tc_stage_bytes(int fmt) {
+  return fmt == kFmtFp8 ? tc_group_bytes(fmt) : kGroupBytesW + (fmt == 0 ? 128 : 512);
+}
 
 struct TcParams {
   const uint8_t* w;
@@ -443,7 +447,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * q + 16 * bp) << 16;
     const uint64_t pol = policy_evict_first();
     const int G = p.K >> 7;
-    constexpr int kSStep = FMT == 0 ? 32 : 128;          // one band's scale bytes per group
+    constexpr int kSStep = FMT == 0 ? 32 : FMT == 1 ? 128 : 0;   // one band's scale bytes per group
+    constexpr int kGB = tc_group_bytes(FMT);             // one band's weight bytes per group
+    constexpr int kTPG = kGB / kTileBytes;
 
     // copy cursor over this warp's groups: (unit, group) in the CTA's order
     uint8_t* ring = Wr + warp * kWRing * kSB;
@@ -462,9 +468,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         c_nb = p.fuse ? (h ? p.I >> 4 : 0) + tile * 8 + (band & 7) : tile * 16 + band;
         c_valid = p.fuse ? tile * 8 + (band & 7) < (p.I >> 4) : c_nb < p.NT;
         const int nb = min(c_nb, p.NT - 1);
-        cw = p.w + ((size_t)nb * p.KB + 2 * g_lo) * kTileBytes + lane * 16;
-        cs = FMT == 0 ? p.s + ((size_t)nb * G + g_lo) * 32 + g * 4
-                      : p.s + ((size_t)nb * p.KB + 2 * g_lo) * 64 + g * 8;
+        cw = p.w + ((size_t)nb * p.KB * (kTPG / 2) + kTPG * g_lo) * kTileBytes + lane * 16;
+        cs = FMT == 0   ? p.s + ((size_t)nb * G + g_lo) * 32 + g * 4
+             : FMT == 1 ? p.s + ((size_t)nb * p.KB + 2 * g_lo) * 64 + g * 8
+                        : p.s;
       }
     };
     c_start();
@@ -473,16 +480,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (c_unit < p.units) {
         if (c_valid) {
           const uint32_t d = ring_s + (c_it % kWRing) * kSB;
-          cpa16(d, cw, pol);
-          cpa16(d + kTileBytes, cw + kTileBytes, pol);
+#pragma unroll
+          for (int i = 0; i < kTPG; ++i) cpa16(d + i * kTileBytes, cw + i * kTileBytes, pol);
           if (FMT == 0) {
             cpa4(d + kGroupBytesW - lane * 12, cs);       // scale slot: lane * 4
-          } else {
+          } else if (FMT == 1) {
             cpa8(d + kGroupBytesW, cs);
             cpa8(d + kGroupBytesW + 8, cs + 64);
           }
         }
-        cw += kGroupBytesW;
+        cw += kGB;
         cs += kSStep;
         if (++c_gi == c_hi) {
           c_unit += gridDim.x;
@@ -506,12 +513,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t ua = it / kASlots;
         cpa_wait<kWRing - 1>();                          // this lane's bytes of group `it`
         const uint8_t* st = ring + (it % kWRing) * kSB;
-        uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+        uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0, w2 = w0, w3 = w0;
         uint32_t sv0 = 0, sv1 = 0, sv2 = 0, sv3 = 0;
         if (real_band) {
           w0 = *reinterpret_cast<const uint4*>(st + lane * 16);
           w1 = *reinterpret_cast<const uint4*>(st + kTileBytes + lane * 16);
-          if (FMT == 0) {
+          if (FMT == kFmtFp8) {
+            w2 = *reinterpret_cast<const uint4*>(st + 2 * kTileBytes + lane * 16);
+            w3 = *reinterpret_cast<const uint4*>(st + 3 * kTileBytes + lane * 16);
+          } else if (FMT == 0) {
             sv0 = *reinterpret_cast<const uint32_t*>(st + kGroupBytesW + lane * 4);
           } else {
             const uint4 sv = *reinterpret_cast<const uint4*>(st + kGroupBytesW + lane * 16);
@@ -530,7 +540,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint4 wv = blk ? w1 : w0;
           const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
           uint32_t r[16];
-          if (FMT == 0) {
+          if (FMT == kFmtFp8) {
+            // 64-block blk = tiles 2 blk and 2 blk + 1; k16 sub-block k uses
+            // words 2 (k & 1) (P0, P1) and 2 (k & 1) + 1 (P2, P3) of tile
+            // 2 blk + (k >> 1); exact e4m3 -> f16, the scale is per tensor
+            const uint4 ta = blk ? w2 : w0, tb = blk ? w3 : w1;
+            const uint32_t fw[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t wa = fw[2 * k], wb = fw[2 * k + 1];
+              r[4 * k + 0] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa));
+              r[4 * k + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb));
+              r[4 * k + 2] = e4m3x2_to_f16x2(static_cast<uint16_t>(wa >> 16));
+              r[4 * k + 3] = e4m3x2_to_f16x2(static_cast<uint16_t>(wb >> 16));
+            }
+          } else if (FMT == 0) {
             const uint32_t s_lo = prmt(sv0, sv0, 0x1010u);  // (s_g, s_g)
             const uint32_t s_hi = prmt(sv0, sv0, 0x3232u);  // (s_g8, s_g8)
 #pragma unroll
@@ -577,7 +601,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int xrow = chunk * p.rows;
       const int mlim = min(p.rows, p.M - xrow);          // rows of this chunk
       float gmul = 1.f;
-      if (FMT == 1) gmul = __ldg(p.g);
+      if (FMT != 0) gmul = __ldg(p.g);                   // NVFP4 and FP8: per-tensor scale
       const size_t Npad = (size_t)p.NT * 16;
       if (p.fuse && p.S == 1) {
         // fused, not split: every warp reads gate (half 0) and up (half 1) for
@@ -600,7 +624,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < kEQ; ++c, hp += p.I) {
               if (mq + c0 + c < mlim) {
                 float gv = v[c], uv = u[c];
-                if (FMT == 1) {
+                if (FMT != 0) {
                   const float rm = __ldg(p.row_mul + mb + c);
                   gv = gv * rm * gmul;
                   uv = uv * rm * gmul;
@@ -624,7 +648,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               for (int c = 0; c < kEC; ++c, yp += p.N) {
                 if (m0 + c0 + c < mlim) {
                   float val = v[c];
-                  if (FMT == 1) val = val * __ldg(p.row_mul + mb + c) * gmul;
+                  if (FMT != 0) val = val * __ldg(p.row_mul + mb + c) * gmul;
                   *yp = __float2bfloat16_rn(val);
                 }
               }
@@ -755,7 +779,7 @@ __global__ void __launch_bounds__(256)
   sum_splits4(ws + (size_t)m * Npad + n0, sstride, S, a);
   if (FUSE) sum_splits4(ws + (size_t)m * Npad + cols + n0, sstride, S, u);
   float rm = 1.f, gm = 1.f;
-  if (FMT == 1) {
+  if (FMT != 0) {
     rm = __ldg(row_mul + m);
     gm = __ldg(g);
   }
@@ -763,10 +787,10 @@ __global__ void __launch_bounds__(256)
   for (int j = 0; j < 4; ++j) {
     if (n0 + j < cols) {
       float val = a[j];
-      if (FMT == 1) val = val * rm * gm;
+      if (FMT != 0) val = val * rm * gm;
       if (FUSE) {
         float uv = u[j];
-        if (FMT == 1) uv = uv * rm * gm;
+        if (FMT != 0) uv = uv * rm * gm;
         val = silu_f32(val) * uv;
       }
       y[(size_t)m * cols + n0 + j] = __float2bfloat16_rn(val);
@@ -808,7 +832,7 @@ template <int FMT, int MPAD>
 cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, const float* row_mul,
                      cudaStream_t st) {
   CUtensorMap map;
-  if (!make_xmap(&map, xsrc, a.M, a.K, MPAD, FMT == 1)) return cudaErrorInvalidValue;
+  if (!make_xmap(&map, xsrc, a.M, a.K, MPAD, FMT != 0)) return cudaErrorInvalidValue;
   TcParams p;
   p.w = static_cast<const uint8_t*>(a.w);
   p.s = static_cast<const uint8_t*>(a.s);
@@ -879,6 +903,12 @@ cudaError_t launch_fmt(const TcPlan& pl, const GemmArgs& a, const void* xsrc, co
   }
 }
 
+template <int MPAD>
+int tc_smem(int fmt) {
+  return fmt == 0 ? TcShape<0, MPAD>::kSmem
+         : fmt == 1 ? TcShape<1, MPAD>::kSmem : TcShape<kFmtFp8, MPAD>::kSmem;
+}
+
 }  // namespace
 
 // Splits K so that the units (256-row tiles x row chunks x K splits, whole
@@ -916,14 +946,14 @@ TcPlan plan_tc(int fmt, int M, int N, int K, int num_sms, int fuse) {
   pl.grid = pl.units < num_sms ? pl.units : num_sms;
   int smem = 0;
   switch (pl.mpad) {
-    case 16: smem = fmt == 0 ? TcShape<0, 16>::kSmem : TcShape<1, 16>::kSmem; break;
-    case 32: smem = fmt == 0 ? TcShape<0, 32>::kSmem : TcShape<1, 32>::kSmem; break;
-    case 48: smem = fmt == 0 ? TcShape<0, 48>::kSmem : TcShape<1, 48>::kSmem; break;
-    case 64: smem = fmt == 0 ? TcShape<0, 64>::kSmem : TcShape<1, 64>::kSmem; break;
-    case 80: smem = fmt == 0 ? TcShape<0, 80>::kSmem : TcShape<1, 80>::kSmem; break;
-    case 96: smem = fmt == 0 ? TcShape<0, 96>::kSmem : TcShape<1, 96>::kSmem; break;
-    case 112: smem = fmt == 0 ? TcShape<0, 112>::kSmem : TcShape<1, 112>::kSmem; break;
-    default: smem = fmt == 0 ? TcShape<0, 128>::kSmem : TcShape<1, 128>::kSmem; break;
+    case 16: smem = tc_smem<16>(fmt); break;
+    case 32: smem = tc_smem<32>(fmt); break;
+    case 48: smem = tc_smem<48>(fmt); break;
+    case 64: smem = tc_smem<64>(fmt); break;
+    case 80: smem = tc_smem<80>(fmt); break;
+    case 96: smem = tc_smem<96>(fmt); break;
+    case 112: smem = tc_smem<112>(fmt); break;
+    default: smem = tc_smem<128>(fmt); break;
   }
   pl.smem = smem;
   return pl;
@@ -940,10 +970,10 @@ size_t tc_counters(const TcPlan& p, int N) {
 }
 
 size_t tc_x_f16_bytes(int fmt, int M, int K) {
-  return fmt == 1 ? (size_t)M * K * 2 + (size_t)M * sizeof(float) : 0;
+  return fmt != 0 ? (size_t)M * K * 2 + (size_t)M * sizeof(float) : 0;
 }
 
-// NVFP4 first rescales all M rows into FP16 (one launch); then one launch of
+// NVFP4 and FP8 first rescale all M rows into FP16 (one launch); then one launch of
 // the tensor-core kernel covers every chunk of rows (plus, when K is split,
 // one reduction launch).
 cudaError_t launch_tc(const TcPlan& pl, const GemmArgs& a, void* xf16_scratch, cudaStream_t st) {
@@ -953,7 +983,7 @@ cudaError_t launch_tc(const TcPlan& pl, const GemmArgs& a, void* xf16_scratch, c
   prep_x_f16_kernel<<<a.M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x), xh, rm, a.K);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_fmt<1>(pl, a, xh, rm, st);
+  return a.fmt == 1 ? launch_fmt<1>(pl, a, xh, rm, st) : launch_fmt<kFmtFp8>(pl, a, xh, rm, st);
 }
 
 }  // namespace w4

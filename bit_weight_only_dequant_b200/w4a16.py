@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(HERE, "libw4a16.so")
 
 FMT_INT4_G128 = 0
 FMT_NVFP4_G16 = 1
-FMTS = {"int4": FMT_INT4_G128, "nvfp4": FMT_NVFP4_G16}
+FMT_FP8_E4M3 = 2
+FMTS = {"int4": FMT_INT4_G128, "nvfp4": FMT_NVFP4_G16, "fp8": FMT_FP8_E4M3}
 
 OK = 0
 ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_DEVICE, ERR_CUDA, ERR_TIMEOUT, ERR_NOMEM = -1, -2, -3, -4, -5, -6, -7

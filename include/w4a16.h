@@ -53,8 +53,9 @@ extern "C" {
 #endif
 
 /* Weight formats. */
-#define W4A16_FMT_INT4_G128 0
-#define W4A16_FMT_NVFP4_G16 1
+#define W4A16_FMT_INT4_G128 0  /* int4 GPTQ, BF16 scale per 128-group */
+#define W4A16_FMT_NVFP4_G16 1  /* e2m1, E4M3 scale per 16-group, fp32 per-tensor scale */
+#define W4A16_FMT_FP8_E4M3 2   /* E4M3 weights (W8A16), fp32 per-tensor scale, no packed scales */
 
 /* Status codes. */
 #define W4A16_OK 0
@@ -84,18 +85,22 @@ extern "C" {
  * time).
  */
 
-/* Bytes of the packed weight buffer: ceil(N/16)*16 * K / 2.  0 on bad args. */
+/* Bytes of the packed weight buffer: ceil(N/16)*16 * K / 2 (4-bit formats),
+ * ceil(N/16)*16 * K (FP8).  0 on bad args. */
 size_t w4a16_packed_weight_bytes(int fmt, int N, int K);
 
 /* Bytes of the packed scale buffer: INT4 ceil(N/16)*16 * K/128 * 2;
- * NVFP4 ceil(N/16)*16 * K/16.  0 on bad args. */
+ * NVFP4 ceil(N/16)*16 * K/16; FP8 0 (one per-tensor scale, passed to the
+ * matmul as global_scale).  0 on bad args. */
 size_t w4a16_packed_scale_bytes(int fmt, int N, int K);
 
 /*
  * Host-side packer: logical checkpoint tensors -> the library's packed layout.
- *   codes:  INT4: int8 q[N][K] in [-8, 7];  NVFP4: uint8 e2m1 codes c[N][K] in 0..15.
+ *   codes:  INT4: int8 q[N][K] in [-8, 7];  NVFP4: uint8 e2m1 codes c[N][K] in 0..15;
+ *           FP8: uint8 E4M3 bytes w8[N][K] (0x7F/0xFF NaN patterns rejected).
  *   scales: INT4: BF16 bit patterns (uint16) s[N][K/128];
- *           NVFP4: E4M3 bytes s8[N][K/16] (0x7F/0xFF NaN patterns rejected).
+ *           NVFP4: E4M3 bytes s8[N][K/16] (0x7F/0xFF NaN patterns rejected);
+ *           FP8: unused (may be NULL), as is packed_scales.
  *   packed_w / packed_scales: host buffers of the sizes above.
  * All pointers are host pointers.  Returns W4A16_ERR_ARG on an out-of-range
  * code or scale (nothing useful is left in the outputs then).
@@ -110,7 +115,8 @@ int w4a16_unpack_host(int fmt, int N, int K, const void* packed_w, const void* p
 /*
  * Device-side packer: same layouts as w4a16_pack_host, all four pointers are
  * device pointers, asynchronous on `stream`.  Codes outside the format's range
- * are not detected (only their low 4 bits are stored).
+ * are not detected (4-bit formats store only the low 4 bits; FP8 NaN bytes
+ * are stored as they are).  FP8: scales and packed_scales unused (may be NULL).
  */
 int w4a16_pack(int fmt, int N, int K, const void* codes, const void* scales,
                void* packed_w, void* packed_scales, void* stream);
@@ -118,7 +124,8 @@ int w4a16_pack(int fmt, int N, int K, const void* codes, const void* scales,
 /*
  * Dequantise to BF16, bit-exact:
  *   w_bf16[n][k] = W_deq[n][k] for n < N, k < K (row-major [N][K], device).
- * global_scale: NVFP4: device pointer to one fp32 g; INT4: must be NULL.
+ * global_scale: NVFP4 and FP8: device pointer to one fp32 g; INT4: must be NULL.
+ * FP8: W_deq = RNE_bf16(e4m3 * g); packed_scales unused (may be NULL).
  */
 int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packed_scales,
                   const float* global_scale, void* w_bf16, void* stream);
@@ -126,8 +133,9 @@ int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packe
 /*
  * The matmul: y[M][N] = x[M][K] . W_deq[N][K]^T.
  *   x_bf16:   device, [M][K] BF16 row-major, 16-byte aligned.
- *   packed_w, packed_scales: device, produced by a packer above, 16-byte aligned.
- *   global_scale: NVFP4: device pointer to one fp32 g; INT4: must be NULL.
+ *   packed_w, packed_scales: device, produced by a packer above, 16-byte aligned
+ *             (FP8: packed_scales unused, may be NULL).
+ *   global_scale: NVFP4 and FP8: device pointer to one fp32 g; INT4: must be NULL.
  *   y_bf16:   device, [M][N] BF16 row-major; must not overlap any input.
  * Picks the kernel by row count (W4A16_PATH_AUTO): the split-K GEMV for
  * M <= 8, and for 9 <= M <= 16 when N >= 16384; the tensor-core path

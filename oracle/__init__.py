@@ -9,7 +9,7 @@ What it computes (plain definitions, no blocking, no fusion):
 * ``formats``: decoders of the storage types named by the checkpoint
   contracts (BF16, OCP FP8-E4M3, FP4-E2M1) and round-to-nearest-even onto
   BF16 from an exact binary64 value.
-* ``w4a16``: dequantisation of the two checkpoint formats into BF16 weights
+* ``w4a16``: dequantisation of the checkpoint formats (int4, NVFP4, FP8) into BF16 weights
   (one rounding of the exact product), then y = x . W_deq^T accumulated in
   fp64, plus the per-element tolerance bound sum_k |W_deq[n][k] * x[m][k]|;
   and the fused gate/up layer h = SiLU(gate) * up with its tolerance.
@@ -23,6 +23,7 @@ from .formats import bf16_to_f64, e4m3_to_f64, e2m1_to_f64, f64_to_bf16_rne  # n
 from .w4a16 import (  # noqa: F401
     dequant_int4_g128,
     dequant_nvfp4,
+    dequant_fp8_e4m3,
     gemm_ref,
     abs_bound,
     within_tolerance,

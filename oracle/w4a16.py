@@ -89,6 +89,23 @@ def dequant_nvfp4(codes: np.ndarray, scale_e4m3: np.ndarray, g: float) -> np.nda
     return f64_to_bf16_rne(e2m1_to_f64(c) * s_per_k * g64)
 
 
+def dequant_fp8_e4m3(codes: np.ndarray, g: float) -> np.ndarray:
+    """W_deq[n][k] = RNE_bf16(e4m3(w8[n][k]) * g); BF16 bits [N][K].
+
+    FP8 weight-only variant (W8A16) of the attention linears, which the NVFP4
+    checkpoint keeps in FP8 (guide "Qwen3.8-27B on DGX Spark (GB10)", section
+    "What Spark-native means").  Reading: E4M3 bytes with one fp32 scale per
+    tensor.  e4m3 (4 significant bits) * fp32 (24) is exact in binary64, so the
+    product is rounded once onto BF16.  w8: uint8 [N][K] (NaN bytes rejected).
+    """
+    c = np.asarray(codes, dtype=np.uint8)
+    v = e4m3_to_f64(c)
+    if not np.all(np.isfinite(v)):
+        raise ValueError("NaN E4M3 weights are not allowed")
+    g64 = float(np.float32(g))
+    return f64_to_bf16_rne(v * g64)
+
+
 def gemm_ref(x_bits: np.ndarray, w_bits: np.ndarray) -> np.ndarray:
     """y_ref[m][n] = sum_k x[m][k] * W_deq[n][k] in binary64 (unrounded).
 

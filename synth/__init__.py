@@ -34,6 +34,9 @@ Value recipes (the workload of the 5120-hidden dense model's linears)
 * NVFP4 group scales (one per 16 K-elements per output column):
   RNE_e4m3(|z| * 0.05), saturating at 448.
 * NVFP4 per-tensor scale: fp32(1/448).
+* FP8-E4M3 weights (W8A16): sign(z) * RNE_e4m3(|z| * 64), z ~ N(0, 1), with
+  the per-tensor scale fp32(1/448).  Drawn on the host only (no CUDA twin);
+  ``device_problem`` copies them to the device.
 """
 
 from __future__ import annotations
@@ -50,6 +53,7 @@ T_S = 2        # int4 bf16 group scales (normal draws)
 T_X = 3        # activations (normal draws)
 T_C = 4        # nvfp4 e2m1 codes
 T_S8 = 5       # nvfp4 e4m3 group scales (normal draws)
+T_W8 = 6       # fp8 e4m3 weights (normal draws)
 
 INT4_GROUP = 128
 NVFP4_GROUP = 16
@@ -176,6 +180,15 @@ def nvfp4_scales(seed: int, N: int, K: int, rows=None) -> np.ndarray:
 
 
 NVFP4_GLOBAL_SCALE = float(np.float32(1.0 / 448.0))
+FP8_GLOBAL_SCALE = float(np.float32(1.0 / 448.0))
+
+
+def fp8_weights(seed: int, N: int, K: int, rows=None) -> np.ndarray:
+    """E4M3 bytes of the weights [len(rows)][K]: sign(z) * RNE_e4m3(|z| * 64)."""
+    rows = np.arange(N, dtype=np.uint64) if rows is None else np.asarray(rows, dtype=np.uint64)
+    idx = rows[:, None] * np.uint64(K) + np.arange(K, dtype=np.uint64)[None, :]
+    z = normals(seed, T_W8, idx)
+    return to_e4m3_bytes(np.abs(z) * 64.0) | np.where(z < 0, 0x80, 0).astype(np.uint8)
 
 
 def problem(fmt: str, seed: int, M: int, N: int, K: int, rows=None) -> dict:
@@ -194,6 +207,10 @@ def problem(fmt: str, seed: int, M: int, N: int, K: int, rows=None) -> dict:
                 "codes": nvfp4_codes(seed, N, K, rows),
                 "scales": nvfp4_scales(seed, N, K, rows),
                 "x": activations(seed, M, K), "g": NVFP4_GLOBAL_SCALE}
+    if fmt == "fp8":
+        return {"fmt": fmt, "M": M, "N": N, "K": K,
+                "codes": fp8_weights(seed, N, K, rows), "scales": None,
+                "x": activations(seed, M, K), "g": FP8_GLOBAL_SCALE}
     raise ValueError(fmt)
 
 
@@ -252,8 +269,16 @@ def device_fill(kind: int, seed: int, tensor_id: int, out, stream=None) -> None:
 
 
 def device_problem(fmt: str, seed: int, M: int, N: int, K: int, device="cuda"):
-    """The tensors of ``problem(fmt, seed, M, N, K)``, drawn on the GPU (torch tensors)."""
+    """The tensors of ``problem(fmt, seed, M, N, K)``, drawn on the GPU (torch tensors).
+
+    FP8 weights have no CUDA twin: they are drawn on the host and copied."""
     import torch
+    if fmt == "fp8":
+        codes = torch.from_numpy(fp8_weights(seed, N, K)).to(device)
+        x = torch.empty((M, K), dtype=torch.int16, device=device)
+        device_fill(KIND_X, seed, T_X, x)
+        return {"fmt": fmt, "M": M, "N": N, "K": K, "codes": codes, "scales": None, "x": x,
+                "g": FP8_GLOBAL_SCALE}
     if fmt == "int4":
         codes = torch.empty((N, K), dtype=torch.int8, device=device)
         scales = torch.empty((N, K // INT4_GROUP), dtype=torch.int16, device=device)

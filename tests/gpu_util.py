@@ -30,7 +30,8 @@ def to_device_problem(p):
     t = torch()
     codes = t.from_numpy(np.ascontiguousarray(p["codes"])).cuda()
     sc = p["scales"]
-    scales = t.from_numpy(np.ascontiguousarray(sc.view(np.int16) if sc.dtype == np.uint16 else sc)).cuda()
+    scales = None if sc is None else t.from_numpy(
+        np.ascontiguousarray(sc.view(np.int16) if sc.dtype == np.uint16 else sc)).cuda()
     x = t.from_numpy(np.ascontiguousarray(p["x"].view(np.int16))).cuda()
     return codes, scales, x
 
@@ -58,6 +59,8 @@ def run_gemm(fmt, codes, scales, x, N, g=None, path=W.PATH_AUTO, y=None):
 def oracle_weights(p):
     if p["fmt"] == "int4":
         return oracle.dequant_int4_g128(p["codes"], p["scales"])
+    if p["fmt"] == "fp8":
+        return oracle.dequant_fp8_e4m3(p["codes"], p["g"])
     return oracle.dequant_nvfp4(p["codes"], p["scales"], p["g"])
 
 

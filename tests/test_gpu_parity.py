@@ -113,6 +113,21 @@ def test_dequant_full_shapes_sampled_rows(fmt, name):
     assert np.array_equal(got, oracle_weights(ph))
 
 
+@pytest.mark.parametrize("g_bits", [0x3B124925, 0x3F800000, 0x3DCCCCCD, 0x0DA24260])
+def test_dequant_fp8_every_code(g_bits):
+    """All 254 finite E4M3 weight bytes, for several per-tensor scales."""
+    t = torch()
+    finite = np.array([b for b in range(256) if (b & 0x7F) != 0x7F], dtype=np.uint8)
+    N, K = 16, 256
+    c = np.resize(finite, (N, K)).astype(np.uint8)
+    g = float(np.array([g_bits], np.uint32).view(np.float32)[0])
+    pw, ps = W.pack_on_device("fp8", N, K, t.from_numpy(c).cuda(), None)
+    got = bf16_bits(W.dequant("fp8", N, K, pw, ps, global_scale=gscale_tensor(g)))
+    want = oracle.dequant_fp8_e4m3(c, g)
+    diff = np.argwhere(got != want)
+    assert diff.size == 0, [(hex(int(c[i, j])), hex(got[i, j]), hex(want[i, j])) for i, j in diff[:8]]
+
+
 # ---------------------------------------------------------------- GEMM parity, full oracle
 
 
@@ -167,6 +182,46 @@ def test_gemm_parity_every_row_count_nvfp4(path, M):
     codes, scales, x = to_device_problem(p)
     y, _ = run_gemm(fmt, codes, scales, x, N, g=p["g"], path=path)
     assert_parity(y, p["x"], oracle_weights(p), f"nvfp4 M={M}")
+
+
+FP8_CASES = [  # M, N, K, path (FP8-E4M3 weights, per-tensor scale)
+    (1, 272, 640, W.PATH_GEMV), (3, 1000, 1024, W.PATH_GEMV), (8, 520, 2048, W.PATH_GEMV),
+    (2, 24, 17408, W.PATH_GEMV), (16, 160, 3072, W.PATH_GEMV), (1, 1, 128, W.PATH_GEMV),
+    (9, 304, 1152, W.PATH_TC), (17, 400, 1536, W.PATH_TC), (64, 272, 640, W.PATH_TC),
+    (33, 48, 12288, W.PATH_TC), (130, 208, 1280, W.PATH_TC), (1, 16, 128, W.PATH_TC),
+]
+
+
+@pytest.mark.parametrize("M,N,K,path", FP8_CASES)
+def test_gemm_parity_fp8(M, N, K, path):
+    p = synth.problem("fp8", 400 + M, M, N, K)
+    codes, scales, x = to_device_problem(p)
+    y, _ = run_gemm("fp8", codes, scales, x, N, g=p["g"], path=path)
+    assert_parity(y, p["x"], oracle_weights(p), f"fp8 M={M} N={N} K={K} path={path}")
+
+
+@pytest.mark.parametrize("fmt,M,I,K,path", [("fp8", 1, 48, 640, W.PATH_GEMV),
+                                            ("fp8", 12, 96, 4096, W.PATH_GEMV),
+                                            ("fp8", 40, 144, 1024, W.PATH_TC),
+                                            ("fp8", 9, 48, 17408, W.PATH_TC)])
+def test_gate_up_silu_parity_fp8(fmt, M, I, K, path):
+    p = synth.problem(fmt, 500 + M, M, 2 * I, K)
+    h = _run_gate_up(fmt, p, I, path)
+    _assert_gate_up_parity(h, p["x"], oracle_weights(p), f"{fmt} M={M} I={I} K={K}")
+
+
+@pytest.mark.parametrize("name,M", [("qkv", 1), ("qkv", 16), ("o", 1), ("o", 64), ("qkv", 200)])
+def test_gemm_parity_fp8_full_shapes_sampled(name, M):
+    K, N = SHAPES[name]
+    t = torch()
+    seed = SEEDS[name]
+    p = synth.device_problem("fp8", seed, M, N, K)
+    y, _ = run_gemm("fp8", p["codes"], p["scales"], p["x"], N, g=p["g"])
+    rows = np.unique(np.concatenate([[0, 15, 16, N - 1], np.random.default_rng(M).integers(0, N, 40)]))
+    ph = synth.problem("fp8", seed, M, N, K, rows=rows)
+    assert_parity(y[:, rows], ph["x"], oracle_weights(ph), f"fp8 {name} M={M}")
+    del p
+    t.cuda.empty_cache()
 
 
 # ---------------------------------------------------------------- GEMM parity at the full shapes

@@ -41,11 +41,14 @@ def test_packed_sizes():
     assert W.w4a16_packed_scale_bytes(1, 8192, 5120) == 8192 * 320
     assert W.w4a16_packed_weight_bytes(0, 17, 128) == 32 * 64          # rows padded to 16
     assert W.w4a16_packed_weight_bytes(0, 16, 100) == 0                 # K not a multiple of 128
-    assert W.w4a16_packed_weight_bytes(2, 16, 128) == 0                 # bad format
+    assert W.w4a16_packed_weight_bytes(3, 16, 128) == 0                 # bad format
+    assert W.w4a16_packed_weight_bytes(2, 8192, 5120) == 8192 * 5120    # FP8: a byte per weight
+    assert W.w4a16_packed_scale_bytes(2, 8192, 5120) == 0               # per-tensor scale only
+    assert W.w4a16_packed_weight_bytes(2, 17, 128) == 32 * 128
 
 
 @pytest.mark.parametrize("fmt,N,K", [("int4", 16, 128), ("int4", 37, 384), ("nvfp4", 16, 128),
-                                     ("nvfp4", 45, 256)])
+                                     ("nvfp4", 45, 256), ("fp8", 16, 128), ("fp8", 45, 384)])
 def test_host_pack_round_trip(fmt, N, K):
     p = synth.problem(fmt, 7, 1, N, K)
     f = W.FMTS[fmt]
@@ -53,10 +56,32 @@ def test_host_pack_round_trip(fmt, N, K):
     s = np.zeros(W.w4a16_packed_scale_bytes(f, N, K), np.uint8)
     assert W.w4a16_pack_host(f, N, K, p["codes"], p["scales"], w, s) == W.OK
     codes = np.zeros_like(p["codes"])
-    scales = np.zeros_like(p["scales"])
+    scales = None if p["scales"] is None else np.zeros_like(p["scales"])
     assert W.w4a16_unpack_host(f, N, K, w, s, codes, scales) == W.OK
     assert np.array_equal(codes, p["codes"])
-    assert np.array_equal(scales, p["scales"])
+    if scales is not None:
+        assert np.array_equal(scales, p["scales"])
+
+
+def test_host_pack_fp8_layout_and_nan_rejection():
+    # FP8: 16 x 32 tiles of 512 bytes; lane 4g + t, k16 sub-block j, words
+    # 2j (P0, P1) and 2j + 1 (P2, P3), a byte per element (restated here)
+    N, K = 32, 128
+    codes = (np.arange(N * K) % 0x7E + 1).astype(np.uint8).reshape(N, K)   # no NaN byte
+    w = np.zeros(W.w4a16_packed_weight_bytes(2, N, K), np.uint8)
+    assert W.w4a16_pack_host(2, N, K, codes, None, w, None) == W.OK
+    for n in range(N):
+        for k in range(K):
+            nt, kt, r, kk = n // 16, k // 32, n % 16, k % 32
+            g, hi, j, kin = r % 8, r // 8, kk // 16, kk % 16
+            t, e = kin // 4, kin % 4
+            pair, second = hi + 2 * (e // 2), e % 2
+            off = ((nt * (K // 32) + kt) * 512 + (4 * g + t) * 16 + (2 * j + pair // 2) * 4
+                   + 2 * (pair % 2) + second)
+            assert w[off] == codes[n, k], (n, k)
+    bad = codes.copy()
+    bad[3, 77] = 0xFF
+    assert W.w4a16_pack_host(2, N, K, bad, None, w, None) == W.ERR_ARG
 
 
 def _layout_position(fmt, n, k, K):
@@ -148,6 +173,8 @@ def test_argument_validation_before_any_device_call():
     assert W.w4a16_gemm(0, 1, 16, 128, None, w, s, None, y, 0) == W.ERR_ARG      # null x
     assert W.w4a16_gemm(0, 1, 16, 128, x, w, s, 1 << 21, y, 0) == W.ERR_ARG      # g for int4
     assert W.w4a16_gemm(1, 1, 16, 128, x, w, s, None, y, 0) == W.ERR_ARG         # no g for nvfp4
+    assert W.w4a16_gemm(2, 1, 16, 128, x, w, None, None, y, 0) == W.ERR_ARG      # no g for fp8
+    assert W.w4a16_gemm(0, 1, 16, 128, x, w, None, None, y, 0) == W.ERR_ARG      # no scales, int4
     assert W.w4a16_gemm(0, 1, 16, 128, x + 2, w, s, None, y, 0) == W.ERR_ALIGN
     assert W.w4a16_gemm_ex(7, 0, 1, 16, 128, x, w, s, None, y, 0) == W.ERR_ARG   # bad path
     assert W.w4a16_dequant(0, 16, 128, w, s, None, y + 8, 0) == W.ERR_ALIGN

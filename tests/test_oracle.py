@@ -430,3 +430,56 @@ def test_gate_up_silu_layout_and_tolerance():
     # plausible mistakes fail: halves swapped, SiLU on the wrong half, SiLU left out
     for wrong in (oracle.silu(up) * gate, gate * up, oracle.silu(gate) * gate):
         assert np.any(np.abs(wrong - h) > allowed)
+
+
+# ---------------------------------------------------------------- FP8-E4M3 weights (W8A16)
+
+
+@pytest.mark.parametrize("g_bits", [0x3B124925, 0x3F800000, 0x3DCCCCCD, 0x0DA24260])
+def test_dequant_fp8_every_code(g_bits):
+    # every finite E4M3 byte times the fp32 scale, against exact rationals
+    g = float(np.array([g_bits], dtype=np.uint32).view(np.float32)[0])
+    finite = [b for b in range(256) if e4m3_value(b) != "nan"]
+    codes = np.array(finite, dtype=np.uint8)[None, :]
+    w = oracle.dequant_fp8_e4m3(codes, g)
+    gv = fp32_value(g_bits)
+    for i, b in enumerate(finite):
+        prod = e4m3_value(b) * gv
+        got = int(w[0, i])
+        if prod == 0:
+            assert got & 0x7FFF == 0 and (got >> 15) == (b >> 7), hex(b)   # signed zeros kept
+        else:
+            assert got == bf16_bits_of(prod), (hex(b), hex(got))
+
+
+def test_dequant_fp8_rejects_nan_and_is_elementwise():
+    with pytest.raises(ValueError):
+        oracle.dequant_fp8_e4m3(np.array([[0x7F]], np.uint8), 1.0)
+    with pytest.raises(ValueError):
+        oracle.dequant_fp8_e4m3(np.array([[0xFF]], np.uint8), 1.0)
+    # no grouping: permuting the codes permutes the weights
+    c = synth.fp8_weights(5, 3, 128)
+    perm = np.random.default_rng(0).permutation(128)
+    g = synth.FP8_GLOBAL_SCALE
+    assert np.array_equal(oracle.dequant_fp8_e4m3(c[:, perm], g), oracle.dequant_fp8_e4m3(c, g)[:, perm])
+
+
+def test_fp8_gemm_brute_force_exact():
+    p = synth.problem("fp8", 15, 2, 3, 128)
+    w = oracle.dequant_fp8_e4m3(p["codes"], p["g"])
+    y = oracle.gemm_ref(p["x"], w)
+    bound = oracle.abs_bound(p["x"], w)
+    ex = _exact_y(p["x"], w)
+    for m in range(2):
+        for n in range(3):
+            assert abs(Fraction(y[m, n]) - ex[m][n]) <= Fraction(128) * pow2(-52) * Fraction(bound[m, n])
+
+
+def test_fp8_draws_follow_the_recipe():
+    c = synth.fp8_weights(7, 64, 1024)
+    v = formats.e4m3_to_f64(c)
+    assert np.all(np.isfinite(v)) and np.abs(v).max() <= 448
+    z = v / 64.0                                   # back to the N(0, 1) scale, up to rounding
+    assert abs(z.mean()) < 0.02 and abs(z.std() - 1.0) < 0.03
+    # the sign comes from the draw: about half negative
+    assert 0.45 < np.mean(c >= 0x80) < 0.55
