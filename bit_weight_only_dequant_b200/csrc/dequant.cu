@@ -10,7 +10,7 @@
 //   odd, 16 spare bits) followed by fp32 -> bf16 to nearest even gives the
 //   correctly rounded BF16 value, subnormal range included.
 // FP8-E4M3 (weight-only FP8 of the attention linears, guide "Qwen3.8-27B on
-//   DGX Spark (GB10)", section "What Spark-native means"): W = RNE_bf16(e4m3
+//   DGX Spark (GB10)", section "The right stack for Spark"): W = RNE_bf16(e4m3
 //   * g) with one fp32 g per tensor, rounded the same way.
 #include "common.cuh"
 #include "kernels.h"

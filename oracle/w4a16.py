@@ -94,7 +94,7 @@ def dequant_fp8_e4m3(codes: np.ndarray, g: float) -> np.ndarray:
 
     FP8 weight-only variant (W8A16) of the attention linears, which the NVFP4
     checkpoint keeps in FP8 (guide "Qwen3.8-27B on DGX Spark (GB10)", section
-    "What Spark-native means").  Reading: E4M3 bytes with one fp32 scale per
+    "The right stack for Spark").  Reading: E4M3 bytes with one fp32 scale per
     tensor.  e4m3 (4 significant bits) * fp32 (24) is exact in binary64, so the
     product is rounded once onto BF16.  w8: uint8 [N][K] (NaN bytes rejected).
     """
