@@ -212,6 +212,26 @@ def cpu_oracle_step(rows_per_shape: int):
     return total, t_work
 
 
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of a list of floats over all ranks; every rank gets it.
+
+    Multi-GPU runs are replicas: each rank times its own copy of the workload
+    and the job's time is the slowest rank's."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_gbps(world, bytes_per_step, steps, seconds):
+    """Aggregate throughput of `world` replicas that each moved `bytes_per_step`
+    for `steps` steps within `seconds` (the slowest rank's time)."""
+    return world * bytes_per_step * steps / seconds / 1e9
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -492,12 +512,9 @@ def run_native(args, rank, world, local_rank):
     sampler.stop()
     ms_total = start.elapsed_time(end)
     W.check(W.w4a16_device_status(stream.cuda_stream), "device status")
-    if world > 1:
-        tt = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks([ms_total], world, "cuda")[0]
     ms_per_step = ms_total / args.steps
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbps(world, step_bytes, args.steps, ms_total * 1e-3)
     clocks = sampler.summary(t_soak, t_end)
     del graph
 
@@ -545,11 +562,8 @@ def run_native(args, rank, world, local_rank):
     for i in range(args.steps):
         e2e_step(i)
     e2e_s = time.perf_counter() - t0
-    if world > 1:
-        tt = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt.item())
-    e2e = {"value": round(world * step_bytes * args.steps / e2e_s / 1e9, 1), "unit": UNIT,
+    e2e_s = max_over_ranks([e2e_s], world, "cuda")[0]
+    e2e = {"value": round(whole_job_gbps(world, step_bytes, args.steps, e2e_s), 1), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": round(e2e_s / args.steps * 1e3, 4),
            "how": "pinned host x of the step -> device (one copy), the four w4a16_gemm calls via "
