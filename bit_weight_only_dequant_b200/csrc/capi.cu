@@ -137,7 +137,7 @@ int check_fmt_shape(int fmt, int N, int K) {
 // Row-count dispatch: the weight-streaming GEMV while the activations are a
 // thin n8 operand, the tcgen05 path once the tensor cores carry real work.
 // The crossovers come from back-to-back timings of both paths on the decode
-// shapes (B200), the same for both formats: the GEMV wins up to M = 8
+// shapes (B200), the same for int4 and NVFP4 (FP8 follows them): the GEMV wins up to M = 8
 // everywhere and at M = 9..16 for the widest layer (N >= 16384: enough
 // 16-row bands per SM); the tensor-core path wins for the other layers at
 // M >= 9 and everywhere at M > 16.

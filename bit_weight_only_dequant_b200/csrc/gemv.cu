@@ -32,11 +32,16 @@
 //    mma.sync m16n8k16 (16 output columns x 16 k) with exact FP16 arithmetic:
 //    int4: 1 shift, 4 LOP3 that drop each nibble into the mantissa of FP16
 //    1024.0, then 4 subtractions / fused multiply-adds that leave q; NVFP4:
-//    4 hardware e2m1 -> f16 conversions.  The activations are the n8 side:
+//    4 hardware e2m1 -> f16 conversions; FP8-E4M3 (two words per 16 k): 4
+//    hardware e4m3 -> f16 conversions.  The activations are the n8 side:
 //    one MMA serves 8 rows.  Group scales multiply the fp32 MMA results
-//    (int4: once per 128-group, NVFP4: once per 16-group).
+//    (int4: once per 128-group, NVFP4: once per 16-group); the per-tensor
+//    scale of NVFP4 and FP8 is applied in the epilogue.
 //  * Split-K partials across CTAs go to a fp32 workspace; the last CTA to
 //    finish a band (arrival counter) adds them in split order.
+//  * Fused gate/up layer (FUSE): each ring stage also holds the up band's
+//    group, a second accumulator set takes it, and the epilogue writes
+//    SiLU(gate) * up.
 #include "common.cuh"
 #include "kernels.h"
 

@@ -79,7 +79,7 @@ extern "C" {
 
 /*
  * Shape rules: 1 <= M <= 8192; N >= 1 (any value; packed buffers are padded
- * to a multiple of 16 rows); K >= 128 and K a multiple of 128 (both formats).
+ * to a multiple of 16 rows); K >= 128 and K a multiple of 128 (every format).
  * The tensor-core path splits M > 128 into ceil(M / 128) chunks of equal row
  * counts inside one launch (beyond M = 128 the tensor cores, not HBM, set the
  * time).
