@@ -79,11 +79,13 @@ def load_traffic():
 
 
 def kernel_source_hash():
+    """Hash of the sources that define the GEMV kernel (the kernel whose DRAM
+    traffic profiles/traffic.json records): its file and the headers it uses."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_weight_only_dequant_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
+        if name in ("gemv.cu", "common.cuh", "layout.h", "kernels.h"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode())
                 h.update(f.read())
