@@ -307,6 +307,31 @@ int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* pac
                        global_scale, y_bf16, stream);
 }
 
+int w4a16_selftest_wait_timeout(void* stream) {
+  DeviceState* d = nullptr;
+  int r = device_state(&d);
+  if (r != W4A16_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return W4A16_ERR_CUDA;
+  unsigned h = 0;
+  if (cudaMemcpy(&h, d->err, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return W4A16_ERR_CUDA;
+  if (h) return W4A16_ERR_TIMEOUT;   // an earlier timeout is still unreported
+  int* out = nullptr;
+  if (cudaMalloc(&out, 2 * sizeof(int)) != cudaSuccess) return W4A16_ERR_NOMEM;
+  int res[2] = {0, 0};
+  cudaError_t e = cudaMemset(out, 0, 2 * sizeof(int));
+  if (e == cudaSuccess) e = w4::launch_wait_timeout_selftest(d->err, out, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(res, out, sizeof(res), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(&h, d->err, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  cudaFree(out);
+  if (e != cudaSuccess) return W4A16_ERR_CUDA;
+  if (cudaMemset(d->err, 0, sizeof(unsigned)) != cudaSuccess) return W4A16_ERR_CUDA;
+  // as designed: both warps gave up and exactly the timeout bit was recorded
+  return (res[0] == 1 && res[1] == 1 && h == w4::kErrTimeout) ? W4A16_OK : W4A16_ERR_TIMEOUT;
+}
+
 int w4a16_device_status(void* stream) {
   DeviceState* d = nullptr;
   int r = device_state(&d);

@@ -62,6 +62,8 @@ size_t tc_workspace_floats(const TcPlan& p, int M, int N);
 size_t tc_counters(const TcPlan& p, int N);
 size_t tc_x_f16_bytes(int fmt, int M, int K);   // NVFP4: FP16 copy of x + row multipliers
 cudaError_t launch_tc(const TcPlan& p, const GemmArgs& a, void* xf16_scratch, cudaStream_t st);
+// Diagnostics: a bounded mbarrier wait that is made to run out (see capi.cu).
+cudaError_t launch_wait_timeout_selftest(unsigned* err, int* out, cudaStream_t st);
 
 // ---------------------------------------------------------------- dequant export / packer
 

@@ -799,6 +799,24 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Diagnostics: two warps wait, through the same bounded waits the kernel
+// above uses, on an mbarrier that nothing arrives at.  The first to exhaust
+// its bound records the timeout in the device error word and raises the
+// CTA's abort flag; the other sees the flag and gives up without waiting out
+// its own bound.  out[w] = 1 if warp w's wait returned false.
+__global__ void __launch_bounds__(64) wait_timeout_selftest_kernel(unsigned* err, int* out) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = warp_wait(&bar, 0, &abort_flag, err);
+  if ((threadIdx.x & 31) == 0) out[threadIdx.x >> 5] = ok ? 0 : 1;
+}
+
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -985,6 +1003,11 @@ cudaError_t launch_tc(const TcPlan& pl, const GemmArgs& a, void* xf16_scratch, c
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return a.fmt == 1 ? launch_fmt<1>(pl, a, xh, rm, st) : launch_fmt<kFmtFp8>(pl, a, xh, rm, st);
+}
+
+cudaError_t launch_wait_timeout_selftest(unsigned* err, int* out, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 64, 0, st>>>(err, out);
+  return cudaGetLastError();
 }
 
 }  // namespace w4

@@ -45,6 +45,7 @@ _SIGS = {
     "w4a16_gemm_gate_up_silu_ex": (_i, [_i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_device_status": (_i, [_vp]),
+    "w4a16_selftest_wait_timeout": (_i, [_vp]),
     "w4a16_status_string": (ctypes.c_char_p, [_i]),
     "w4a16_version": (_i, []),
 }
@@ -164,6 +165,10 @@ def w4a16_gemm_path(fmt, M, N, K):
 
 def w4a16_device_status(stream=None):
     return lib().w4a16_device_status(_stream(stream))
+
+
+def w4a16_selftest_wait_timeout(stream=None):
+    return lib().w4a16_selftest_wait_timeout(_stream(stream))
 
 
 def w4a16_version():

@@ -209,6 +209,20 @@ int w4a16_gemm_path(int fmt, int M, int N, int K);
 int w4a16_device_status(void* stream);
 
 /* Human-readable name of a status code (static string). */
+/*
+ * Diagnostics of the kernels' failure path, without a fault: launches a tiny
+ * kernel whose two warps wait, through the library's own bounded mbarrier
+ * waits, on a barrier that nothing arrives at.  After the bound (about two
+ * seconds of SM clock) the first warp records W4A16_ERR_TIMEOUT in the device
+ * error word and raises its CTA's abort flag, the second gives up on seeing
+ * the flag, and the kernel exits normally.  Synchronises `stream`, then
+ * checks and clears the error word.  Returns W4A16_OK when all of that
+ * happened as designed, W4A16_ERR_TIMEOUT when it did not (or when an
+ * earlier timeout was still unreported), W4A16_ERR_CUDA / W4A16_ERR_NOMEM /
+ * W4A16_ERR_DEVICE on failures of the call itself.
+ */
+int w4a16_selftest_wait_timeout(void* stream);
+
 const char* w4a16_status_string(int status);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

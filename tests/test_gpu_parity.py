@@ -442,6 +442,17 @@ def test_golden_examples_on_gpu():
     assert list(y) == d["expected"]["y"]
 
 
+def test_bounded_wait_runs_out_reports_a_timeout_and_leaves_the_context_usable():
+    # a wait on an mbarrier that nothing arrives at gives up after its bound
+    # (about two seconds), records W4A16_ERR_TIMEOUT and the kernel exits
+    assert W.w4a16_selftest_wait_timeout() == W.OK
+    assert W.w4a16_device_status() == W.OK          # the word was read and cleared
+    p = synth.problem("int4", 11, 3, 64, 256)      # the context still computes correctly
+    codes, scales, x = to_device_problem(p)
+    y, _ = run_gemm("int4", codes, scales, x, 64)
+    assert_parity(y, p["x"], oracle_weights(p), "after the timeout self-test")
+
+
 def test_device_status_is_clean():
     assert W.w4a16_device_status() == W.OK
 
