@@ -224,6 +224,20 @@ def test_gemm_parity_fp8_full_shapes_sampled(name, M):
     t.cuda.empty_cache()
 
 
+TC_EDGES = [  # fmt, M, N, K: ragged N against the 256-row tile, the smallest K, chunk edges
+    ("int4", 9, 1, 128), ("int4", 64, 17, 128), ("int4", 129, 255, 256), ("int4", 17, 257, 384),
+    ("nvfp4", 9, 1, 128), ("nvfp4", 130, 257, 256), ("fp8", 64, 17, 128), ("fp8", 257, 255, 384),
+]
+
+
+@pytest.mark.parametrize("fmt,M,N,K", TC_EDGES)
+def test_tensor_core_edges(fmt, M, N, K):
+    p = synth.problem(fmt, 600 + M + N, M, N, K)
+    codes, scales, x = to_device_problem(p)
+    y, _ = run_gemm(fmt, codes, scales, x, N, g=p["g"], path=W.PATH_TC)
+    assert_parity(y, p["x"], oracle_weights(p), f"TC {fmt} M={M} N={N} K={K}")
+
+
 # ---------------------------------------------------------------- GEMM parity at the full shapes
 
 

@@ -32,6 +32,8 @@ def _torch():
 def _weights(p):
     if p["fmt"] == "int4":
         return oracle.dequant_int4_g128(p["codes"], p["scales"])
+    if p["fmt"] == "fp8":
+        return oracle.dequant_fp8_e4m3(p["codes"], p["g"])
     return oracle.dequant_nvfp4(p["codes"], p["scales"], p["g"])
 
 
@@ -40,6 +42,8 @@ def _weights(p):
     ("int4", 1, 17408, 5120, 3),
     ("nvfp4", 3, 1000, 1024, 51),
     ("int4", 16, 400, 3072, 90),
+    ("fp8", 4, 1000, 2048, 91),
+    ("fp8", 2, 512, 17408, 92),    # FP8 with a long K: split-K through the scratch
 ])
 def test_noalloc_matches_gemm_on_consecutive_calls(fmt, M, N, K, seed):
     t = _torch()
