@@ -488,8 +488,14 @@ def run_native(args, rank, world, local_rank):
                 fn(i)
     props = torch.cuda.get_device_properties(local_rank)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
-    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-    sampler = ClockSampler(gpu_id, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv"))
+    # the raw clock samples go to a CSV only when W4A16_CLOCKS_DIR names a folder;
+    # their summary is always part of the JSON line
+    clocks_dir = os.environ.get("W4A16_CLOCKS_DIR")
+    clocks_csv = None
+    if clocks_dir:
+        os.makedirs(clocks_dir, exist_ok=True)
+        clocks_csv = os.path.join(clocks_dir, f"clocks_rank{rank}.csv")
+    sampler = ClockSampler(gpu_id, clocks_csv)
     sampler.start()
     time.sleep(0.3)
     t_soak = time.time()
