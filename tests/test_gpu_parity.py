@@ -419,14 +419,19 @@ def test_output_guard_bands_and_full_coverage():
 
 
 def test_repeated_calls_are_bit_identical():
+    # fixed reduction orders everywhere (split-K partials are added in split
+    # order on both paths), so repeated calls agree bit for bit
     t = torch()
-    for fmt, M, N, K in (("int4", 8, 5120, 17408), ("int4", 1, 17408, 5120), ("nvfp4", 9, 1024, 6144)):
+    for fmt, M, N, K in (("int4", 8, 5120, 17408), ("int4", 1, 17408, 5120), ("nvfp4", 9, 1024, 6144),
+                         ("int4", 64, 5120, 6144), ("int4", 200, 2048, 5120), ("fp8", 33, 1024, 17408)):
         p = synth.device_problem(fmt, 80, M, N, K)
         pw, ps = W.pack_on_device(fmt, N, K, p["codes"], p["scales"])
         g = gscale_tensor(p["g"])
         xb = p["x"].view(t.bfloat16)
         ys = [bf16_bits(W.gemm(fmt, xb, pw, ps, N, global_scale=g)) for _ in range(3)]
         assert all(np.array_equal(ys[0], yy) for yy in ys[1:]), (fmt, M, N, K)
+        hs = [bf16_bits(W.gate_up_silu(fmt, xb, pw, ps, N // 2, global_scale=g)) for _ in range(2)]
+        assert np.array_equal(hs[0], hs[1]), (fmt, M, N, K, "fused")
 
 
 def test_golden_examples_on_gpu():
