@@ -618,8 +618,9 @@ def run_native(args, rank, world, local_rank):
                                  f"({copies * step_wbytes / 1e6:.0f} MB per cycle, L2 126 MB)",
                            "timing": "CUDA graph of the K steps back to back, CUDA events on "
                                      "the launching stream around the replay, max over ranks; "
-                                     "per-kernel durations from a second graph with an event "
-                                     "pair around every launch",
+                                     "the roofline's launch duration is that replay over the "
+                                     "launches it holds; per-shape durations from each shape "
+                                     "alone, back to back in its own graph, one event pair",
                            "replicas": world},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
                 "gpu_launches": len(launches) * args.steps,
