@@ -9,7 +9,10 @@ M = 1 (int4 GPTQ g128): QKV 5120->8192, O 6144->5120, gate/up 5120->34816,
 down 17408->5120, run back to back on one stream.  ``value`` is algorithmic
 bytes (packed weights + scales + activations + outputs) per second over the
 timed steps, aggregated over all GPUs.  The other configurations (every row
-count, NVFP4, the 64-layer sweep) are reported in ``sweep`` / ``whole_stack``.
+count, NVFP4, the 64-layer sweep) and the widened rows (M up to 2048, FP8
+weights, the fused gate/up layer) are reported in ``sweep``, ``gate_up_silu``
+and ``whole_stack``.  ``--case fmt,M,N,K[,path]`` launches one GEMM a few
+times for a profiler.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 Multi-GPU: launched by torchrun, one process per GPU; each GPU runs its own
