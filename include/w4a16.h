@@ -31,16 +31,19 @@
  *    cudaStream_t passed as void*, NULL = legacy default stream).  The library
  *    keeps no pointer after a call returns; buffers must stay alive until the
  *    stream has executed the work.
- *  - The caller owns every buffer passed in.  The GEMM keeps a small
- *    library-owned fp32 workspace per (device, stream) for split-K partial
- *    sums; it is allocated on the first call that needs it on that stream
- *    (make that first call before capturing the stream into a CUDA graph).
+ *  - The caller owns every buffer passed in.  The GEMM keeps a
+ *    library-owned workspace per (device, stream): fp32 split-K partial sums
+ *    and, on the tensor-core path for NVFP4 and FP8, an FP16 copy of x.  It is
+ *    allocated (stream-ordered) on the first call that needs it on that
+ *    stream and grown when a larger problem needs more; make a call of the
+ *    largest shape before capturing the stream into a CUDA graph.
  *  - Accuracy: per element |y - y_ref| <= 2^-7 * sum_k |W_deq[n][k] x[m][k]|
  *    + 1e-3 against the fp64 dequantise-then-matmul, and w4a16_dequant is
- *    bit-exact.  The NVFP4 path rescales each activation row slice by a power
- *    of two into FP16 for the tensor cores: elements more than 2^29 below their
- *    row slice's largest magnitude lose low bits (absolute error at most
- *    2^-40 of that largest magnitude per element).
+ *    bit-exact.  The FP16 tensor-core operands (the GEMV in every format, the
+ *    tcgen05 path for NVFP4 and FP8) take each activation row (slice) scaled
+ *    by a power of two into FP16: elements more than 2^29 below their row
+ *    slice's largest magnitude lose low bits (absolute error at most 2^-40 of
+ *    that largest magnitude per element).
  */
 #ifndef W4A16_H
 #define W4A16_H
