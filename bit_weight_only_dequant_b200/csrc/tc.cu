@@ -364,6 +364,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- activations (lane 0)
+    // launched with programmatic dependent launch: x (and its FP16 copy) may
+    // come from the previous kernel on the stream
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     uint32_t it = 0;
     bool ok = true;
     if (lane == 0) {
@@ -502,6 +505,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
 #pragma unroll
     for (int k = 0; k < kWRing; ++k) copy_next();
+    // the first weight copies are in flight; everything after (y, the split-K
+    // partials, the row multipliers) may depend on the previous kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     uint32_t it = 0, unit_i = 0;
     bool ok = true;
@@ -771,6 +777,9 @@ __global__ void __launch_bounds__(256)
     tc_splitk_reduce(const float* __restrict__ ws, int S, int M, int cols, int Npad,
                      const float* __restrict__ row_mul, const float* __restrict__ g,
                      __nv_bfloat16* __restrict__ y) {
+  // a following GEMM may start streaming its weights now (it waits for this
+  // grid before it touches anything this grid reads or writes)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int m = blockIdx.y;
   const int n0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
@@ -883,8 +892,22 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
     if (e != cudaSuccess) return e;
     smem_set[dev] = pl.smem;
   }
-  tc_kernel<FMT, MPAD><<<pl.grid, kTcThreads, pl.smem, st>>>(map, p);
-  cudaError_t e = cudaGetLastError();
+  // int4: programmatic dependent launch, so on each SM freed by the previous
+  // kernel the CTA starts streaming weights before that kernel has finished;
+  // the warps that read x or write results wait for it (griddepcontrol.wait).
+  // Measured 3-8 % faster back to back.  NVFP4 and FP8 follow their own FP16
+  // rescale kernel and keep an ordinary launch (no gain measured there).
+  cudaLaunchConfig_t kcfg = {};
+  kcfg.gridDim = dim3((unsigned)pl.grid, 1, 1);
+  kcfg.blockDim = dim3(kTcThreads, 1, 1);
+  kcfg.dynamicSmemBytes = (size_t)pl.smem;
+  kcfg.stream = st;
+  cudaLaunchAttribute kattr[1];
+  kattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  kattr[0].val.programmaticStreamSerializationAllowed = 1;
+  kcfg.attrs = kattr;
+  kcfg.numAttrs = FMT == 0 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&kcfg, tc_kernel<FMT, MPAD>, map, p);
   if (e != cudaSuccess || pl.S == 1) return e;
 
   const int cols = a.fuse ? a.N / 2 : a.N;
