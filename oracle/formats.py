@@ -78,3 +78,47 @@ def f64_to_bf16_rne(v: np.ndarray) -> np.ndarray:
     zero = r == 0
     bits = np.where(zero, np.where(np.signbit(v), np.uint16(0x8000), np.uint16(0)), bits)
     return bits.astype(np.uint16)
+
+
+def f64_to_e4m3_rne(v: np.ndarray) -> np.ndarray:
+    """Round non-negative float64 values to OCP FP8-E4M3 bytes, nearest, ties to even.
+
+    Saturates at 448 (0x7E), the largest finite value; never produces the NaN
+    pattern.  Normal range: 4 significant bits; subnormals (below 2**-6):
+    quantum 2**-9.  Used for block scales, which are non-negative.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    if np.any(v < 0) or np.any(np.isnan(v)):
+        raise ValueError("E4M3 block scales are rounded from non-negative values")
+    m, e = np.frexp(v)
+    r = np.ldexp(np.rint(np.ldexp(m, 4)), e - 4)
+    r = np.where(v < 2.0 ** -6, np.ldexp(np.rint(np.ldexp(v, 9)), -9), r)
+    r = np.minimum(r, 448.0)
+    out = np.zeros(v.shape, dtype=np.uint8)
+    sub = (r > 0) & (r < 2.0 ** -6)
+    out[sub] = np.ldexp(r[sub], 9).astype(np.uint8)
+    nrm = r >= 2.0 ** -6
+    mm, ee = np.frexp(r[nrm])
+    out[nrm] = (((ee - 1 + 7).astype(np.int64) << 3) | (np.ldexp(mm, 4) - 8).astype(np.int64)).astype(np.uint8)
+    return out
+
+
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def f64_to_e2m1_rne(v: np.ndarray) -> np.ndarray:
+    """Round float64 values to FP4-E2M1 codes, nearest, ties to the even code.
+
+    Magnitudes at or above 6 saturate to 6 (code 7); the sign goes to bit 3
+    (negative zero included).  "Even" is the code whose mantissa bit is 0.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    grid = np.array(E2M1_MAGNITUDES)
+    lo = np.clip(np.searchsorted(grid, a, side="right") - 1, 0, 7)
+    hi = np.minimum(lo + 1, 7)
+    d_lo = a - grid[lo]
+    d_hi = grid[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0) & (hi != lo))
+    mag = np.where(a >= 6.0, 7, np.where(pick_hi, hi, lo))
+    return (mag | np.where(np.signbit(v), 8, 0)).astype(np.uint8)

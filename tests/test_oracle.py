@@ -483,3 +483,87 @@ def test_fp8_draws_follow_the_recipe():
     assert abs(z.mean()) < 0.02 and abs(z.std() - 1.0) < 0.03
     # the sign comes from the draw: about half negative
     assert 0.45 < np.mean(c >= 0x80) < 0.55
+
+
+# ---------------------------------------------------------------- W4A4 NVFP4 groundwork (activation quantiser)
+
+
+def test_e2m1_rounding_table():
+    # the E2M1 grid 0, 0.5, 1, 1.5, 2, 3, 4, 6; ties go to the code with mantissa bit 0
+    cases = [(0.0, 0), (0.2, 0), (0.25, 0), (0.3, 1), (0.75, 2), (1.25, 2), (1.3, 3), (1.75, 4),
+             (2.5, 4), (2.6, 5), (3.5, 6), (5.0, 6), (5.1, 7), (6.0, 7), (7.5, 7), (1e30, 7)]
+    v = np.array([c[0] for c in cases])
+    assert list(formats.f64_to_e2m1_rne(v)) == [c[1] for c in cases]
+    assert list(formats.f64_to_e2m1_rne(-v)) == [c[1] | 8 for c in cases]       # sign bit, -0 too
+    # every code decodes back to itself
+    codes = np.arange(16, dtype=np.uint8)
+    back = formats.f64_to_e2m1_rne(formats.e2m1_to_f64(codes))
+    assert np.array_equal(back, codes)
+
+
+def test_e4m3_encoder_round_trip_ties_and_saturation():
+    finite = np.array([b for b in range(0x7F)], dtype=np.uint8)           # non-negative, no NaN
+    vals = formats.e4m3_to_f64(finite)
+    assert np.array_equal(formats.f64_to_e4m3_rne(vals), finite)
+    # midpoints between neighbours: ties to the even code (mantissa LSB 0)
+    mids = (vals[:-1] + vals[1:]) / 2
+    want = np.where(finite[:-1] % 2 == 0, finite[:-1], finite[1:])
+    assert np.array_equal(formats.f64_to_e4m3_rne(mids), want)
+    assert formats.f64_to_e4m3_rne(np.array([449.0, 1e9]))[0] == 0x7E           # saturates at 448
+    with pytest.raises(ValueError):
+        formats.f64_to_e4m3_rne(np.array([-1.0]))
+
+
+def test_w4a4_quantiser_reproduces_representable_blocks():
+    # rows built as e2m1 * e4m3 * g_x with the block's largest magnitude 6:
+    # the quantiser must return exactly those codes and scales
+    rng = np.random.default_rng(5)
+    g = 2.0 ** -9                  # a power of two keeps every product exact in BF16
+    M, K = 3, 64
+    codes = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    codes[:, ::16] = 7                                                     # each block reaches +6
+    s8 = rng.integers(0x20, 0x60, size=(M, K // 16)).astype(np.uint8)
+    x = formats.e2m1_to_f64(codes) * np.repeat(formats.e4m3_to_f64(s8), 16, axis=1) * g
+    x_bits = formats.f64_to_bf16_rne(x)
+    assert np.array_equal(formats.bf16_to_f64(x_bits), x)                  # exactly representable
+    q, s = oracle.w4a4.quantize_activations(x_bits, g)
+    assert np.array_equal(s, s8)
+    zero = formats.e2m1_to_f64(codes) == 0
+    assert np.array_equal(q[~zero], codes[~zero])                           # +-0 may differ in sign only
+
+
+def test_w4a4_quantiser_zero_blocks_scale_and_error_bound():
+    p = synth.problem("int4", 41, 4, 1, 256)
+    x_bits = p["x"].copy()
+    x_bits[1, 32:48] = 0                                                    # one all-zero block
+    g = oracle.w4a4.activation_global_scale(x_bits)
+    q, s = oracle.w4a4.quantize_activations(x_bits, g)
+    assert s[1, 2] == 0 and np.all(formats.e2m1_to_f64(q[1, 32:48]) == 0)
+    x = formats.bf16_to_f64(x_bits)
+    xh = oracle.w4a4.dequant_activations(q, s, g)
+    amax = np.repeat(np.abs(x).reshape(4, 16, 16).max(axis=2), 16, axis=1)
+    assert np.all(np.abs(xh - x) <= 0.25 * amax + 1e-30)                   # E2M1 spacing + scale rounding
+    # the block's largest element maps to the top of the grid (|code| 6, or 4 after a scale round-up)
+    top = np.abs(formats.e2m1_to_f64(q)).reshape(4, 16, 16).max(axis=2)
+    assert np.all(np.isin(top[s > 0], [4.0, 6.0]))
+    # the tensor's largest magnitude sets g_x: its block scale is 448 (or just below)
+    assert formats.e4m3_to_f64(s).max() >= 416
+
+
+def test_w4a4_gemm_brute_force_exact():
+    from exact import e2m1_value, e4m3_value, fp32_value
+    M, N, K = 2, 3, 32
+    px = synth.problem("int4", 42, M, 1, K)
+    g_x = oracle.w4a4.activation_global_scale(px["x"])
+    xq, xs = oracle.w4a4.quantize_activations(px["x"], g_x)
+    pw = synth.problem("nvfp4", 43, 1, N, K)
+    y = oracle.w4a4.gemm_w4a4_ref(xq, xs, g_x, pw["codes"], pw["scales"], pw["g"])
+    gx = fp32_value(int(np.array([g_x], np.float32).view(np.uint32)[0]))
+    gw = fp32_value(int(np.array([pw["g"]], np.float32).view(np.uint32)[0]))
+    for m in range(M):
+        for n in range(N):
+            ex = sum(e2m1_value(int(xq[m, k])) * e4m3_value(int(xs[m, k // 16])) * gx *
+                     e2m1_value(int(pw["codes"][n, k])) * e4m3_value(int(pw["scales"][n, k // 16])) * gw
+                     for k in range(K))
+            # exact block-scaled sum, then two roundings by the fp32 scales
+            assert abs(Fraction(y[m, n]) - ex) <= pow2(-51) * abs(ex)
