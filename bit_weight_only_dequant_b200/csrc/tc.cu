@@ -15,9 +15,12 @@
 //    its own bytes, as in the GEMV), turns its 32 bytes per group into 64
 //    scaled operands in registers (int4: q -> BF16 times the BF16 group scale
 //    with one rounding, exactly W_deq; NVFP4: e2m1 -> FP16 times the E4M3
-//    scale, exact) and writes them straight into a tensor-memory A slot with
+//    scale, exact; FP8: e4m3 -> FP16, exact, the per-tensor scale applied in
+//    the epilogue) and writes them straight into a tensor-memory A slot with
 //    tcgen05.st 16x256b, whose register layout matches the packed pairs.
-//    Shared memory never holds dequantised weights.
+//    Shared memory never holds dequantised weights.  Fused gate/up layer:
+//    the first 128-row half takes 8 gate bands and the second the matching
+//    up bands, so the epilogue finds gate and up of a row in one TMEM lane.
 //  * warp 16 (producer): lane 0 loads the two SWIZZLE_128B activation boxes
 //    of each group with 2-D TMA (rows past M zero-filled) into a ring.
 //  * warp 17 (MMA): tcgen05.mma kind::f16, A (weights, 128 rows) from tensor
@@ -29,8 +32,11 @@
 //    order.
 // Tensor memory: D (two 128-row halves of Mpad columns), then A slots of one
 // group (2 halves x 64 columns) in the rest of the 512 columns.  Every
-// mbarrier wait is bounded; a timeout raises the device error word, the CTA
-// drains its copies and MMAs and frees tensor memory.
+// mbarrier wait is bounded and polled by all lanes of the waiting warp; a
+// timeout raises the device error word, the CTA drains its copies and MMAs
+// and frees tensor memory.  int4 launches use programmatic dependent launch:
+// weights stream before the previous kernel has finished, x is read and
+// results are written after griddepcontrol.wait.
 //
 // M > 128 runs as chunks of at most 128 activation rows (the MMA's N); a unit
 // of work is (tile, chunk, K split), and the chunks of one tile are adjacent
