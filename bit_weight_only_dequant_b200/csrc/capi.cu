@@ -307,6 +307,28 @@ int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* pac
                        global_scale, y_bf16, stream);
 }
 
+int w4a16_plan(int path, int fmt, int M, int N, int K, int fuse, int num_sms, int* out,
+               int out_len) {
+  if (fuse != 0 && fuse != 1) return W4A16_ERR_ARG;
+  const int r = check_fmt_shape(fmt, N, K);
+  if (r != W4A16_OK) return r;
+  if (M < 1 || M > W4A16_MAX_M || num_sms < 1 || !out || out_len < 9) return W4A16_ERR_ARG;
+  if (fuse && (N % 32 != 0)) return W4A16_ERR_SHAPE;
+  if (path == W4A16_PATH_AUTO) path = choose_path(fmt, M, N, K);
+  if (path == W4A16_PATH_GEMV) {
+    if (M > W4A16_GEMV_MAX_M) return W4A16_ERR_SHAPE;
+    const w4::GemvPlan pl = w4::plan_gemv(fmt, M, N, K, num_sms, fuse);
+    const int v[9] = {pl.S, pl.kslice, pl.ctas_x, pl.mt, pl.wn, pl.wk, pl.depth, pl.ngp, pl.smem};
+    for (int i = 0; i < 9; ++i) out[i] = v[i];
+    return pl.S == 0 ? W4A16_ERR_SHAPE : W4A16_PATH_GEMV;
+  }
+  if (path != W4A16_PATH_TC) return W4A16_ERR_ARG;
+  const w4::TcPlan pl = w4::plan_tc(fmt, M, N, K, num_sms, fuse);
+  const int v[9] = {pl.chunks, pl.rows, pl.mpad, pl.S, pl.kbs, pl.units, pl.grid, pl.smem, 0};
+  for (int i = 0; i < 9; ++i) out[i] = v[i];
+  return W4A16_PATH_TC;
+}
+
 int w4a16_selftest_wait_timeout(void* stream) {
   DeviceState* d = nullptr;
   int r = device_state(&d);

@@ -46,6 +46,7 @@ _SIGS = {
     "w4a16_gemm_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_device_status": (_i, [_vp]),
     "w4a16_selftest_wait_timeout": (_i, [_vp]),
+    "w4a16_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _i]),
     "w4a16_status_string": (ctypes.c_char_p, [_i]),
     "w4a16_version": (_i, []),
 }
@@ -165,6 +166,14 @@ def w4a16_gemm_path(fmt, M, N, K):
 
 def w4a16_device_status(stream=None):
     return lib().w4a16_device_status(_stream(stream))
+
+
+def w4a16_plan(path, fmt, M, N, K, fuse=0, num_sms=148):
+    """(status or path, the nine plan fields) for a shape, computed on the host."""
+    import numpy as np
+    out = np.zeros(9, dtype=np.int32)
+    r = lib().w4a16_plan(path, fmt, M, N, K, fuse, num_sms, out.ctypes.data, 9)
+    return r, [int(v) for v in out]
 
 
 def w4a16_selftest_wait_timeout(stream=None):

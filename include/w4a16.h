@@ -213,6 +213,21 @@ int w4a16_device_status(void* stream);
 
 /* Human-readable name of a status code (static string). */
 /*
+ * Diagnostics: the launch plan the library would use, computed on the host
+ * (no device call; num_sms stands for the device's SM count).  path:
+ * W4A16_PATH_AUTO, _GEMV or _TC; fuse: 1 for w4a16_gemm_gate_up_silu with
+ * N = 2I.  out[0..8] (out_len >= 9):
+ *   GEMV: K splits, K elements per split, CTAs per split, 8-row tiles, bands
+ *         in flight per CTA, K pieces per band, ring depth, groups per piece,
+ *         dynamic shared memory bytes;
+ *   TC:   row chunks, rows per chunk, padded rows (MMA N), K splits, 64-blocks
+ *         per split, work units, CTAs, dynamic shared memory bytes, 0.
+ * Returns the path (W4A16_PATH_GEMV or W4A16_PATH_TC) or a negative status.
+ */
+int w4a16_plan(int path, int fmt, int M, int N, int K, int fuse, int num_sms, int* out,
+               int out_len);
+
+/*
  * Diagnostics of the kernels' failure path, without a fault: launches a tiny
  * kernel whose two warps wait, through the library's own bounded mbarrier
  * waits, on a barrier that nothing arrives at.  After the bound (about two

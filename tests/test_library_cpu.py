@@ -213,3 +213,55 @@ def test_dispatcher_path_table():
     assert W.w4a16_gemm_path(1, 256, 17408, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 8192, 5120, 5120) == W.PATH_TC
     assert W.w4a16_gemm_path(0, 8193, 5120, 5120) == W.ERR_SHAPE
+
+
+DECODE = [(5120, 8192), (6144, 5120), (5120, 34816), (17408, 5120), (5120, 17408), (128, 16),
+          (384, 1000), (17408, 24), (12288, 48)]
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("fuse", [0, 1])
+def test_gemv_plans_are_consistent(fmt, fuse):
+    # every GEMV plan the planner hands out covers K exactly with whole
+    # 128-groups, uses an instantiated ring depth and fits in shared memory
+    for K, N in DECODE:
+        if fuse and N % 32:
+            continue
+        for M in (1, 2, 5, 8, 9, 12, 16):
+            r, (S, kslice, ctas, mt, wn, wk, depth, ngp, smem) = W.w4a16_plan(W.PATH_GEMV, fmt, M, N, K,
+                                                                              fuse)
+            assert r == W.PATH_GEMV, (fmt, fuse, M, N, K, r)
+            assert S >= 1 and kslice % 128 == 0 and S * kslice >= K > (S - 1) * kslice
+            assert mt == (1 if M <= 8 else 2)
+            assert wn * wk == 16 and wn & (wn - 1) == 0
+            assert depth in ((2, 3, 4) if (fuse or fmt == 2) else (2, 3, 4, 5, 6, 8))
+            assert ngp % depth == 0 and ngp * wk * 128 >= min(kslice, K)
+            bands = (N // 2 if fuse else N + 15) // 16
+            assert 1 <= ctas <= bands and ctas * S <= 148
+            assert 0 < smem <= 227 * 1024
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("fuse", [0, 1])
+def test_tensor_core_plans_are_consistent(fmt, fuse):
+    for K, N in DECODE:
+        if fuse and N % 32:
+            continue
+        for M in (1, 9, 16, 17, 64, 65, 128, 129, 200, 256, 1000, 8192):
+            r, (chunks, rows, mpad, S, kbs, units, grid, smem, _) = W.w4a16_plan(W.PATH_TC, fmt, M, N,
+                                                                                 K, fuse)
+            assert r == W.PATH_TC
+            assert chunks * rows >= M > (chunks - 1) * rows and rows <= 128
+            assert mpad % 16 == 0 and rows <= mpad <= 128 and mpad - rows < 16
+            assert S >= 1 and kbs % 2 == 0 and S * kbs * 64 >= K > (S - 1) * kbs * 64
+            tiles = (N // 2 + 127) // 128 if fuse else (N + 255) // 256
+            assert units == tiles * chunks * S
+            assert 1 <= grid <= min(units, 148)
+            assert 120 * 1024 <= smem <= 227 * 1024
+
+
+def test_plans_follow_the_dispatcher():
+    assert W.w4a16_plan(W.PATH_AUTO, 0, 1, 17408, 5120)[0] == W.PATH_GEMV
+    assert W.w4a16_plan(W.PATH_AUTO, 0, 64, 34816, 5120)[0] == W.PATH_TC
+    assert W.w4a16_plan(W.PATH_GEMV, 0, 17, 16, 128)[0] == W.ERR_SHAPE
+    assert W.w4a16_plan(W.PATH_TC, 0, 1, 24, 128, fuse=1)[0] == W.ERR_SHAPE      # 2I not a multiple of 32
