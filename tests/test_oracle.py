@@ -245,6 +245,70 @@ def test_gemm_brute_force_exact(fmt, M, N, K, seed):
             assert abs(y[m, n]) <= bound[m, n] * (1 + 1e-12)
 
 
+def _exact_abs_bound(x_bits, w_bits):
+    """sum_k |x[m][k] * W_deq[n][k]| in exact rationals, by loops over k."""
+    M, K = x_bits.shape
+    N = w_bits.shape[0]
+    xs = [[abs(bf16_value(int(b))) for b in row] for row in x_bits]
+    ws = [[abs(bf16_value(int(b))) for b in row] for row in w_bits]
+    return [[sum(xs[m][k] * ws[n][k] for k in range(K)) for n in range(N)] for m in range(M)]
+
+
+def _bound_pins(bound_fn):
+    """Checks of a tolerance-scale function against what fixes sum_k |W x|;
+    returns the names of the checks it fails."""
+    fails = []
+    # exact rationals on seeded brute-force shapes of both formats
+    for fmt, M, N, K, seed in (("int4", 2, 3, 256, 15), ("nvfp4", 3, 2, 128, 16)):
+        p = synth.problem(fmt, seed, M, N, K)
+        w = (oracle.dequant_int4_g128(p["codes"], p["scales"]) if fmt == "int4"
+             else oracle.dequant_nvfp4(p["codes"], p["scales"], p["g"]))
+        b = bound_fn(p["x"], w)
+        ex = _exact_abs_bound(p["x"], w)
+        # K non-negative exact products summed in binary64: relative error <= K * 2**-53
+        if any(abs(Fraction(b[m, n]) - ex[m][n]) > Fraction(K) * pow2(-53) * ex[m][n]
+               for m in range(M) for n in range(N)):
+            fails.append("exact")
+    # closed form: x = (1, -1, 1, -1, ...) and W_deq = 1 everywhere cancel to
+    # y = 0 while the bound counts every term: K
+    K = 256
+    x = np.tile(np.array([0x3F80, 0xBF80], np.uint16), (1, K // 2))
+    w = np.full((2, K), 0x3F80, np.uint16)
+    if not np.all(bound_fn(x, w) == K):
+        fails.append("cancelling signs")
+    # one term: |x_k| * |W_k| for a negative x and a negative weight
+    x1 = np.zeros((1, K), np.uint16)
+    x1[0, 7] = 0xC040                        # -3
+    w1 = np.zeros((1, K), np.uint16)
+    w1[0, 7] = 0xBF00                        # -0.5
+    w1[0, 8] = 0x4000                        # 2, paired with x = 0: contributes 0
+    if bound_fn(x1, w1)[0, 0] != 1.5:
+        fails.append("one term")
+    return fails
+
+
+def test_abs_bound_pinned():
+    assert _bound_pins(oracle.abs_bound) == []
+
+
+def test_abs_bound_pins_catch_planted_mistakes():
+    def abs_outside(x, w):         # |sum_k x w| instead of sum_k |x w|
+        return np.abs(oracle.gemm_ref(x, w))
+
+    def abs_of_x_only(x, w):       # forgets the weights' signs
+        return np.abs(formats.bf16_to_f64(x)) @ formats.bf16_to_f64(w).T
+
+    def abs_of_w_only(x, w):       # forgets the activations' signs
+        return formats.bf16_to_f64(x) @ np.abs(formats.bf16_to_f64(w)).T
+
+    def dropped_term(x, w):        # drops the last k
+        return np.abs(formats.bf16_to_f64(x))[:, :-1] @ np.abs(formats.bf16_to_f64(w))[:, :-1].T
+
+    for mutant in (abs_outside, abs_of_x_only, abs_of_w_only, dropped_term):
+        assert _bound_pins(mutant) != [], mutant.__name__
+    assert "cancelling signs" in _bound_pins(abs_outside)
+
+
 def _int4_case(seed=21, M=4, N=40, K=384):
     p = synth.problem("int4", seed, M, N, K)
     return p, oracle.dequant_int4_g128(p["codes"], p["scales"])
