@@ -294,3 +294,106 @@ def device_problem(fmt: str, seed: int, M: int, N: int, K: int, device="cuda"):
     x = torch.empty((M, K), dtype=torch.int16, device=device)
     device_fill(KIND_X, seed, T_X, x)
     return {"fmt": fmt, "M": M, "N": N, "K": K, "codes": codes, "scales": scales, "x": x, "g": g}
+
+
+# ---------------------------------------------------------------- edge-value problems
+#
+# Inputs built to reach the corners of the storage formats rather than the
+# checkpoint's typical values: negative, subnormal, zero and very large
+# scales; groups whose codes are all zero next to ordinary ones; activation
+# rows whose magnitudes span many binades.  Drawn from the same counter-based
+# generator (tensor ids of their own), so both sides of a parity check get the
+# same bits.
+
+T_ADV_CAT = 20     # per (n, group): which scale category
+T_ADV_BITS = 21    # per (n, group): random bits of the scale
+T_ADV_ZERO = 22    # per (n, group): all-zero-code group
+T_ADV_CODE = 23    # per (n, k): codes / weight bytes
+T_ADV_XMAG = 24    # per (m, k): activation exponents
+T_ADV_X = 25       # per (m, k): activation values
+
+FINITE_E4M3 = np.array([b for b in range(256) if (b & 0x7F) != 0x7F], dtype=np.uint8)
+
+
+def _adv_u(seed, tensor_id, shape):
+    idx = np.arange(int(np.prod(shape)), dtype=np.uint64).reshape(shape)
+    return raw64(seed, tensor_id, idx)
+
+
+def adversarial_problem(fmt: str, seed: int, M: int, N: int, K: int,
+                        regime: str = "extreme") -> dict:
+    """A problem whose weights and activations sit at the formats' edges.
+
+    regime "extreme": int4 BF16 group scales drawn from six categories per
+      (n, group) -- positive and negative normals of moderate size, subnormals
+      (either sign), +-0, large (2^60 .. 2^100) and tiny (2^-126 .. 2^-100)
+      normals; NVFP4 E4M3 block scales uniform over all 254 finite bytes (sign,
+      subnormals and zero included); FP8 weight bytes uniform over the finite
+      bytes.  One group in five has all codes equal to zero.  x ~ N(0, 1).
+    regime "wide": scales of moderate size (2^-30 .. 2^30, either sign, some
+      zero and subnormal), and activation rows whose magnitudes span up to
+      2^-24 .. 2^24 within one row: row m % 3 == 0 is N(0, 1), == 1 is
+      z * 2^u with u uniform on [-24, 24] per element, == 2 is mostly zero
+      with a few large entries.
+    The NVFP4 per-tensor scale is fp32(1/448) ("extreme") or 2^-20 ("wide");
+    FP8 uses fp32(1/448) or 2^20.
+    """
+    if regime not in ("extreme", "wide"):
+        raise ValueError(regime)
+    out = {"fmt": fmt, "M": M, "N": N, "K": K, "regime": regime}
+    zero_groups = (_adv_u(seed, T_ADV_ZERO, (N, K // INT4_GROUP)) >> np.uint64(61)) == 0  # 1 in 8
+    zero_k = np.repeat(zero_groups, INT4_GROUP, axis=1)
+    codes_raw = (_adv_u(seed, T_ADV_CODE, (N, K)) >> np.uint64(56)).astype(np.uint8)
+    if fmt == "int4":
+        q = ((codes_raw >> 4).astype(np.int16) - 8).astype(np.int8)
+        out["codes"] = np.where(zero_k, 0, q).astype(np.int8)
+        G = K // INT4_GROUP
+        cat = (_adv_u(seed, T_ADV_CAT, (N, G)) % np.uint64(6)).astype(np.int64)
+        bits = _adv_u(seed, T_ADV_BITS, (N, G))
+        sign = ((bits >> np.uint64(63)) & np.uint64(1)).astype(np.uint16) << 15
+        mant = (bits & np.uint64(0x7F)).astype(np.uint16)
+        r = ((bits >> np.uint64(8)) % np.uint64(1 << 20)).astype(np.int64)
+        if regime == "extreme":
+            e_mod = 127 - 8 + r % 12                              # 2^-8 .. 2^3
+            e_big = 127 + 60 + r % 41                             # 2^60 .. 2^100
+            e_tiny = 1 + r % 27                                   # 2^-126 .. 2^-100
+        else:
+            e_mod = 127 - 30 + r % 61                             # 2^-30 .. 2^30
+            e_big = 127 + r % 31
+            e_tiny = 127 - 30 + r % 31
+        e = np.select([cat == 0, cat == 1, cat == 2, cat == 3, cat == 4, cat == 5],
+                      [e_mod, e_mod, 0, 0, e_big, e_tiny]).astype(np.uint16)
+        m = np.where(cat == 3, 0, np.where(cat == 2, np.maximum(mant, 1), mant)).astype(np.uint16)
+        s = np.where(cat == 0, 0, sign).astype(np.uint16)         # category 0 positive
+        s = np.where(cat == 1, 0x8000, s).astype(np.uint16)        # category 1 negative
+        out["scales"] = (s | (e << 7) | m).astype(np.uint16)
+        out["g"] = None
+    elif fmt == "nvfp4":
+        c = codes_raw & np.uint8(0xF)
+        zero_code = np.where((codes_raw >> 7) == 1, 8, 0).astype(np.uint8)   # +0 or -0
+        out["codes"] = np.where(zero_k, zero_code, c).astype(np.uint8)
+        G = K // NVFP4_GROUP
+        pick = _adv_u(seed, T_ADV_BITS, (N, G)) % np.uint64(len(FINITE_E4M3))
+        sc = FINITE_E4M3[pick.astype(np.int64)]
+        out["scales"] = sc.astype(np.uint8)
+        out["g"] = float(np.float32(1.0 / 448.0)) if regime == "extreme" else 2.0 ** -20
+    elif fmt == "fp8":
+        pick = (_adv_u(seed, T_ADV_CODE, (N, K)) >> np.uint64(8)) % np.uint64(len(FINITE_E4M3))
+        w8 = FINITE_E4M3[pick.astype(np.int64)]
+        out["codes"] = np.where(zero_k, 0, w8).astype(np.uint8)
+        out["scales"] = None
+        out["g"] = float(np.float32(1.0 / 448.0)) if regime == "extreme" else 2.0 ** 20
+    else:
+        raise ValueError(fmt)
+    # activations
+    z = normals(seed, T_ADV_X, np.arange(M * K, dtype=np.uint64).reshape(M, K))
+    if regime == "extreme":
+        xv = z
+    else:
+        u = (_adv_u(seed, T_ADV_XMAG, (M, K)) >> np.uint64(11)).astype(np.float64) * 2.0 ** -53
+        rows = np.arange(M)[:, None] % 3
+        wide = z * np.exp2(np.floor(u * 49.0) - 24.0)
+        sparse = np.where(u < 0.02, z * 2.0 ** 20, 0.0)
+        xv = np.where(rows == 0, z, np.where(rows == 1, wide, sparse))
+    out["x"] = to_bf16_bits(xv)
+    return out

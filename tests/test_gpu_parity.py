@@ -532,3 +532,62 @@ def test_chained_layers_read_their_inputs_after_they_are_written(fmt, M, path, g
         y = bufs[i + 1].float().cpu().numpy().astype(np.float64)
         assert not np.isnan(y).any(), (fmt, M, i)
         assert_parity(y, x_in, wref, f"{fmt} M={M} layer {i}")
+
+
+# ---------------------------------------------------------------- edge values through the GEMMs
+# Scales that are negative, subnormal, zero, very large or very small; groups
+# whose codes are all zero; activation rows spanning up to 2^-24 .. 2^24 (see
+# synth.adversarial_problem).  Both paths, every format, element by element
+# against the oracle at the accuracy contract.
+
+EDGE_CASES = (
+    [("int4", reg, W.PATH_GEMV, M, 264, 1024) for reg in ("extreme", "wide") for M in (1, 3, 8, 16)] +
+    [("int4", reg, W.PATH_TC, M, 264, 1024) for reg in ("extreme", "wide") for M in (9, 64, 130)] +
+    [("int4", reg, path, M, 40, 17408) for reg in ("extreme", "wide")
+     for path, M in ((W.PATH_GEMV, 2), (W.PATH_TC, 17))] +
+    [("nvfp4", reg, W.PATH_GEMV, M, 208, 1280) for reg in ("extreme", "wide") for M in (1, 5, 16)] +
+    [("nvfp4", reg, W.PATH_TC, M, 208, 1280) for reg in ("extreme", "wide") for M in (9, 64)] +
+    [("nvfp4", reg, path, M, 48, 12288) for reg in ("extreme", "wide")
+     for path, M in ((W.PATH_GEMV, 3), (W.PATH_TC, 40))] +
+    [("fp8", reg, W.PATH_GEMV, M, 200, 1536) for reg in ("extreme", "wide") for M in (2, 12)] +
+    [("fp8", reg, W.PATH_TC, M, 200, 1536) for reg in ("extreme", "wide") for M in (33, 64)])
+
+
+@pytest.mark.parametrize("fmt,regime,path,M,N,K", EDGE_CASES)
+def test_gemm_parity_edge_values(fmt, regime, path, M, N, K):
+    p = synth.adversarial_problem(fmt, 700 + M + K % 97, M, N, K, regime)
+    codes, scales, x = to_device_problem(p)
+    y, _ = run_gemm(fmt, codes, scales, x, N, g=p["g"], path=path)
+    w = oracle_weights(p)
+    assert np.isfinite(oracle.gemm_ref(p["x"], w)).all()
+    assert_parity(y, p["x"], w, f"edge {fmt} {regime} path={path} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("fmt,regime,path,M,I,K", [
+    ("int4", "extreme", W.PATH_GEMV, 4, 64, 2048), ("int4", "wide", W.PATH_TC, 24, 144, 1024),
+    ("nvfp4", "extreme", W.PATH_TC, 64, 48, 1280), ("fp8", "wide", W.PATH_GEMV, 7, 96, 1536)])
+def test_gate_up_silu_parity_edge_values(fmt, regime, path, M, I, K):
+    p = synth.adversarial_problem(fmt, 750 + M, M, 2 * I, K, regime)
+    h = _run_gate_up(fmt, p, I, path)
+    _assert_gate_up_parity(h, p["x"], oracle_weights(p), f"edge gate/up {fmt} {regime} M={M}")
+
+
+# ---------------------------------------------------------------- the output projection
+# The whole-stack sweep's 5120 -> 248,320 int4 output projection (layer seed
+# 71): the largest packed weight (636 MB) and output the library addresses.
+
+
+@pytest.mark.parametrize("M,path", [(1, W.PATH_AUTO), (16, W.PATH_AUTO), (16, W.PATH_TC),
+                                    (64, W.PATH_AUTO)])
+def test_gemm_parity_output_projection_sampled(M, path):
+    K, N, seed = 5120, 248320, 71
+    t = torch()
+    p = synth.device_problem("int4", seed, M, N, K)
+    y, (pw, ps, _) = run_gemm("int4", p["codes"], p["scales"], p["x"], N, path=path)
+    del p
+    rows = np.unique(np.concatenate([[0, 15, 16, 255, 256, N - 257, N - 16, N - 1],
+                                     np.random.default_rng(M + path).integers(0, N, 48)]))
+    ph = synth.problem("int4", seed, M, N, K, rows=rows)
+    assert_parity(y[:, rows], ph["x"], oracle_weights(ph), f"output projection M={M} path={path}")
+    del pw, ps
+    t.cuda.empty_cache()

@@ -95,3 +95,25 @@ def test_nvfp4_golden_example_oracle():
     x = np.zeros((1, 16), dtype=np.uint16)
     x[0, :8] = 0x3F80
     assert list(oracle.gemm_ref(x, w)[0]) == d["expected"]["y"]
+
+
+def test_edge_value_problems_reach_the_corners():
+    # the edge-value inputs of the GPU parity tests contain what they claim
+    p = synth.adversarial_problem("int4", 1, 6, 64, 2048, "extreme")
+    s = p["scales"]
+    e = (s >> 7) & 0xFF
+    assert ((s & 0x8000) != 0).any() and ((s & 0x8000) == 0).any()        # both signs
+    assert ((e == 0) & ((s & 0x7F) != 0)).any()                            # subnormal
+    assert ((s & 0x7FFF) == 0).any()                                       # zero
+    assert (e >= 127 + 90).any() and ((e >= 1) & (e <= 27)).any()          # huge and tiny
+    q = p["codes"].reshape(64, -1, 128)
+    zero_groups = (q == 0).all(axis=2)
+    assert zero_groups.any() and (~zero_groups).any()
+    n = synth.adversarial_problem("nvfp4", 2, 3, 32, 1024, "extreme")
+    b = n["scales"]
+    assert ((b & 0x78) == 0).any() and (b & 0x80).any() and ((b & 0x7F) != 0x7F).all()
+    w = synth.adversarial_problem("int4", 3, 3, 16, 1024, "wide")
+    xv = oracle.bf16_to_f64(w["x"])
+    nz = np.abs(xv[1][xv[1] != 0])
+    assert np.log2(nz.max() / nz.min()) > 30                               # a row spans > 2^30
+    assert (xv[2] == 0).mean() > 0.9 and np.abs(xv[2]).max() > 2 ** 15
