@@ -1,5 +1,5 @@
 // Device helpers shared by the kernels: status word, bounded mbarrier waits,
-// bulk copies, bit-level unpacking and warp-level MMA wrappers (sm_100a).
+// the L2 eviction policy, bit-level unpacking and warp-level MMA wrappers (sm_100a).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -70,30 +70,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, unsigne
   return false;
 }
 
-// ------------------------------------------------------------------ bulk copy (TMA, 1-D)
+// ------------------------------------------------------------------ L2 policy
 
-// Global -> shared bulk copy completing on an mbarrier (tx bytes).  Both
-// addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Same with an L2 eviction hint: the streamed weights are read exactly once.
-__device__ __forceinline__ void bulk_g2s_evict_first(void* smem_dst, const void* gmem_src,
-                                                     uint32_t bytes, uint64_t* bar,
-                                                     uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
-      "[%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
-      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
+// The streamed weights are read exactly once: evict them from L2 first.
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -42,6 +42,8 @@
 //  * Fused gate/up layer (FUSE): each ring stage also holds the up band's
 //    group, a second accumulator set takes it, and the epilogue writes
 //    SiLU(gate) * up.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -626,20 +628,28 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
   cpa_wait<0>();  // nothing is in flight at exit
 }
 
+// Raise the dynamic shared memory limit of one kernel variant, once per
+// device (kept out of the steady state).  Two host threads may both set it the
+// first time; the attribute call is idempotent and the flag is atomic.
 template <int FMT, int MT, int D, bool FUSE>
-cudaError_t launch_d(const Params& p, const GemvPlan& pl, cudaStream_t st) {
-  // raise the dynamic shared memory limit once per device (kept out of the
-  // steady state so launches can be captured in CUDA graphs)
-  static bool smem_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
+cudaError_t prepare_d(int dev) {
+  static std::atomic<bool> smem_set[64];
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!smem_set[dev]) {
+  if (!smem_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemv_kernel<FMT, MT, D, FUSE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return e;
-    smem_set[dev] = true;
+    smem_set[dev].store(true, std::memory_order_release);
   }
+  return cudaSuccess;
+}
+
+template <int FMT, int MT, int D, bool FUSE>
+cudaError_t launch_d(const Params& p, const GemvPlan& pl, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = prepare_d<FMT, MT, D, FUSE>(dev)) != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.ctas_x, pl.S);
   cfg.blockDim = dim3(Cfg<FMT, MT, FUSE>::kWarps * 32);
@@ -721,7 +731,38 @@ int header_of(int fmt, int mt, int fuse) {
   return mt == 1 ? Cfg<0, 1>::kHeader : Cfg<0, 2>::kHeader;
 }
 
+// Every ring depth a plan can pick for one (format, row tiles, fusion).
+template <int FMT, int MT, bool FUSE>
+cudaError_t prepare_t(int dev) {
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = prepare_d<FMT, MT, 2, FUSE>(dev);
+  if (e == cudaSuccess) e = prepare_d<FMT, MT, 3, FUSE>(dev);
+  if (e == cudaSuccess) e = prepare_d<FMT, MT, 4, FUSE>(dev);
+  if constexpr (!FUSE && FMT != kFmtFp8) {
+    if (e == cudaSuccess) e = prepare_d<FMT, MT, 5, FUSE>(dev);
+    if (e == cudaSuccess) e = prepare_d<FMT, MT, 6, FUSE>(dev);
+    if (e == cudaSuccess) e = prepare_d<FMT, MT, 8, FUSE>(dev);
+  }
+  return e;
+}
+
 }  // namespace
+
+cudaError_t gemv_prepare_all(int fuse) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const cudaError_t r[6] = {
+      fuse ? prepare_t<0, 1, true>(dev) : prepare_t<0, 1, false>(dev),
+      fuse ? prepare_t<0, 2, true>(dev) : prepare_t<0, 2, false>(dev),
+      fuse ? prepare_t<1, 1, true>(dev) : prepare_t<1, 1, false>(dev),
+      fuse ? prepare_t<1, 2, true>(dev) : prepare_t<1, 2, false>(dev),
+      fuse ? prepare_t<2, 1, true>(dev) : prepare_t<2, 1, false>(dev),
+      fuse ? prepare_t<2, 2, true>(dev) : prepare_t<2, 2, false>(dev)};
+  for (cudaError_t x : r)
+    if (x != cudaSuccess) return x;
+  return cudaSuccess;
+}
 
 // Picks the K splits across CTAs (S), the warp grid (wn bands x wk pieces,
 // both powers of two) and the ring depth D.  Every warp's piece is padded to

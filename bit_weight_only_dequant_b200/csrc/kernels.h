@@ -39,6 +39,9 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms, int fuse = 0);
 size_t gemv_workspace_floats(const GemvPlan& p, int M, int N);
 size_t gemv_counters(const GemvPlan& p, int N);
 cudaError_t launch_gemv(const GemvPlan& p, const GemmArgs& a, cudaStream_t st);
+// Set the launch attributes of every GEMV kernel variant (plain or fused) on
+// the current device, so that no later launch has to.
+cudaError_t gemv_prepare_all(int fuse);
 
 // ---------------------------------------------------------------- tensor-core path (tcgen05)
 

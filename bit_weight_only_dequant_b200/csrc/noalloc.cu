@@ -1,12 +1,12 @@
 // w4a16_gemm_noalloc: the split-K GEMV for callers that cannot allocate
 // device memory.
 //
-// Who needs it: code that issues the matmul while a stream is being captured
-// into a CUDA graph (cudaMalloc is not allowed during a global-mode capture),
-// and applications that reserve all device memory up front in their own
-// allocator or pool (serving engines that hand every byte to weights and KV
-// cache) and forbid any later cudaMalloc, including the hidden one that
-// w4a16_gemm makes the first time a stream needs split-K workspace.
+// Who needs it: applications that reserve all device memory up front for
+// their own allocator or pool (serving engines that hand every byte to
+// weights and KV cache) and forbid any later cudaMalloc, including the hidden
+// one that w4a16_gemm makes the first time a stream needs split-K workspace;
+// and latency-critical code that must not call cudaMalloc in its steady state,
+// since an allocation can synchronise the device and stall every stream.
 //
 // The scratch lives in one file-scope __device__ array of kScratchBytes that
 // every GPU which loads this library keeps until the process exits.  Host code
@@ -15,8 +15,9 @@
 // current) and passed to the kernel.  Every call shares the array: calls whose
 // GPU work overlaps (two streams, or two host threads on one device) race, and
 // the array keeps whatever the last call left there, so each call clears the
-// parts that must start at zero (the status word and the split-K arrival
-// counters) with a stream-ordered memset.
+// part that must start at zero (the split-K arrival counters) with a
+// stream-ordered memset.  The GEMV has no bounded waits, so a call cannot
+// time out; the first 256 bytes of the array are reserved.
 #include <mutex>
 
 #include "../../include/w4a16.h"
@@ -26,7 +27,7 @@
 namespace {
 
 constexpr size_t kScratchBytes = 8u << 20;      // 8 MiB
-constexpr size_t kStatusBytes = 256;            // status word, padded to keep alignment
+constexpr size_t kStatusBytes = 256;            // reserved, keeps the counters aligned
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 struct NoAllocDevice {
@@ -39,8 +40,10 @@ struct NoAllocDevice {
 std::mutex g_na_mu;
 NoAllocDevice g_na_dev[64];
 
-// Once per device, with that device current: check the architecture and
-// resolve the device address of the scratch array.  Allocates nothing.
+// Once per device, with that device current: check the architecture,
+// resolve the device address of the scratch array and set the launch
+// attributes of every GEMV kernel variant this entry point can launch, so that
+// later calls (of any shape) only launch.  Allocates nothing.
 int noalloc_setup(NoAllocDevice** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
@@ -57,6 +60,7 @@ int noalloc_setup(NoAllocDevice** out) {
       if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
         return W4A16_ERR_CUDA;
       d.base = static_cast<unsigned char*>(ptr);
+      if (w4::gemv_prepare_all(0) != cudaSuccess) return W4A16_ERR_CUDA;
     }
     d.ready = true;
   }

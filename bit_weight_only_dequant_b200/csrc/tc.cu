@@ -45,6 +45,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -888,15 +890,19 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   p.chunks = pl.chunks;
   p.rows = pl.rows;
   p.units = p.tiles * pl.chunks * pl.S;
-  static int smem_set[64] = {0};
+  // the dynamic shared memory limit, raised once per device and variant (an
+  // atomic flag: host threads may race here; the attribute call is idempotent)
+  static std::atomic<int> smem_set[64];
   int dev = 0;
-  cudaGetDevice(&dev);
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (smem_set[dev] < pl.smem) {
+  if (smem_set[dev].load(std::memory_order_acquire) < pl.smem) {
     cudaError_t e =
         cudaFuncSetAttribute(tc_kernel<FMT, MPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
     if (e != cudaSuccess) return e;
-    smem_set[dev] = pl.smem;
+    int cur = smem_set[dev].load(std::memory_order_relaxed);
+    while (cur < pl.smem && !smem_set[dev].compare_exchange_weak(cur, pl.smem)) {
+    }
   }
   // int4: programmatic dependent launch, so on each SM freed by the previous
   // kernel the CTA starts streaming weights before that kernel has finished;

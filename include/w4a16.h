@@ -178,11 +178,12 @@ int w4a16_gemm_gate_up_silu_ex(int path, int fmt, int M, int I, int K, const voi
 
 /*
  * The split-K GEMV (M <= W4A16_GEMV_MAX_M) for callers that cannot allocate
- * device memory: code that issues the matmul while its stream is being
- * captured into a CUDA graph, where cudaMalloc is not allowed, and
- * applications that reserve all device memory up front in their own pool and
- * forbid later allocations.  No counterpart on the source pages: it is a
- * deployment variant of w4a16_gemm.
+ * device memory: applications that reserve all device memory up front for
+ * their own pool or allocator and forbid any later cudaMalloc (including the
+ * one w4a16_gemm makes the first time a stream needs split-K workspace), and
+ * latency-critical code that must not allocate in its steady state, because
+ * an allocation can synchronise the device.  No counterpart on the source
+ * pages: it is a deployment variant of w4a16_gemm.
  *   Same arguments, layouts and results as w4a16_gemm on the GEMV path.
  *   Scratch: a fixed 8 MiB array in device global memory owned by the library
  *   (every GPU that loads the library holds it until the process exits).  A
@@ -190,12 +191,12 @@ int w4a16_gemm_gate_up_silu_ex(int path, int fmt, int M, int I, int K, const voi
  *   W4A16_ERR_SCRATCH without launching; M > W4A16_GEMV_MAX_M returns
  *   W4A16_ERR_SHAPE.  Calls neither allocate nor free device memory.
  *   The first call on a device resolves the array's device address and sets
- *   kernel attributes; make that first call before any stream capture.
+ *   the launch attributes of every kernel variant this entry point uses; make
+ *   that first call before any stream capture.
  *   All calls share the array: calls whose GPU work overlaps (different
  *   streams, or threads sharing a device) race and must be serialised by the
- *   caller.  Each call clears, in stream order, the parts that must start at
- *   zero.  A bounded-wait timeout inside this call is recorded in the array's
- *   own status word and is not reported by w4a16_device_status.
+ *   caller.  Each call clears, in stream order, the part that must start at
+ *   zero.  The GEMV has no bounded waits, so these calls cannot time out.
  */
 int w4a16_gemm_noalloc(int fmt, int M, int N, int K, const void* x_bf16, const void* packed_w,
                        const void* packed_scales, const float* global_scale, void* y_bf16,
