@@ -200,6 +200,82 @@ def cpu_oracle_sample(seconds: float):
     return done_bytes / busy / 1e9, desc, busy
 
 
+def _oracle_worker_init():
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        pass
+
+
+def _oracle_blocks(task):
+    """One worker's share of an all-cores oracle run: ``blocks`` blocks of
+    ``rows`` output columns of one shape (inputs generated first, not timed).
+    Returns (weight+scale bytes processed, seconds of oracle work)."""
+    import oracle
+    import synth
+    fmt, M, N, K, seed, first_row, rows, blocks = task
+    x = synth.activations(seed, M, K)
+    probs = []
+    for b in range(blocks):
+        r0 = (first_row + b * rows) % N
+        probs.append(synth.problem(fmt, seed, M, N, K, rows=np.arange(r0, min(N, r0 + rows))))
+    t0 = time.perf_counter()
+    done = 0.0
+    for p in probs:
+        wd = (oracle.dequant_int4_g128(p["codes"], p["scales"]) if fmt == "int4"
+              else oracle.dequant_nvfp4(p["codes"], p["scales"], p["g"]))
+        oracle.gemm_ref(x, wd)
+        done += p["codes"].shape[0] * K * (0.5 + (2 / 128 if fmt == "int4" else 1 / 16))
+    return done, time.perf_counter() - t0
+
+
+def weight_bytes(fmt, N, K):
+    return N * K * (0.5 + (2 / 128 if fmt == "int4" else 1 / 16))
+
+
+def cpu_oracle_all_cores(rows=256, blocks=2):
+    """The oracle on every host core at once (one process per core, started
+    with spawn, one BLAS thread each), per configuration: every core takes
+    ``blocks`` blocks of ``rows`` output columns of each shape of the
+    configuration; the configuration's oracle time is extrapolated from the
+    bytes the cores processed per second (the slowest core's time).  The
+    whole-stack configuration is extrapolated from the int4 rates at
+    M = 1 / 16 / 64."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    cores = os.cpu_count() or 1
+    configs = [("decode int4 M=1", "int4", [1], [(K, N, s) for _, K, N, s in DECODE_SHAPES])]
+    configs += [(f"verify int4 M={M}", "int4", [M], [(K, N, 5) for _, K, N, _ in DECODE_SHAPES])
+                for M in (2, 4, 9, 16, 64)]
+    configs += [(f"nvfp4 M={M}", "nvfp4", [M], [(K, N, 6) for _, K, N, _ in DECODE_SHAPES])
+                for M in (1, 9, 64)]
+    out = {"cores": cores, "threads_per_core": 1, "rows_per_block": rows, "blocks_per_core": blocks,
+           "by_config": {}}
+    with cf.ProcessPoolExecutor(max_workers=cores, mp_context=mp.get_context("spawn"),
+                                initializer=_oracle_worker_init) as ex:
+        list(ex.map(_oracle_blocks, [("int4", 1, 256, 128, 0, 0, 16, 1)] * cores))   # warm the pool
+        for label, fmt, (M,), shapes in configs:
+            done = busy = 0.0
+            full = 0.0
+            for K, N, seed in shapes:
+                tasks = [(fmt, M, N, K, seed, c * rows * blocks, rows, blocks) for c in range(cores)]
+                res = list(ex.map(_oracle_blocks, tasks))
+                done += sum(r[0] for r in res)
+                busy += max(r[1] for r in res)
+                full += weight_bytes(fmt, N, K)
+            gbps = done / busy / 1e9
+            out["by_config"][label] = {"GBps": round(gbps, 4),
+                                       "s_per_step_extrapolated": round(full / (gbps * 1e9), 4)}
+    stack = sum(weight_bytes("int4", N, K) for _, K, N, _ in DECODE_SHAPES) * 64 + \
+        weight_bytes("int4", 248320, 5120)
+    for M, key in ((1, "decode int4 M=1"), (16, "verify int4 M=16"), (64, "verify int4 M=64")):
+        r = out["by_config"][key]["GBps"]
+        out["by_config"][f"whole stack int4 M={M} (extrapolated)"] = {
+            "GBps": r, "s_per_step_extrapolated": round(stack / (r * 1e9), 2)}
+    return out
+
+
 def cpu_oracle_step(rows_per_shape: int):
     """One reference step: the oracle on the first rows of every decode shape."""
     import oracle
@@ -297,30 +373,42 @@ def copies_for(weight_bytes):
     return max(2, min(16, int(np.ceil(3 * L2_BYTES / max(1, weight_bytes)))))
 
 
-def time_back_to_back(launch, reps, stream):
+REPEATS = 5
+
+
+def spread(values):
+    """Median and range of repeated timings (ms)."""
+    v = sorted(values)
+    return {"median": statistics.median(v), "min": v[0], "max": v[-1], "n": len(v)}
+
+
+def time_back_to_back(launch, reps, stream, repeats=REPEATS):
     """Capture ``reps`` calls of ``launch(r)`` back to back in one CUDA graph
     (no event between launches, so a launch may start its weight prologue
     while the previous one finishes, as in a decode step), replay it once to
-    warm up, then time one replay with CUDA events on the launching stream.
-    Returns milliseconds per call."""
+    warm up, then time ``repeats`` replays, each with its own CUDA events on
+    the launching stream and a synchronize on both sides.  Returns the
+    milliseconds per call of every replay."""
     import torch
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         for r in range(reps):
             launch(r)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         g.replay()  # warm replay
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        start.record()
-        g.replay()
-        end.record()
-    torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / reps
+    out = []
+    for _ in range(repeats):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            start.record()
+            g.replay()
+            end.record()
+        torch.cuda.synchronize()
+        out.append(start.elapsed_time(end) / reps)
     del g
-    return ms
+    return out
 
 
 def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
@@ -343,7 +431,8 @@ def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
         for r in range(3):
             launch(r)
     torch.cuda.synchronize()
-    us = time_back_to_back(launch, reps, stream) * 1e3
+    rep = spread([v * 1e3 for v in time_back_to_back(launch, reps, stream)])
+    us = rep["median"]
     b = alg_bytes(fmt, M, N, K)
     fl = flops(M, N, K)
     t_mem = b / (peaks["hbm_gbs"] * 1e9)
@@ -352,7 +441,8 @@ def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
     del ws
     torch.cuda.empty_cache()
     return {"fmt": fmt, "shape": name, "K": K, "N": N, "M": M, "path": int(path),
-            "us": round(us, 3), "GBps": round(b / us / 1e3, 1), "TFLOPs": round(fl / us / 1e6, 2),
+            "us": round(us, 3), "us_min": round(rep["min"], 3), "us_max": round(rep["max"], 3),
+            "GBps": round(b / us / 1e3, 1), "TFLOPs": round(fl / us / 1e6, 2),
             "bound": "hbm" if t_mem >= t_tc else "tensor",
             "frac_roofline": round(t_roof * 1e6 / us, 4),
             "frac_of_8TBps": round(b / us / 1e3 / 8000.0, 4)}
@@ -383,13 +473,15 @@ def gate_up_entry(fmt, M, seed, peaks, stream, reps=24):
         for r in range(3):
             launch(r)
     torch.cuda.synchronize()
-    us = time_back_to_back(launch, reps, stream) * 1e3
+    rep = spread([v * 1e3 for v in time_back_to_back(launch, reps, stream)])
+    us = rep["median"]
     b = alg_bytes(fmt, M, N, K) - 2 * M * N + 2 * M * I
     fl = flops(M, N, K)
     t_roof = max(b / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
     del ws
     torch.cuda.empty_cache()
     return {"fmt": fmt, "M": M, "K": K, "I": I, "path": int(path), "us": round(us, 3),
+            "us_min": round(rep["min"], 3), "us_max": round(rep["max"], 3),
             "GBps": round(b / us / 1e3, 1), "frac_roofline": round(t_roof * 1e6 / us, 4)}
 
 
@@ -423,10 +515,12 @@ def whole_stack(Ms, peaks, stream, reps=3):
         with torch.cuda.stream(stream):
             step(0)
         torch.cuda.synchronize()
-        ms = time_back_to_back(step, reps, stream)
+        rep = spread(time_back_to_back(step, reps, stream))
+        ms = rep["median"]
         b = sum(alg_bytes("int4", M, N, K) for K, N, _, _ in layers)
         fl = sum(flops(M, N, K) for K, N, _, _ in layers)
-        out["by_M"][str(M)] = {"ms_per_step": round(ms, 4), "steps_per_s": round(1e3 / ms, 2),
+        out["by_M"][str(M)] = {"ms_per_step": round(ms, 4), "ms_min": round(rep["min"], 4),
+                               "ms_max": round(rep["max"], 4), "steps_per_s": round(1e3 / ms, 2),
                                "GBps": round(b / ms / 1e6, 1), "TFLOPs": round(fl / ms / 1e9, 2),
                                "weight_bound_steps_per_s_at_peak": round(
                                    peaks["hbm_gbs"] * 1e9 / wbytes, 1)}
@@ -506,24 +600,30 @@ def run_native(args, rank, world, local_rank):
     while time.time() < soak_until:
         graph.replay()
         torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        start.record()
-        graph.replay()
-        end.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    # REPEATS timed replays of the K steps, each bracketed by a barrier and a
+    # synchronize; the line reports the median replay (max over ranks)
+    replay_ms = []
+    for _ in range(REPEATS):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            start.record()
+            graph.replay()
+            end.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        replay_ms.append(start.elapsed_time(end))
     t_end = time.time()
     time.sleep(0.25)
     sampler.stop()
-    ms_total = start.elapsed_time(end)
     W.check(W.w4a16_device_status(stream.cuda_stream), "device status")
-    ms_total = max_over_ranks([ms_total], world, "cuda")[0]
+    replay_ms = max_over_ranks(replay_ms, world, "cuda")
+    rep = spread(replay_ms)
+    ms_total = rep["median"]
     ms_per_step = ms_total / args.steps
     value = whole_job_gbps(world, step_bytes, args.steps, ms_total * 1e-3)
     clocks = sampler.summary(t_soak, t_end)
@@ -536,7 +636,8 @@ def run_native(args, rank, world, local_rank):
     n_launch = len(launches) * args.steps
     avg_ms = ms_total / n_launch
     achieved = float(launch_bytes.mean() / (avg_ms * 1e-3) / 1e9)
-    per_shape_ms = [time_back_to_back(fn, max(24, 2 * copies), stream) for fn in launches]
+    per_shape_rep = [spread(time_back_to_back(fn, max(24, 2 * copies), stream)) for fn in launches]
+    per_shape_ms = [r["median"] for r in per_shape_rep]
     traffic = load_traffic()
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -546,6 +647,9 @@ def run_native(args, rank, world, local_rank):
                 "avg_launch_us": round(avg_ms * 1e3, 3),
                 "per_shape_us": {name: round(per_shape_ms[j] * 1e3, 3)
                                  for j, (name, *_) in enumerate(wsets)},
+                "per_shape_us_range": {name: [round(per_shape_rep[j]["min"] * 1e3, 3),
+                                              round(per_shape_rep[j]["max"] * 1e3, 3)]
+                                       for j, (name, *_) in enumerate(wsets)},
                 "per_shape_frac": {name: round(float(launch_bytes[j] / (per_shape_ms[j] * 1e-3)
                                                      / 1e9 / peaks["hbm_gbs"]), 4)
                                    for j, (name, *_) in enumerate(wsets)}}
@@ -609,6 +713,8 @@ def run_native(args, rank, world, local_rank):
     if rank == 0 and world == 1:
         v, desc, secs = cpu_oracle_sample(args.cpu_seconds)
         cpu = {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+        if not args.no_cpu_all:
+            cpu["all_cores"] = cpu_oracle_all_cores()
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -625,6 +731,10 @@ def run_native(args, rank, world, local_rank):
                                      "launches it holds; per-shape durations from each shape "
                                      "alone, back to back in its own graph, one event pair",
                            "replicas": world},
+                "timing_repeats": {"ms_per_step": [round(v / args.steps, 5) for v in replay_ms],
+                                   "median": round(rep["median"] / args.steps, 5),
+                                   "min": round(rep["min"] / args.steps, 5),
+                                   "max": round(rep["max"] / args.steps, 5)},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
                 "gpu_launches": len(launches) * args.steps,
                 "peaks": peaks}
@@ -663,6 +773,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-stack", action="store_true")
+    ap.add_argument("--no-cpu-all", action="store_true", help="skip the all-cores oracle timing")
     ap.add_argument("--case", default=None,
                     help="profiling mode: launch one GEMM fmt,M,N,K[,path] --launches times")
     ap.add_argument("--launches", type=int, default=5)
