@@ -53,7 +53,8 @@ namespace {
 
 constexpr int kRowWords = 64;                                // per-row words (M <= 64)
 constexpr int kRowAuxOff = kRowWords * 4;
-constexpr int kRedOff = 2 * kRowWords * 4;                   // per-lane partial sums
+constexpr int kBarOff = 2 * kRowWords * 4;                   // mbarrier of the activation copy
+constexpr int kRedOff = kBarOff + 128;                       // per-lane partial sums
 constexpr int kMaxSmem = 232448;                             // 227 KB opt-in
 constexpr int kMaxDepth = 8;                                 // ring stages per warp
 constexpr int kGroupBytes = 2 * kTileBytes;                  // packed 4-bit weights of one band-group
@@ -77,7 +78,6 @@ struct Cfg {
   static constexpr int kWarps = 16;
   static constexpr int kRedBytes = kWarps * 32 * 4 * MT * 4 * (FUSE ? 2 : 1);  // per-lane partial sums
   static constexpr int kHeader = (kRedOff + kRedBytes + 127) / 128 * 128;
-  static constexpr int kCache = 4;                              // staging chunks in registers
 };
 
 struct Params {
@@ -90,6 +90,7 @@ struct Params {
   unsigned* counters;
   unsigned* err;
   int M, N, K, NT, S, kslice, row_stride;          // row_stride in bytes
+  int stage_log2;                                  // log2 of the staging threads per row
   int bq, br;                                      // bands per CTA: bq, plus one for the first br
   int wn, wn_log2, wk_log2;                        // warp grid: wn bands x 2^wk_log2 pieces
   int ngp;                                         // groups per piece, padded to the ring depth
@@ -136,67 +137,79 @@ __device__ __forceinline__ int perm64(int kin) {
   return t * 16 + j * 4 + e;
 }
 
-__device__ __forceinline__ float max_abs8(uint4 v) {
-  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-  float mx = 0.f;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    mx = fmaxf(mx, fabsf(__uint_as_float(u[e] << 16)));
-    mx = fmaxf(mx, fabsf(__uint_as_float(u[e] & 0xFFFF0000u)));
-  }
-  return mx;
+// Lane-wise maximum of two pairs of unsigned 16-bit integers.
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
-// Copy x[:, k_lo:k_lo+k_len] into the FP16 image (see the file comment).
-// Each row is handled by W/M whole warps, so a thread's chunks (8 BF16) all
-// belong to one row.  row_aux must be zero and visible to all threads on
-// entry; ends with a barrier after which the image and row_mul are valid.
-template <int CACHE>
-__device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t* xs,
-                                  float* row_mul, unsigned* row_aux) {
-  const int warps = blockDim.x >> 5;
-  const int wpr = warps / p.M;                      // warps per row (>= 1 since M <= warps)
+// 1-D bulk copy global -> shared completing on an mbarrier (no multicast):
+// both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Hint: bring a byte range into L2 (no data is returned to the SM, so it may
+// run before the previous kernel on the stream has finished writing it).
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// The CTA's slice of the activations as the FP16 image (see the file
+// comment).  Warp 0 has bulk-copied each row's raw BF16 slice into that row
+// of the image (completing on xbar); this waits for it, takes every row's
+// largest magnitude, and rewrites each 64-block in place as FP16 scaled by
+// the row's power of two, k permuted.  Every row has 2^stage_log2 threads (a
+// power of two, at least a warp; rows past M have idle threads), so a warp's
+// 32 lanes always hold the 8 chunks (16 bytes each) of 4 whole blocks of one
+// row and the in-place rewrite of a block needs only the warp itself.  All
+// 16 warps run this at once, so its cost is its instruction count: no
+// divisions, 32-bit offsets.  row_aux must be zero and visible on entry.
+// Ends with a barrier after which the image and row_mul are valid.  Returns
+// false if the copy did not complete (bounded wait).
+__device__ bool stage_activations(const Params& p, int k_len, uint8_t* xs, float* row_mul,
+                                  unsigned* row_aux, uint64_t* xbar) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = warp / wpr;
-  const bool worker = m < p.M;
-  const int tpr = wpr * 32;                         // threads per row
-  const int j = (warp - m * wpr) * 32 + lane;       // index within the row's threads
-  const int cpr = k_len / 8;                        // 16-byte chunks per row
-  const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)(worker ? m : 0) * p.K + k_lo);
-  uint4 cache[CACHE];
-  float mx = 0.f;
-  if (worker) {
-    for (int c0 = 0; c0 < cpr; c0 += CACHE * tpr) {
-#pragma unroll
-      for (int i = 0; i < CACHE; ++i) {
-        const int c = c0 + i * tpr + j;
-        const uint4 v = c < cpr ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-        if (c0 == 0) cache[i] = v;
-        mx = fmaxf(mx, max_abs8(v));
-      }
+  // warp 0 waits for the copy, the others at the barrier
+  const bool ok = __syncthreads_and(warp == 0 ? mbar_wait(xbar, 0, p.err) : true) != 0;
+  const int tpr = 1 << p.stage_log2;
+  const int m = threadIdx.x >> p.stage_log2;
+  const int c_first = (threadIdx.x & (tpr - 1)) - lane;      // this warp's first chunk of the row
+  const int cpr = k_len >> 3;                                 // 16-byte chunks per row
+  uint8_t* row = xs + m * p.row_stride;
+  if (m < p.M) {
+    // magnitudes compared as integers (BF16 bits with the sign cleared order
+    // like the values), two per instruction
+    uint32_t mx = 0u;
+    for (int c = c_first + lane; c < cpr; c += tpr) {
+      const uint4 v = *reinterpret_cast<const uint4*>(row + c * 16);
+      mx = vmax_u16x2(mx, vmax_u16x2(vmax_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                     vmax_u16x2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
     }
-    const unsigned r = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
-    if (lane == 0) atomicMax(row_aux + m, r);
+    const unsigned r = __reduce_max_sync(0xffffffffu, max(mx & 0xFFFFu, mx >> 16));
+    if (lane == 0) atomicMax(row_aux + m, r << 16);           // fp32 bits of the BF16 value
   }
   __syncthreads();
-  if (!worker) {
-    __syncthreads();
-    return;
-  }
-  const float rmax = __uint_as_float(row_aux[m]);
-  const bool scaled = rmax > 0.f && isfinite(rmax);
-  // max * 2^sh in [2^14, 2^15); |sh| <= 126 keeps 2^sh and 2^-sh normal floats
-  // (rows whose largest magnitude is below 2^-112 keep fewer FP16 bits)
-  const int sh = scaled ? min(126, 14 - ilogbf(rmax)) : 0;
-  const float mul = __int_as_float((127 + sh) << 23);        // 2^sh, exact
-  if (j == 0) row_mul[m] = __int_as_float((127 - sh) << 23);  // 2^-sh
-  uint8_t* row = xs + (size_t)m * p.row_stride;
-  for (int c0 = 0; c0 < cpr; c0 += CACHE * tpr) {
-#pragma unroll
-    for (int i = 0; i < CACHE; ++i) {
-      const int c = c0 + i * tpr + j;
+  if (m < p.M) {
+    const float rmax = __uint_as_float(row_aux[m]);
+    const bool scaled = rmax > 0.f && isfinite(rmax);
+    // max * 2^sh in [2^14, 2^15); |sh| <= 126 keeps 2^sh and 2^-sh normal floats
+    // (rows whose largest magnitude is below 2^-112 keep fewer FP16 bits)
+    const int sh = scaled ? min(126, 14 - ilogbf(rmax)) : 0;
+    const float mul = __int_as_float((127 + sh) << 23);       // 2^sh, exact
+    if (c_first + lane == 0) row_mul[m] = __int_as_float((127 - sh) << 23);   // 2^-sh
+    for (int c0 = c_first; c0 < cpr; c0 += tpr) {
+      const int c = c0 + lane;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (c < cpr) v = *reinterpret_cast<const uint4*>(row + c * 16);
+      __syncwarp();                                 // the 4 blocks are read before any is rewritten
       if (c < cpr) {
-        const uint4 v = c0 == 0 ? cache[i] : src[c];
         uint32_t out[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -205,15 +218,22 @@ __device__ void stage_activations(const Params& p, int k_lo, int k_len, uint8_t*
           __half2 h = __floats2half2_rn(lo, hi);
           out[e] = *reinterpret_cast<uint32_t*>(&h);
         }
-        const int kin0 = c * 8;
-        uint8_t* blk = row + (kin0 >> 6) * 128;
-        const int in = kin0 & 63;
-        *reinterpret_cast<uint2*>(blk + perm64(in) * 2) = make_uint2(out[0], out[1]);
-        *reinterpret_cast<uint2*>(blk + perm64(in + 4) * 2) = make_uint2(out[2], out[3]);
+        uint8_t* blk = row + (c >> 3) * 128;
+        const int in = (c & 7) * 8;
+        // the first half of a chunk lands in banks 0-7 / 16-23 of its block,
+        // the second in 8-15 / 24-31: odd blocks store them in the other
+        // order, so each half-warp's stores cover all 32 banks once
+        const bool odd = (c >> 3) & 1;
+        const uint2 first = odd ? make_uint2(out[2], out[3]) : make_uint2(out[0], out[1]);
+        const uint2 second = odd ? make_uint2(out[0], out[1]) : make_uint2(out[2], out[3]);
+        *reinterpret_cast<uint2*>(blk + perm64(in + (odd ? 4 : 0)) * 2) = first;
+        *reinterpret_cast<uint2*>(blk + perm64(in + (odd ? 0 : 4)) * 2) = second;
       }
+      __syncwarp();
     }
   }
   __syncthreads();
+  return ok;
 }
 
 // c = A . B (fresh accumulator), fp32
@@ -384,6 +404,34 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
   prev = __shfl_sync(0xffffffffu, prev, 0);
   if (prev != static_cast<unsigned>(p.S - 1)) return;
   __threadfence();
+  // sum the splits in split order; the loads of kB splits are issued
+  // together (one round trip per batch instead of one per split)
+  constexpr int kV = MT * 4 * (FUSE ? 2 : 1);          // values of this lane
+  constexpr int kB = 32 / kV;                          // 32 loads in flight per lane
+  float sum[kV];
+#pragma unroll
+  for (int j = 0; j < kV; ++j) sum[j] = 0.f;
+  const size_t sstride = (size_t)p.M * Npad;
+  for (int sp0 = 0; sp0 < p.S; sp0 += kB) {
+    float part[kB][kV];
+#pragma unroll
+    for (int b = 0; b < kB; ++b)
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = mt * 8 + 2 * t + (i & 1);
+          const int n = n0 + 8 * (i >> 1);
+          const bool ld = sp0 + b < p.S && m < p.M && n < cols;
+          const float* src = p.ws + (size_t)(sp0 + b) * sstride + (size_t)m * Npad + n;
+          part[b][mt * 4 + i] = ld ? __ldcg(src) : 0.f;
+          if (FUSE) part[b][MT * 4 + mt * 4 + i] = ld ? __ldcg(src + p.I) : 0.f;
+        }
+#pragma unroll
+    for (int b = 0; b < kB; ++b)
+#pragma unroll
+      for (int j = 0; j < kV; ++j) sum[j] += part[b][j];
+  }
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -391,14 +439,8 @@ __device__ __forceinline__ void band_epilogue(const Params& p, int band, int spl
       const int m = mt * 8 + 2 * t + (i & 1);
       const int n = n0 + 8 * (i >> 1);
       if (m < p.M && n < cols) {
-        float v = 0.f, u = 0.f;
-        for (int sp = 0; sp < p.S; ++sp) {
-          const float* src = p.ws + ((size_t)sp * p.M + m) * Npad + n;
-          v += __ldcg(src);
-          if (FUSE) u += __ldcg(src + p.I);
-        }
-        v *= gmul;
-        if (FUSE) v = silu_f32(v) * (u * gmul);
+        float v = sum[mt * 4 + i] * gmul;
+        if (FUSE) v = silu_f32(v) * (sum[MT * 4 + mt * 4 + i] * gmul);
         p.y[(size_t)m * cols + n] = __float2bfloat16_rn(v);
       }
     }
@@ -423,7 +465,12 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
   const int g = lane >> 2, t = lane & 3;
   const uint8_t* ring = smem + C::kHeader + warp * D * kSB;       // this warp's stages
   uint8_t* xs = smem + C::kHeader + C::kWarps * D * kSB;          // activation image
+  uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   if (threadIdx.x < kRowWords) row_aux[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) {
+    mbar_init(xbar, 1);
+    fence_mbar_init();
+  }
   pdl_launch_dependents();
 
   // work of this CTA and warp (no divisions: the host passes quotients and
@@ -503,18 +550,24 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
     }
   };
 
-  // The first groups go out before the activations are staged, the rest of
-  // the first block right after: a full block of copies queued ahead of the
-  // activation loads delays them behind the weights (measured).
-  constexpr int kPre = D < 2 ? D : 2;
+  // Before the previous kernel on the stream has finished: the activation
+  // slice is prefetched into L2 (a hint only) and the whole first block of
+  // the weight ring is issued (weights are never written by a kernel here).
+  const uint32_t x_bytes = (uint32_t)groups * 256;   // one row's slice, BF16
+  if (threadIdx.x < p.M) prefetch_l2(p.x + (size_t)threadIdx.x * p.K + k_lo, x_bytes);
 #pragma unroll
-  for (int k = 0; k < kPre; ++k) copy_item(k);
+  for (int k = 0; k < D; ++k) copy_item(k);
 
   pdl_wait();          // the activations may come from the previous kernel
-  __syncthreads();     // row_aux zeroed
-  stage_activations<C::kCache>(p, k_lo, groups * 128, xs, row_mul, row_aux);
-#pragma unroll
-  for (int k = kPre; k < D; ++k) copy_item(k);
+  __syncthreads();     // row_aux zeroed, xbar initialised
+  if (warp == 0) {
+    if (lane == 0) mbar_arrive_expect_tx(xbar, x_bytes * p.M);
+    __syncwarp();
+    if (lane < p.M)
+      bulk_g2s(smem_u32(xs + lane * p.row_stride), p.x + (size_t)lane * p.K + k_lo, x_bytes,
+               smem_u32(xbar));
+  }
+  const bool x_ok = stage_activations(p, groups * 128, xs, row_mul, row_aux, xbar);
   next_block();
 
   // activation rows of this lane (row m = 8 mt + g); rows past M alias row 0:
@@ -626,6 +679,7 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
     __syncthreads();
   }
   cpa_wait<0>();  // nothing is in flight at exit
+  if (!x_ok) mbar_wait(xbar, 0, p.err);   // the activation copy, if it ever lands
 }
 
 // Raise the dynamic shared memory limit of one kernel variant, once per
@@ -694,6 +748,8 @@ cudaError_t launch_t(const GemvPlan& pl, const GemmArgs& a, cudaStream_t st) {
   p.bq = p.NT / pl.ctas_x;
   p.br = p.NT % pl.ctas_x;
   p.row_stride = (pl.kslice / 64) * 128 + 16;
+  // staging threads per row: the CTA's threads over M rounded up to a power of two
+  p.stage_log2 = ilog2(Cfg<FMT, MT, FUSE>::kWarps * 32) - ilog2(a.M);
   p.wn = pl.wn;
   p.wn_log2 = ilog2(pl.wn);
   p.wk_log2 = ilog2(pl.wk);

@@ -278,11 +278,17 @@ struct TcShape {
   static constexpr int kASlots = (kTmemCols - kAColBase) / 128;
   static constexpr int kXStage = 2 * MPAD * 128;             // two 64-k activation boxes
   static constexpr int kWRingBytes = kDeqWarps * kWRing * tc_stage_bytes(FMT);
-  static constexpr int kXRing =                               // activation stages (groups)
-      4 * kXStage + kWRingBytes + 2048 <= kMaxSmem ? 4 : 3;
+  // activation stages (groups): as many as fit, up to 8.  Every CTA reads the
+  // same activation tile at about the same time, so a load takes thousands
+  // of cycles to land (measured); the depth of this ring, not the bytes,
+  // sets how fast the MMA warp can be fed.
+  static constexpr int kXFit = (kMaxSmem - kWRingBytes - 2048) / kXStage;
+  static constexpr int kXRing = kXFit > 8 ? 8 : kXFit;
   static constexpr int kSmemUse = kXRing * kXStage + kWRingBytes + 1024 /* barriers */;
   static constexpr int kSmem = (kSmemUse + 1024 /* align */ > kMinSmem) ? kSmemUse + 1024 : kMinSmem;
   static_assert(kSmem <= kMaxSmem, "stage rings exceed shared memory");
+  static_assert(kXRing >= 3, "activation ring");
+  static_assert(2 * kXRing + 2 * kASlots + 4 <= 128, "barrier area");
   static_assert(kASlots >= 2 && kAColBase + kASlots * 128 <= kTmemCols, "tensor memory layout");
   static_assert(MPAD % 16 == 0 && MPAD <= kTcMaxRows, "MMA N");
 };
