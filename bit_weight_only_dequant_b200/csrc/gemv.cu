@@ -21,9 +21,11 @@
 //    barrier guards the ring; only the lane's own cp.async groups are waited
 //    for.  The ring holds up to eight groups per warp (up to 144 KB per SM
 //    in flight) without spending registers, and runs on from one band's
-//    piece into the next.  The first copies are issued before the activations
-//    are staged and, under programmatic dependent launch, before the previous
-//    kernel on the stream has finished: only the activations depend on it.
+//    piece into the next.  Under programmatic dependent launch the CTA starts
+//    before the previous kernel on the stream has finished but then only
+//    prefetches its first weights and the activations into L2: any operand
+//    may have been written by that kernel, so every read into the SM comes
+//    after griddepcontrol.wait.
 //  * The CTA copies its slice of the activations into shared memory as FP16,
 //    each row rescaled by a power of two so that its largest magnitude lies in
 //    [2^14, 2^15) (exact for every BF16 value in FP16's normal range), k
@@ -176,8 +178,14 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 __device__ bool stage_activations(const Params& p, int k_len, uint8_t* xs, float* row_mul,
                                   unsigned* row_aux, uint64_t* xbar) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // warp 0 waits for the copy, the others at the barrier
-  const bool ok = __syncthreads_and(warp == 0 ? mbar_wait(xbar, 0, p.err) : true) != 0;
+  // warp 0 waits for the copy (converged again before the barrier), the
+  // others at the barrier
+  bool ok_w = true;
+  if (warp == 0) {
+    ok_w = mbar_wait(xbar, 0, p.err);
+    ok_w = __all_sync(0xffffffffu, ok_w);
+  }
+  const bool ok = __syncthreads_and(ok_w) != 0;
   const int tpr = 1 << p.stage_log2;
   const int m = threadIdx.x >> p.stage_log2;
   const int c_first = (threadIdx.x & (tpr - 1)) - lane;      // this warp's first chunk of the row
@@ -550,15 +558,25 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
     }
   };
 
-  // Before the previous kernel on the stream has finished: the activation
-  // slice is prefetched into L2 (a hint only) and the whole first block of
-  // the weight ring is issued (weights are never written by a kernel here).
+  // Before the previous kernel on the stream has finished, only hints: the
+  // activation slice and this warp's first block of weights are prefetched
+  // into L2.  Any operand may have been written by that kernel (a packer, a
+  // previous layer), so nothing is read into the SM before the wait.
   const uint32_t x_bytes = (uint32_t)groups * 256;   // one row's slice, BF16
   if (threadIdx.x < p.M) prefetch_l2(p.x + (size_t)threadIdx.x * p.K + k_lo, x_bytes);
+  if (lane == 0 && c_blocks > 0 && ng > 0) {
+    const uint32_t n0 = (uint32_t)min(D, ng);        // the block's groups, contiguous from cw
+    prefetch_l2(cw, n0 * kGB);
+    if (FMT != kFmtFp8) prefetch_l2(cs, n0 * kSStep);
+    if (FUSE) {
+      prefetch_l2(cw + p.up_w, n0 * kGB);
+      if (FMT != kFmtFp8) prefetch_l2(cs + p.up_s, n0 * kSStep);
+    }
+  }
+
+  pdl_wait();          // the operands may come from the previous kernel
 #pragma unroll
   for (int k = 0; k < D; ++k) copy_item(k);
-
-  pdl_wait();          // the activations may come from the previous kernel
   __syncthreads();     // row_aux zeroed, xbar initialised
   if (warp == 0) {
     if (lane == 0) mbar_arrive_expect_tx(xbar, x_bytes * p.M);
