@@ -448,6 +448,40 @@ def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
             "frac_of_8TBps": round(b / us / 1e3 / 8000.0, 4)}
 
 
+def w4a4_entry(name, K, N, M, seed, peaks, stream, reps=24):
+    """W4A4 NVFP4 (activations quantised inside the call) at one decode shape:
+    the quantiser and the matmul, back to back like the sweep.  Algorithmic
+    bytes: the NVFP4 weights and scales, x and y."""
+    import torch
+    from bit_weight_only_dequant_b200 import w4a16 as W
+    f = W.FMTS["nvfp4"]
+    wbytes = W.w4a16_packed_weight_bytes(f, N, K) + W.w4a16_packed_scale_bytes(f, N, K)
+    ws = make_weights("nvfp4", seed, N, K, copies_for(wbytes))
+    x = make_x("nvfp4", seed, M, K)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda")
+
+    def launch(r, ws=ws):
+        pw, ps = ws[r % len(ws)]
+        W.check(W.w4a16_gemm_w4a4(M, N, K, x, pw, ps, g, y, stream.cuda_stream), "gemm_w4a4")
+
+    with torch.cuda.stream(stream):
+        for r in range(3):
+            launch(r)
+    torch.cuda.synchronize()
+    rep = spread([v * 1e3 for v in time_back_to_back(launch, reps, stream)])
+    us = rep["median"]
+    b = alg_bytes("nvfp4", M, N, K)
+    fl = flops(M, N, K)
+    t_roof = max(b / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+    del ws
+    torch.cuda.empty_cache()
+    return {"fmt": "w4a4_nvfp4", "shape": name, "K": K, "N": N, "M": M,
+            "path": int(W.w4a16_gemm_path(f, M, N, K)), "us": round(us, 3),
+            "us_min": round(rep["min"], 3), "us_max": round(rep["max"], 3),
+            "GBps": round(b / us / 1e3, 1), "frac_roofline": round(t_roof * 1e6 / us, 4)}
+
+
 def gate_up_entry(fmt, M, seed, peaks, stream, reps=24):
     """The fused gate/up layer h = SiLU(gate) * up at the decode gate/up shape
     (K = 5120, I = 17408: the 34816-row weight), back to back like the sweep.
@@ -702,6 +736,8 @@ def run_native(args, rank, world, local_rank):
         for fmt, n, K, N, Mv, s in target + cfg2 + cfg3 + cfg4 + cfg5:
             entries.append(sweep_entry(fmt, n, K, N, Mv, s, peaks, stream))
         extra["sweep"] = entries
+        extra["w4a4"] = [w4a4_entry(n, K, N, Mv, 6, peaks, stream) for Mv in (1, 9, 64)
+                         for n, K, N, _ in DECODE_SHAPES]
         extra["gate_up_silu"] = [gate_up_entry(fmt, Mv, 3, peaks, stream)
                                  for fmt, Mv in (("int4", 1), ("int4", 4), ("int4", 9),
                                                  ("int4", 16), ("int4", 64), ("int4", 256),

@@ -272,6 +272,29 @@ int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packe
                                       static_cast<cudaStream_t>(stream)));
 }
 
+// W4A4: scratch of its own per (device, stream) -- [amax word, g_x, g_eff,
+// pad to 256 B][block-scaled activations BF16 M x K] -- so that the matmul's
+// own workspace can grow without freeing memory this call still reads.
+std::map<std::pair<int, cudaStream_t>, Workspace> g_w4a4_ws;
+
+int w4a4_scratch(cudaStream_t st, size_t bytes, uint8_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W4A16_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_w4a4_ws[std::make_pair(dev, st)];
+  if (w.base == nullptr || w.bytes < bytes) {
+    size_t nb = bytes > 2 * w.bytes ? bytes : 2 * w.bytes;
+    nb = (nb + 255) / 256 * 256;
+    void* base = nullptr;
+    if (cudaMallocAsync(&base, nb, st) != cudaSuccess) return W4A16_ERR_NOMEM;
+    if (w.base) cudaFreeAsync(w.base, st);
+    w.base = base;
+    w.bytes = nb;
+  }
+  *out = static_cast<uint8_t*>(w.base);
+  return W4A16_OK;
+}
+
 int w4a16_gemm_path(int fmt, int M, int N, int K) {
   const int r = check_fmt_shape(fmt, N, K);
   if (r != W4A16_OK) return r;
@@ -305,6 +328,57 @@ int w4a16_gemm(int fmt, int M, int N, int K, const void* x_bf16, const void* pac
                const void* packed_scales, const float* global_scale, void* y_bf16, void* stream) {
   return w4a16_gemm_ex(W4A16_PATH_AUTO, fmt, M, N, K, x_bf16, packed_w, packed_scales,
                        global_scale, y_bf16, stream);
+}
+
+int w4a16_quantize_act_nvfp4(int M, int K, const void* x_bf16, void* codes, void* scales,
+                             float* g_x, void* stream) {
+  if (M < 1 || M > W4A16_MAX_M || K < 128 || K % 128 != 0) return W4A16_ERR_SHAPE;
+  if (!x_bf16 || !codes || !scales || !g_x) return W4A16_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(codes)) return W4A16_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  int r = device_state(&d);
+  if (r != W4A16_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* scratch = nullptr;
+  if ((r = w4a4_scratch(st, 256, &scratch)) != W4A16_OK) return r;
+  return status_of(w4::launch_act_quant(M, K, x_bf16, reinterpret_cast<unsigned*>(scratch),
+                                        nullptr, codes, scales, nullptr, g_x, nullptr, st));
+}
+
+int w4a16_gemm_w4a4_ex(int path, int M, int N, int K, const void* x_bf16, const void* packed_w,
+                       const void* packed_scales, const float* global_scale_w, void* y_bf16,
+                       void* stream) {
+  int r = check_fmt_shape(W4A16_FMT_NVFP4_G16, N, K);
+  if (r != W4A16_OK) return r;
+  if (M < 1 || M > W4A16_MAX_M) return W4A16_ERR_SHAPE;
+  if (!x_bf16 || !packed_w || !packed_scales || !global_scale_w || !y_bf16) return W4A16_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(packed_w) || !aligned16(packed_scales) || !aligned16(y_bf16))
+    return W4A16_ERR_ALIGN;
+  if (path != W4A16_PATH_AUTO && path != W4A16_PATH_GEMV && path != W4A16_PATH_TC)
+    return W4A16_ERR_ARG;
+  if (path == W4A16_PATH_GEMV && M > W4A16_GEMV_MAX_M) return W4A16_ERR_SHAPE;
+  DeviceState* d = nullptr;
+  if ((r = device_state(&d)) != W4A16_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* scratch = nullptr;
+  if ((r = w4a4_scratch(st, 256 + (size_t)M * K * 2, &scratch)) != W4A16_OK) return r;
+  unsigned* amax = reinterpret_cast<unsigned*>(scratch);
+  float* g_eff = reinterpret_cast<float*>(scratch + 8);
+  void* xq = scratch + 256;
+  cudaError_t e = w4::launch_act_quant(M, K, x_bf16, amax, global_scale_w, nullptr, nullptr, xq,
+                                       nullptr, g_eff, st);
+  if (e != cudaSuccess) return W4A16_ERR_CUDA;
+  // the block-scaled activations are exact BF16 values; the NVFP4 matmul on
+  // them with the per-tensor scale g_w * g_x is the W4A4 product
+  return run_gemm(path, W4A16_FMT_NVFP4_G16, M, N, K, xq, packed_w, packed_scales, g_eff, y_bf16,
+                  stream, 0);
+}
+
+int w4a16_gemm_w4a4(int M, int N, int K, const void* x_bf16, const void* packed_w,
+                    const void* packed_scales, const float* global_scale_w, void* y_bf16,
+                    void* stream) {
+  return w4a16_gemm_w4a4_ex(W4A16_PATH_AUTO, M, N, K, x_bf16, packed_w, packed_scales,
+                            global_scale_w, y_bf16, stream);
 }
 
 int w4a16_plan(int path, int fmt, int M, int N, int K, int fuse, int num_sms, int* out,

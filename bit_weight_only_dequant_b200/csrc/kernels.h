@@ -68,6 +68,15 @@ cudaError_t launch_tc(const TcPlan& p, const GemmArgs& a, void* xf16_scratch, cu
 // Diagnostics: a bounded mbarrier wait that is made to run out (see capi.cu).
 cudaError_t launch_wait_timeout_selftest(unsigned* err, int* out, cudaStream_t st);
 
+// ---------------------------------------------------------------- W4A4: activation quantiser
+
+// x [M][K] BF16 -> NVFP4 (codes, E4M3 block scales, fp32 g_x); every output
+// optional.  amax_bits: one device word of scratch.  xq: the block-scaled
+// values e2m1 * e4m3 as BF16 [M][K]; g_eff: g_w * g_x (g_w may be null: g_x).
+cudaError_t launch_act_quant(int M, int K, const void* x, unsigned* amax_bits, const float* g_w,
+                             void* codes, void* scales, void* xq, float* g_x, float* g_eff,
+                             cudaStream_t st);
+
 // ---------------------------------------------------------------- dequant export / packer
 
 cudaError_t launch_dequant(int fmt, int N, int K, const void* w, const void* s, const float* g,

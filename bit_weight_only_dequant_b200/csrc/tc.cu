@@ -385,13 +385,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     if (lane == 0) {
+      int s = 0;                      // ring stage of group `it`
+      uint32_t u = 0;                 // times the ring has wrapped (it / kXRing)
       for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
         int tile, chunk, split, g_lo, g_hi;
         unit_range(p, unit, tile, chunk, split, g_lo, g_hi);
         const int xrow = chunk * p.rows;
-        for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
-          const int s = it % kXRing;
-          const uint32_t u = it / kXRing;
+        for (int gi = g_lo; gi < g_hi; ++gi, ++it, s = s + 1 == kXRing ? 0 : s + 1,
+                 u += s == 0 ? 1u : 0u) {
           if (u > 0 && !tc_wait(xfree + s, (u - 1) & 1, abort_flag, p.err)) {
             ok = false;
             break;
@@ -412,6 +413,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---------------------------------------------------------------- MMA issuer (whole warp)
     constexpr uint32_t idesc = make_idesc(FMT == 0 ? 1 : 0, MPAD);
     uint32_t it = 0, unit_i = 0;
+    int x_slot = 0, a_slot = 0;       // stage / slot of group `it`
+    uint32_t x_par = 0, a_par = 0;    // their phase parity
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
       int tile, chunk, split, g_lo, g_hi;
@@ -423,11 +426,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
       }
       for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
-        const int xs_ = it % kXRing, sl = it % kASlots;
-        if (!warp_wait(xfull + xs_, (it / kXRing) & 1, abort_flag, p.err) ||
-            !warp_wait(afull + sl, (it / kASlots) & 1, abort_flag, p.err)) {
+        const int xs_ = x_slot, sl = a_slot;
+        if (!warp_wait(xfull + xs_, x_par, abort_flag, p.err) ||
+            !warp_wait(afull + sl, a_par, abort_flag, p.err)) {
           ok = false;
           break;
+        }
+        // the next group's stage / slot and phase parity (no division)
+        if (++x_slot == kXRing) {
+          x_slot = 0;
+          x_par ^= 1u;
+        }
+        if (++a_slot == kASlots) {
+          a_slot = 0;
+          a_par ^= 1u;
         }
         tc_fence_after();
         const uint64_t b0 = sw128_desc(smem_u32(Xs + xs_ * Sh::kXStage));
@@ -532,14 +544,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int k = 0; k < kWRing; ++k) copy_next();
 
     uint32_t it = 0, unit_i = 0;
+    int sl = 0;                       // tensor-memory slot of group `it`
+    uint32_t ua = 0;                  // times the slots have wrapped (it / kASlots)
+    const uint32_t a_base = tmem + lane_base + kAColBase + h * 64;
     bool ok = true;
     for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x, ++unit_i) {
       int tile, chunk, split, g_lo, g_hi;
       unit_range(p, unit, tile, chunk, split, g_lo, g_hi);
       const bool real_band = p.fuse ? tile * 8 + (band & 7) < (p.I >> 4) : tile * 16 + band < p.NT;
       for (int gi = g_lo; gi < g_hi; ++gi, ++it) {
-        const int sl = it % kASlots;
-        const uint32_t ua = it / kASlots;
         cpa_wait<kWRing - 1>();                          // this lane's bytes of group `it`
         const uint8_t* st = ring + (it % kWRing) * kSB;
         uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0, w2 = w0, w3 = w0;
@@ -608,12 +621,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               r[4 * k + 3] = hmul2_f16(e2m1x2_to_f16x2(wd[k] >> 24), s_hi);
             }
           }
-          tmem_st_16x256b_x4(tmem + lane_base + kAColBase + sl * 128 + h * 64 + blk * 32, r);
+          tmem_st_16x256b_x4(a_base + sl * 128 + blk * 32, r);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(afull + sl);
+        if (++sl == kASlots) {
+          sl = 0;
+          ++ua;
+        }
       }
       if (!ok) break;
 

@@ -1,0 +1,179 @@
+// W4A4 NVFP4: the activations quantised to NVFP4 as well (model card
+// "SuperQwen3.8-27b-abliterated-NVFP4-2xDGX", table "Release highlights":
+// W4A4 NVFP4, group size 16).  The pages name only the format; the reading
+// taken (the plainest one consistent with the weight side of the format):
+//
+//   g_x = fp32(amax |x|) / fp32(6 * 448)        one fp32 scale per tensor
+//                                               (1.0 for an all-zero x)
+//   s   = RNE_e4m3(amax_block / (6 * g_x))      one E4M3 scale per row and
+//                                               16 consecutive k, saturating
+//                                               at 448
+//   q   = RNE_e2m1(x / (e4m3(s) * g_x))         E2M1 codes, ties to the even
+//                                               code, saturating at +-6
+//
+// every product and division in fp32 with round-to-nearest (no contraction),
+// so the codes and scales are decided exactly as a reference that follows the
+// same steps in fp32 decides them.  The rounding onto E4M3 and E2M1 is done
+// with explicit comparisons and integer arithmetic, not with the hardware
+// conversions, so that every tie and saturation rule is the one stated here.
+//
+// The quantised activation x_hat = e2m1(q) * e4m3(s) * g_x: e2m1 * e4m3 has
+// at most 6 significant bits and lies in [2^-10, 2688], so it is exact in
+// BF16 and FP16; the product with g_x is left to the matmul, whose per-tensor
+// scale becomes g_w * g_x.  The matmul itself is then the NVFP4 path of this
+// library on the block-scaled activation values: at decode and verify row
+// counts W4A4 moves the same weight bytes as W4A16, so the same kernels bound
+// it.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace w4 {
+
+namespace {
+
+// Largest |x| of the tensor as the fp32 bits of a BF16 value (magnitude bits
+// compared as integers, which order like the values).  amax_bits must be zero.
+__global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __restrict__ x,
+                                                       long long n8, unsigned* amax_bits) {
+  const uint4* v = reinterpret_cast<const uint4*>(x);
+  uint32_t mx = 0u;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+       i += (long long)gridDim.x * blockDim.x) {
+    const uint4 c = __ldg(v + i);
+    const uint32_t w[4] = {c.x & 0x7FFF7FFFu, c.y & 0x7FFF7FFFu, c.z & 0x7FFF7FFFu,
+                           c.w & 0x7FFF7FFFu};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mx = max(mx, max(w[j] & 0xFFFFu, w[j] >> 16));
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, mx << 16);
+}
+
+// RNE onto E4M3 of a non-negative, finite fp32 value, saturating at 448
+// (0x7E); the value 480 that rounding could reach is not finite in E4M3.
+__device__ __forceinline__ uint32_t rne_e4m3(float t) {
+  if (!(t > 0.f)) return 0u;
+  if (t >= 448.f) return 0x7Eu;
+  if (t < 0.015625f) {                               // below 2^-6: quantum 2^-9
+    // t * 2^9 is exact; rintf rounds half to even; the result 8 is the
+    // smallest normal 2^-6, whose code is also 8
+    return (uint32_t)rintf(t * 512.f);
+  }
+  int e;
+  const float m = frexpf(t, &e);                     // t = m 2^e, m in [0.5, 1)
+  // 4 significant bits: mantissa steps of 2^(e-4)
+  uint32_t r = (uint32_t)rintf(ldexpf(m, 4));        // 8 .. 16, exact scaling
+  if (r == 16u) {
+    r = 8u;
+    ++e;
+  }
+  // value = r 2^(e-4) = (1 + (r-8)/8) 2^(e-1): exponent field e - 1 + 7
+  const uint32_t code = ((uint32_t)(e + 6) << 3) | (r - 8u);
+  return code > 0x7Eu ? 0x7Eu : code;
+}
+
+// RNE onto E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the code
+// whose mantissa bit is 0, saturating at 6; the sign goes to bit 3 (negative
+// zero included).  The thresholds are the midpoints between neighbours, each
+// tie going to the even side.
+__device__ __forceinline__ uint32_t rne_e2m1(float v) {
+  const float a = fabsf(v);
+  const uint32_t mag = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+                       (a >= 3.5f) + (a > 5.f);
+  return mag | (signbit(v) ? 8u : 0u);
+}
+
+__device__ __forceinline__ float e2m1_mag(uint32_t c) {
+  const uint32_t m = c & 7u;
+  return m < 2 ? 0.5f * m : ldexpf(1.f + 0.5f * (m & 1u), (int)(m >> 1) - 1);
+}
+
+__device__ __forceinline__ float e4m3_val(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  return e == 0 ? ldexpf((float)m, -9) : ldexpf(1.f + m * 0.125f, (int)e - 7);
+}
+
+__device__ __forceinline__ float global_scale(unsigned amax_bits) {
+  const float amax = __uint_as_float(amax_bits);
+  return amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f;   // 6 * 448 = 2688 exactly
+}
+
+// One thread per (row, 16-block): codes (one per byte, [M][K]), the E4M3
+// scale ([M][K/16]) and the block-scaled values e2m1 * e4m3 as BF16 ([M][K]),
+// each output optional.  Thread 0 also writes g_x and, if g_w is given,
+// g_w * g_x (fp32, one rounding): the matmul's per-tensor scale.
+__global__ void __launch_bounds__(256)
+    act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
+                     const unsigned* __restrict__ amax_bits, const float* __restrict__ g_w,
+                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                     __nv_bfloat16* __restrict__ xq, float* g_x_out, float* g_eff_out) {
+  const float g = global_scale(__ldg(amax_bits));
+  const long long nblk = (long long)M * (K >> 4);
+  const long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (b == 0) {
+    if (g_x_out) *g_x_out = g;
+    if (g_eff_out) *g_eff_out = g_w ? __fmul_rn(__ldg(g_w), g) : g;
+  }
+  if (b >= nblk) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x) + 2 * b;
+  const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
+  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  float v[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[2 * j] = __uint_as_float(w[j] << 16);
+    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+  float amax_b = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) amax_b = fmaxf(amax_b, fabsf(v[j]));
+  const float t = __fdiv_rn(amax_b, __fmul_rn(6.f, g));
+  const uint32_t s8 = rne_e4m3(t);
+  const float sv = e4m3_val(s8);
+  const float step = __fmul_rn(sv, g);
+  uint32_t q[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) q[j] = step > 0.f ? rne_e2m1(__fdiv_rn(v[j], step)) : 0u;
+  if (codes) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      pk[j] = q[4 * j] | (q[4 * j + 1] << 8) | (q[4 * j + 2] << 16) | (q[4 * j + 3] << 24);
+    *reinterpret_cast<uint4*>(codes + 16 * b) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+  if (scales) scales[b] = (uint8_t)s8;
+  if (xq) {
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      // e2m1 * e4m3: at most 6 significant bits, exact in fp32 and in BF16
+      const float lo = (q[2 * j] & 8u ? -1.f : 1.f) * e2m1_mag(q[2 * j]) * sv;
+      const float hi = (q[2 * j + 1] & 8u ? -1.f : 1.f) * e2m1_mag(q[2 * j + 1]) * sv;
+      __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+      o[j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(xq) + 2 * b;
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(int M, int K, const void* x, unsigned* amax_bits, const float* g_w,
+                             void* codes, void* scales, void* xq, float* g_x, float* g_eff,
+                             cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  const long long n8 = (long long)M * K / 8;
+  const int grid_a = (int)min(1184ll, (n8 + 255) / 256);
+  act_amax_kernel<<<grid_a, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), n8, amax_bits);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const long long nblk = (long long)M * (K / 16);
+  act_quant_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), M, K, amax_bits, g_w, static_cast<uint8_t*>(codes),
+      static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xq), g_x, g_eff);
+  return cudaGetLastError();
+}
+
+}  // namespace w4

@@ -44,6 +44,9 @@ _SIGS = {
     "w4a16_gemm_gate_up_silu": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_gate_up_silu_ex": (_i, [_i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_quantize_act_nvfp4": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_gemm_w4a4": (_i, [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_gemm_w4a4_ex": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_device_status": (_i, [_vp]),
     "w4a16_selftest_wait_timeout": (_i, [_vp]),
     "w4a16_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _i]),
@@ -160,6 +163,21 @@ def w4a16_gemm_gate_up_silu_ex(path, fmt, M, I, K, x, packed_w, packed_scales, g
                                             _stream(stream))
 
 
+def w4a16_quantize_act_nvfp4(M, K, x, codes, scales, g_x, stream=None):
+    return lib().w4a16_quantize_act_nvfp4(M, K, _ptr(x), _ptr(codes), _ptr(scales), _ptr(g_x),
+                                          _stream(stream))
+
+
+def w4a16_gemm_w4a4(M, N, K, x, packed_w, packed_scales, global_scale_w, y, stream=None):
+    return lib().w4a16_gemm_w4a4(M, N, K, _ptr(x), _ptr(packed_w), _ptr(packed_scales),
+                                 _ptr(global_scale_w), _ptr(y), _stream(stream))
+
+
+def w4a16_gemm_w4a4_ex(path, M, N, K, x, packed_w, packed_scales, global_scale_w, y, stream=None):
+    return lib().w4a16_gemm_w4a4_ex(path, M, N, K, _ptr(x), _ptr(packed_w), _ptr(packed_scales),
+                                    _ptr(global_scale_w), _ptr(y), _stream(stream))
+
+
 def w4a16_gemm_path(fmt, M, N, K):
     return lib().w4a16_gemm_path(fmt, M, N, K)
 
@@ -221,6 +239,30 @@ def gate_up_silu(fmt: str, x, packed_w, packed_scales, I: int, global_scale=None
     check(w4a16_gemm_gate_up_silu_ex(path, FMTS[fmt], M, I, K, x, packed_w, packed_scales,
                                      global_scale, h, stream), "w4a16_gemm_gate_up_silu")
     return h
+
+
+def quantize_act_nvfp4(x, stream=None):
+    """NVFP4 activation quantiser on a BF16 CUDA tensor x [M][K]: returns
+    (codes uint8 [M][K], E4M3 scales uint8 [M][K/16], g_x fp32 [1])."""
+    import torch
+    M, K = x.shape
+    codes = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
+    g_x = torch.empty(1, dtype=torch.float32, device=x.device)
+    check(w4a16_quantize_act_nvfp4(M, K, x, codes, scales, g_x, stream), "w4a16_quantize_act_nvfp4")
+    return codes, scales, g_x
+
+
+def gemm_w4a4(x, packed_w, packed_scales, N: int, global_scale_w, y=None, path=PATH_AUTO,
+              stream=None):
+    """W4A4 NVFP4 matmul of a BF16 CUDA tensor x [M][K]; returns y (BF16 [M][N])."""
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    check(w4a16_gemm_w4a4_ex(path, M, N, K, x, packed_w, packed_scales, global_scale_w, y, stream),
+          "w4a16_gemm_w4a4")
+    return y
 
 
 def dequant(fmt: str, N: int, K: int, packed_w, packed_scales, global_scale=None, out=None,

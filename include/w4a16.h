@@ -202,6 +202,44 @@ int w4a16_gemm_noalloc(int fmt, int M, int N, int K, const void* x_bf16, const v
                        const void* packed_scales, const float* global_scale, void* y_bf16,
                        void* stream);
 
+/*
+ * W4A4 NVFP4: the activations quantised to NVFP4 as well (model card
+ * "SuperQwen3.8-27b-abliterated-NVFP4-2xDGX", table "Release highlights":
+ * W4A4 NVFP4, group size 16).  The pages name only the format; the reading
+ * taken, every step in fp32 with round-to-nearest:
+ *   g_x = amax|x| / (6 * 448)                 (1.0 for an all-zero x)
+ *   s[m][j] = RNE_e4m3(amax_{k in 16-block j}|x[m][k]| / (6 * g_x)), saturating at 448
+ *   q[m][k] = RNE_e2m1(x[m][k] / (e4m3(s[m][k/16]) * g_x)), ties to the even code,
+ *             saturating at +-6 (0 when the scale is 0)
+ *
+ * Quantiser alone: x_bf16 [M][K] (device, 16-byte aligned, K a multiple of
+ * 128, 1 <= M <= 8192) -> codes (device, [M][K] bytes, one E2M1 code in the
+ * low 4 bits of each, 16-byte aligned), scales (device, [M][K/16] E4M3
+ * bytes), g_x (device, one fp32).  Asynchronous on `stream`.
+ */
+int w4a16_quantize_act_nvfp4(int M, int K, const void* x_bf16, void* codes, void* scales,
+                             float* g_x, void* stream);
+
+/*
+ * The W4A4 matmul: y[M][N] = BF16(sum_k x_hat[m][k] * W[n][k]) with
+ * x_hat = e2m1(q) * e4m3(s) * g_x (the quantiser above, run inside the call)
+ * and W the NVFP4 weights at their exact values e2m1 * e4m3 * g_w.
+ *   x_bf16, y_bf16: as for w4a16_gemm.  packed_w, packed_scales: NVFP4
+ *   weights packed as for w4a16_gemm (W4A16_FMT_NVFP4_G16).  global_scale_w:
+ *   device pointer to the weights' fp32 g_w.
+ * Accuracy: |y - y_ref| <= 2^-7 * sum_k |x_hat W| + 1e-3 against the exact
+ * W4A4 product.  The library keeps a scratch per (device, stream) for the
+ * quantised activations (M x K BF16), allocated like the matmul workspace.
+ */
+int w4a16_gemm_w4a4(int M, int N, int K, const void* x_bf16, const void* packed_w,
+                    const void* packed_scales, const float* global_scale_w, void* y_bf16,
+                    void* stream);
+
+/* Same as w4a16_gemm_w4a4 with an explicit path (W4A16_PATH_*). */
+int w4a16_gemm_w4a4_ex(int path, int M, int N, int K, const void* x_bf16, const void* packed_w,
+                       const void* packed_scales, const float* global_scale_w, void* y_bf16,
+                       void* stream);
+
 /* The path W4A16_PATH_AUTO would take for these arguments (>0), or a status. */
 int w4a16_gemm_path(int fmt, int M, int N, int K);
 
