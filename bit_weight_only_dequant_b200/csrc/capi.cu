@@ -272,8 +272,8 @@ int w4a16_dequant(int fmt, int N, int K, const void* packed_w, const void* packe
                                       static_cast<cudaStream_t>(stream)));
 }
 
-// W4A4: scratch of its own per (device, stream) -- [amax word, g_x, g_eff,
-// pad to 256 B][block-scaled activations BF16 M x K] -- so that the matmul's
+// W4A4: scratch of its own per (device, stream) -- [amax word, arrival
+// counter, g_eff, pad to 256 B][block-scaled activations BF16 M x K] -- so that the matmul's
 // own workspace can grow without freeing memory this call still reads.
 std::map<std::pair<int, cudaStream_t>, Workspace> g_w4a4_ws;
 
@@ -287,6 +287,8 @@ int w4a4_scratch(cudaStream_t st, size_t bytes, uint8_t** out) {
     nb = (nb + 255) / 256 * 256;
     void* base = nullptr;
     if (cudaMallocAsync(&base, nb, st) != cudaSuccess) return W4A16_ERR_NOMEM;
+    // the quantiser's amax word and arrival counter start (and are left) zero
+    if (cudaMemsetAsync(base, 0, 256, st) != cudaSuccess) return W4A16_ERR_CUDA;
     if (w.base) cudaFreeAsync(w.base, st);
     w.base = base;
     w.bytes = nb;

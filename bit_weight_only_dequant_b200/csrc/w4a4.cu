@@ -32,9 +32,13 @@ namespace w4 {
 namespace {
 
 // Largest |x| of the tensor as the fp32 bits of a BF16 value (magnitude bits
-// compared as integers, which order like the values).  amax_bits must be zero.
+// compared as integers, which order like the values).  amax_bits is zero on
+// entry: the quantiser kernel of the previous call cleared it.  Launched with
+// programmatic dependent launch: x may come from the previous kernel.
 __global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __restrict__ x,
                                                        long long n8, unsigned* amax_bits) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint4* v = reinterpret_cast<const uint4*>(x);
   uint32_t mx = 0u;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
@@ -98,24 +102,14 @@ __device__ __forceinline__ float global_scale(unsigned amax_bits) {
   return amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f;   // 6 * 448 = 2688 exactly
 }
 
-// One thread per (row, 16-block): codes (one per byte, [M][K]), the E4M3
-// scale ([M][K/16]) and the block-scaled values e2m1 * e4m3 as BF16 ([M][K]),
-// each output optional.  Thread 0 also writes g_x and, if g_w is given,
-// g_w * g_x (fp32, one rounding): the matmul's per-tensor scale.
-__global__ void __launch_bounds__(256)
-    act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
-                     const unsigned* __restrict__ amax_bits, const float* __restrict__ g_w,
-                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                     __nv_bfloat16* __restrict__ xq, float* g_x_out, float* g_eff_out) {
-  const float g = global_scale(__ldg(amax_bits));
-  const long long nblk = (long long)M * (K >> 4);
-  const long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (b == 0) {
-    if (g_x_out) *g_x_out = g;
-    if (g_eff_out) *g_eff_out = g_w ? __fmul_rn(__ldg(g_w), g) : g;
-  }
+// Quantise the 16-block b (row b / (K/16)): codes (one per byte, [M][K]),
+// the E4M3 scale ([M][K/16]) and the block-scaled values e2m1 * e4m3 as BF16
+// ([M][K]), each output optional.
+__device__ __forceinline__ void quantize_block(const __nv_bfloat16* __restrict__ x, long long b,
+                                               long long nblk, float g, uint8_t* codes,
+                                               uint8_t* scales, __nv_bfloat16* xq) {
   if (b >= nblk) return;
-  const uint4* src = reinterpret_cast<const uint4*>(x) + 2 * b;
+  const uint4* src = reinterpret_cast<const uint4*>(x) + 2 * b;   // the block's 16 values
   const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
   const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   float v[16];
@@ -158,22 +152,64 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// One thread per (row, 16-block).  Thread 0 also writes g_x and, if g_w is
+// given, g_w * g_x (fp32, one rounding): the matmul's per-tensor scale.
+// Launched behind act_amax_kernel with programmatic dependent launch; the
+// last CTA to finish clears amax_bits[0] and its arrival counter
+// amax_bits[1] for the next call.
+__global__ void __launch_bounds__(256)
+    act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, unsigned* amax_bits,
+                     const float* __restrict__ g_w, uint8_t* __restrict__ codes,
+                     uint8_t* __restrict__ scales, __nv_bfloat16* __restrict__ xq,
+                     float* g_x_out, float* g_eff_out) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float g = global_scale(*reinterpret_cast<volatile unsigned*>(amax_bits));
+  const long long nblk = (long long)M * (K >> 4);
+  const long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (b == 0) {
+    if (g_x_out) *g_x_out = g;
+    if (g_eff_out) *g_eff_out = g_w ? __fmul_rn(__ldg(g_w), g) : g;
+  }
+  quantize_block(x, b, nblk, g, codes, scales, xq);
+  // every thread of this CTA has read amax_bits: the last CTA clears it
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    unsigned* done = amax_bits + 1;
+    if (atomicAdd(done, 1u) == gridDim.x - 1) {
+      amax_bits[0] = 0u;
+      *done = 0u;
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_act_quant(int M, int K, const void* x, unsigned* amax_bits, const float* g_w,
                              void* codes, void* scales, void* xq, float* g_x, float* g_eff,
                              cudaStream_t st) {
-  cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(unsigned), st);
-  if (e != cudaSuccess) return e;
+  // amax_bits[0..1] are zero between calls (zeroed once when the scratch is
+  // allocated, cleared again by the last quantiser CTA of every call)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   const long long n8 = (long long)M * K / 8;
-  const int grid_a = (int)min(1184ll, (n8 + 255) / 256);
-  act_amax_kernel<<<grid_a, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), n8, amax_bits);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  cfg.gridDim = dim3((unsigned)min(1184ll, (n8 + 255) / 256), 1, 1);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, act_amax_kernel, static_cast<const __nv_bfloat16*>(x),
+                                     n8, amax_bits);
+  if (e != cudaSuccess) return e;
   const long long nblk = (long long)M * (K / 16);
-  act_quant_kernel<<<(unsigned)((nblk + 255) / 256), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), M, K, amax_bits, g_w, static_cast<uint8_t*>(codes),
-      static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xq), g_x, g_eff);
-  return cudaGetLastError();
+  cfg.gridDim = dim3((unsigned)((nblk + 255) / 256), 1, 1);
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel, static_cast<const __nv_bfloat16*>(x), M, K,
+                            amax_bits, g_w, static_cast<uint8_t*>(codes),
+                            static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xq), g_x,
+                            g_eff);
 }
 
 }  // namespace w4
