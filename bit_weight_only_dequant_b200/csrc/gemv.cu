@@ -575,9 +575,8 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
   }
 
   pdl_wait();          // the operands may come from the previous kernel
-#pragma unroll
-  for (int k = 0; k < D; ++k) copy_item(k);
-  __syncthreads();     // row_aux zeroed, xbar initialised
+  // the activation copy goes out first (warp 0 initialised its barrier), then
+  // the first block of the weight ring
   if (warp == 0) {
     if (lane == 0) mbar_arrive_expect_tx(xbar, x_bytes * p.M);
     __syncwarp();
@@ -585,6 +584,9 @@ __global__ void __launch_bounds__(Cfg<FMT, MT, FUSE>::kWarps * 32, 1) gemv_kerne
       bulk_g2s(smem_u32(xs + lane * p.row_stride), p.x + (size_t)lane * p.K + k_lo, x_bytes,
                smem_u32(xbar));
   }
+#pragma unroll
+  for (int k = 0; k < D; ++k) copy_item(k);
+  __syncthreads();     // row_aux zeroed
   const bool x_ok = stage_activations(p, groups * 128, xs, row_mul, row_aux, xbar);
   next_block();
 
