@@ -11,8 +11,9 @@ bytes (packed weights + scales + activations + outputs) per second over the
 timed steps, aggregated over all GPUs.  The other configurations (every row
 count, NVFP4, the 64-layer sweep) and the widened rows (M up to 2048, FP8
 weights, the fused gate/up layer) are reported in ``sweep``, ``gate_up_silu``
-and ``whole_stack``.  ``--case fmt,M,N,K[,path]`` launches one GEMM a few
-times for a profiler.
+and ``whole_stack``.  ``--case fmt,M,N,K[,path][;...]`` launches GEMMs a few
+times for a profiler; ``--traffic-csv`` turns an ncu capture of the decode
+shapes into profiles/traffic.json.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 Multi-GPU: launched by torchrun, one process per GPU; each GPU runs its own
@@ -350,7 +351,7 @@ def make_weights(fmt, seed, N, K, copies):
     import torch
     import synth
     from bit_weight_only_dequant_b200 import w4a16 as W
-    p = synth.device_problem(fmt, seed, 1, N, K)
+    p = synth.device_problem("nvfp4" if fmt == "nvfp4_bs" else fmt, seed, 1, N, K)
     pw, ps = W.pack_on_device(fmt, N, K, p["codes"], p["scales"])
     del p
     ws = [(pw, ps)]
@@ -448,22 +449,29 @@ def sweep_entry(fmt, name, K, N, M, seed, peaks, stream, reps=24):
             "frac_of_8TBps": round(b / us / 1e3 / 8000.0, 4)}
 
 
-def w4a4_entry(name, K, N, M, seed, peaks, stream, reps=24):
+def w4a4_entry(name, K, N, M, seed, peaks, stream, reps=24, block_scaled=False):
     """W4A4 NVFP4 (activations quantised inside the call) at one decode shape:
     the quantiser and the matmul, back to back like the sweep.  Algorithmic
-    bytes: the NVFP4 weights and scales, x and y."""
+    bytes: the NVFP4 weights and scales, x and y.  block_scaled: the
+    tcgen05 kind::mxf4nvf4 path (weights in its own layout, same bytes);
+    its tensor roofline is the FP4 peak (the measured BF16 peak times the
+    nominal 4x ratio)."""
     import torch
     from bit_weight_only_dequant_b200 import w4a16 as W
-    f = W.FMTS["nvfp4"]
+    wfmt = "nvfp4_bs" if block_scaled else "nvfp4"
+    f = W.FMTS[wfmt]
     wbytes = W.w4a16_packed_weight_bytes(f, N, K) + W.w4a16_packed_scale_bytes(f, N, K)
-    ws = make_weights("nvfp4", seed, N, K, copies_for(wbytes))
+    ws = make_weights(wfmt, seed, N, K, copies_for(wbytes))
     x = make_x("nvfp4", seed, M, K)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda")
 
     def launch(r, ws=ws):
         pw, ps = ws[r % len(ws)]
-        W.check(W.w4a16_gemm_w4a4(M, N, K, x, pw, ps, g, y, stream.cuda_stream), "gemm_w4a4")
+        if block_scaled:
+            W.check(W.w4a16_gemm_w4a4_bs(M, N, K, x, pw, ps, g, y, stream.cuda_stream), "gemm_w4a4_bs")
+        else:
+            W.check(W.w4a16_gemm_w4a4(M, N, K, x, pw, ps, g, y, stream.cuda_stream), "gemm_w4a4")
 
     with torch.cuda.stream(stream):
         for r in range(3):
@@ -473,11 +481,13 @@ def w4a4_entry(name, K, N, M, seed, peaks, stream, reps=24):
     us = rep["median"]
     b = alg_bytes("nvfp4", M, N, K)
     fl = flops(M, N, K)
-    t_roof = max(b / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+    tpeak = peaks["bf16_tflops"] * (4.0 if block_scaled else 1.0)
+    t_roof = max(b / (peaks["hbm_gbs"] * 1e9), fl / (tpeak * 1e12))
     del ws
     torch.cuda.empty_cache()
-    return {"fmt": "w4a4_nvfp4", "shape": name, "K": K, "N": N, "M": M,
-            "path": int(W.w4a16_gemm_path(f, M, N, K)), "us": round(us, 3),
+    path = W.PATH_BS if block_scaled else int(W.w4a16_gemm_path(W.FMTS["nvfp4"], M, N, K))
+    return {"fmt": "w4a4_nvfp4_bs" if block_scaled else "w4a4_nvfp4", "shape": name, "K": K, "N": N,
+            "M": M, "path": path, "us": round(us, 3),
             "us_min": round(rep["min"], 3), "us_max": round(rep["max"], 3),
             "GBps": round(b / us / 1e3, 1), "frac_roofline": round(t_roof * 1e6 / us, 4)}
 
@@ -736,6 +746,8 @@ def run_native(args, rank, world, local_rank):
         for fmt, n, K, N, Mv, s in target + cfg2 + cfg3 + cfg4 + cfg5:
             entries.append(sweep_entry(fmt, n, K, N, Mv, s, peaks, stream))
         extra["sweep"] = entries
+        extra["w4a4_block_scaled"] = [w4a4_entry(n, K, N, Mv, 6, peaks, stream, block_scaled=True)
+                                      for Mv in (1, 9, 64) for n, K, N, _ in DECODE_SHAPES]
         extra["w4a4"] = [w4a4_entry(n, K, N, Mv, 6, peaks, stream) for Mv in (1, 9, 64)
                          for n, K, N, _ in DECODE_SHAPES]
         extra["gate_up_silu"] = [gate_up_entry(fmt, Mv, 3, peaks, stream)
@@ -778,25 +790,91 @@ def run_native(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
-def run_case(spec: str, launches: int):
-    """Launch one GEMM a few times (for profilers): spec = fmt,M,N,K[,path]."""
+def run_case(specs: str, launches: int):
+    """Launch GEMMs a few times each (for profilers).  specs = one or more
+    fmt,M,N,K[,path] separated by ';', run in that order; fmt is int4, nvfp4,
+    fp8 or w4a4 (NVFP4 weights, activations quantised by the library)."""
     import torch
     from bit_weight_only_dequant_b200 import w4a16 as W
-    parts = spec.split(",")
-    fmt, M, N, K = parts[0], int(parts[1]), int(parts[2]), int(parts[3])
-    path = int(parts[4]) if len(parts) > 4 else W.PATH_AUTO
     torch.cuda.set_device(0)
-    f = W.FMTS[fmt]
-    (pw, ps), = make_weights(fmt, 3, N, K, 1)
-    x = make_x(fmt, 3, M, K)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if fmt != "int4" else None
-    for _ in range(launches):
-        W.check(W.w4a16_gemm_ex(path, f, M, N, K, x, pw, ps, g, y), "gemm")
-    torch.cuda.synchronize()
-    W.check(W.w4a16_device_status(), "device status")
-    print(json.dumps({"case": spec, "launches": launches, "path": W.w4a16_gemm_path(f, M, N, K)
-                      if path == W.PATH_AUTO else path}))
+    out = []
+    for spec in specs.split(";"):
+        parts = spec.split(",")
+        fmt, M, N, K = parts[0], int(parts[1]), int(parts[2]), int(parts[3])
+        path = int(parts[4]) if len(parts) > 4 else W.PATH_AUTO
+        wfmt = "nvfp4" if fmt == "w4a4" else fmt
+        f = W.FMTS[wfmt]
+        (pw, ps), = make_weights(wfmt, 3, N, K, 1)
+        x = make_x(wfmt, 3, M, K)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if wfmt != "int4" else None
+        for _ in range(launches):
+            if fmt == "w4a4":
+                W.check(W.w4a16_gemm_w4a4_ex(path, M, N, K, x, pw, ps, g, y), "gemm_w4a4")
+            else:
+                W.check(W.w4a16_gemm_ex(path, f, M, N, K, x, pw, ps, g, y), "gemm")
+        torch.cuda.synchronize()
+        W.check(W.w4a16_device_status(), "device status")
+        out.append({"case": spec, "launches": launches,
+                    "path": W.w4a16_gemm_path(f, M, N, K) if path == W.PATH_AUTO else path})
+        del pw, ps, x, y
+        torch.cuda.empty_cache()
+    print(json.dumps(out))
+
+
+TRAFFIC_SPECS = ";".join(f"int4,1,{N},{K},1" for _, K, N, _ in DECODE_SHAPES)
+
+
+def _ncu_value(value: str, unit: str) -> float:
+    v = float(value.replace(",", ""))
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "nsecond": 1, "ns": 1,
+             "usecond": 1e3, "us": 1e3, "msecond": 1e6, "ms": 1e6}
+    if unit not in scale:
+        raise ValueError(f"unexpected ncu unit {unit!r}")
+    return v * scale[unit]
+
+
+def write_traffic(csv_path: str, launches: int, out_path=None):
+    """profiles/traffic.json from one ncu CSV of the GEMV over the four decode
+    shapes at M = 1 (``--case`` with TRAFFIC_SPECS, ``launches`` per shape, all
+    captured): per shape the last launch's DRAM bytes, stamped with the hash of
+    the GEMV's sources as they are now."""
+    import csv
+    rows = {}
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    for r in csv.DictReader(lines):
+        if "gemv" not in r["Kernel Name"]:
+            continue
+        rows.setdefault(int(r["ID"]), {})[r["Metric Name"]] = _ncu_value(r["Metric Value"],
+                                                                          r["Metric Unit"])
+    ids = sorted(rows)
+    if len(ids) != launches * len(DECODE_SHAPES):
+        raise SystemExit(f"expected {launches * len(DECODE_SHAPES)} GEMV launches, found {len(ids)}")
+    per_shape, total, alg = {}, 0.0, 0
+    for i, (name, K, N, _) in enumerate(DECODE_SHAPES):
+        m = rows[ids[(i + 1) * launches - 1]]
+        rd, wr = m["dram__bytes_read.sum"], m["dram__bytes_write.sum"]
+        a = int(alg_bytes("int4", 1, N, K))
+        per_shape[f"{name} {K}->{N}"] = {"dram_read": int(rd), "dram_write": int(wr), "algorithmic": a,
+                                         "ncu_duration_ns": int(m["gpu__time_duration.sum"])}
+        total += rd + wr
+        alg += a
+    n = len(DECODE_SHAPES)
+    d = {"kernel": "gemv_kernel<int4, 1 m-tile> (the four launches of the decode step at M=1)",
+         "dram_bytes_per_launch": int(round(total / n)), "algorithmic_bytes_per_launch": alg // n,
+         "per_shape": per_shape,
+         "metrics": "dram__bytes_read.sum + dram__bytes_write.sum of the last captured launch per shape",
+         "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                     "--clock-control none --print-units base -k regex:gemv --csv --log-file CSV "
+                     f"python bench.py --case '{TRAFFIC_SPECS}' --launches {launches}; then "
+                     f"python bench.py --traffic-csv CSV --launches {launches}"),
+         "source_hash": kernel_source_hash()}
+    with open(out_path or os.path.join(ROOT, "profiles", "traffic.json"), "w") as f:
+        json.dump(d, f, indent=1)
+        f.write("\n")
+    print(json.dumps({"dram_bytes_per_launch": d["dram_bytes_per_launch"],
+                      "algorithmic_bytes_per_launch": d["algorithmic_bytes_per_launch"]}))
 
 
 def main():
@@ -811,9 +889,14 @@ def main():
     ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-cpu-all", action="store_true", help="skip the all-cores oracle timing")
     ap.add_argument("--case", default=None,
-                    help="profiling mode: launch one GEMM fmt,M,N,K[,path] --launches times")
+                    help="profiling mode: launch GEMMs fmt,M,N,K[,path][;...] --launches times each")
     ap.add_argument("--launches", type=int, default=5)
+    ap.add_argument("--traffic-csv", default=None,
+                    help="write profiles/traffic.json from an ncu CSV of --case over the decode shapes")
     args = ap.parse_args()
+    if args.traffic_csv:
+        write_traffic(args.traffic_csv, args.launches)
+        return
     if args.case:
         run_case(args.case, args.launches)
         return

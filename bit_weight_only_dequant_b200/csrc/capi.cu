@@ -5,6 +5,7 @@
 #include <utility>
 
 #include "../../include/w4a16.h"
+#include "bs.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -125,8 +126,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool has_global_scale(int fmt) { return fmt != W4A16_FMT_INT4_G128; }
 bool has_packed_scales(int fmt) { return fmt != W4A16_FMT_FP8_E4M3; }
 
-int check_fmt_shape(int fmt, int N, int K) {
-  if (fmt != W4A16_FMT_INT4_G128 && fmt != W4A16_FMT_NVFP4_G16 && fmt != W4A16_FMT_FP8_E4M3)
+// allow_bs: the block-scaled W4A4 weight layout (packers, sizes, its matmul)
+int check_fmt_shape(int fmt, int N, int K, bool allow_bs = false) {
+  if (fmt != W4A16_FMT_INT4_G128 && fmt != W4A16_FMT_NVFP4_G16 && fmt != W4A16_FMT_FP8_E4M3 &&
+      !(allow_bs && fmt == W4A16_FMT_NVFP4_BS))
     return W4A16_ERR_ARG;
   if (N < 1 || K < 128 || K % 128 != 0) return W4A16_ERR_SHAPE;
   // packed tensors are addressed with 32-bit tile/scale indices in places
@@ -213,38 +216,46 @@ int run_gemm(int path, int fmt, int M, int N, int K, const void* x_bf16, const v
 extern "C" {
 
 size_t w4a16_packed_weight_bytes(int fmt, int N, int K) {
-  if (check_fmt_shape(fmt, N, K) != W4A16_OK) return 0;
+  if (check_fmt_shape(fmt, N, K, true) != W4A16_OK) return 0;
+  if (fmt == W4A16_FMT_NVFP4_BS) return (size_t)w4::bs_weight_bytes(N, K);
   return (size_t)w4::weight_bytes(fmt, N, K);
 }
 
 size_t w4a16_packed_scale_bytes(int fmt, int N, int K) {
-  if (check_fmt_shape(fmt, N, K) != W4A16_OK) return 0;
+  if (check_fmt_shape(fmt, N, K, true) != W4A16_OK) return 0;
+  if (fmt == W4A16_FMT_NVFP4_BS) return (size_t)w4::bs_scale_bytes(N, K);
   return (size_t)w4::scale_bytes(fmt, N, K);
 }
 
 int w4a16_pack_host(int fmt, int N, int K, const void* codes, const void* scales, void* packed_w,
                     void* packed_scales) {
-  const int r = check_fmt_shape(fmt, N, K);
+  const int r = check_fmt_shape(fmt, N, K, true);
   if (r != W4A16_OK) return r;
   if (!codes || !packed_w || (has_packed_scales(fmt) && (!scales || !packed_scales)))
     return W4A16_ERR_ARG;
+  if (fmt == W4A16_FMT_NVFP4_BS)
+    return w4::pack_host_bs(N, K, codes, scales, packed_w, packed_scales) == 0 ? W4A16_OK
+                                                                              : W4A16_ERR_ARG;
   return w4::pack_host(fmt, N, K, codes, scales, packed_w, packed_scales) == 0 ? W4A16_OK
                                                                                : W4A16_ERR_ARG;
 }
 
 int w4a16_unpack_host(int fmt, int N, int K, const void* packed_w, const void* packed_scales,
                       void* codes, void* scales) {
-  const int r = check_fmt_shape(fmt, N, K);
+  const int r = check_fmt_shape(fmt, N, K, true);
   if (r != W4A16_OK) return r;
   if (!codes || !packed_w || (has_packed_scales(fmt) && (!scales || !packed_scales)))
     return W4A16_ERR_ARG;
+  if (fmt == W4A16_FMT_NVFP4_BS)
+    return w4::unpack_host_bs(N, K, packed_w, packed_scales, codes, scales) == 0 ? W4A16_OK
+                                                                                : W4A16_ERR_ARG;
   return w4::unpack_host(fmt, N, K, packed_w, packed_scales, codes, scales) == 0 ? W4A16_OK
                                                                                  : W4A16_ERR_ARG;
 }
 
 int w4a16_pack(int fmt, int N, int K, const void* codes, const void* scales, void* packed_w,
                void* packed_scales, void* stream) {
-  int r = check_fmt_shape(fmt, N, K);
+  int r = check_fmt_shape(fmt, N, K, true);
   if (r != W4A16_OK) return r;
   if (!codes || !packed_w || (has_packed_scales(fmt) && (!scales || !packed_scales)))
     return W4A16_ERR_ARG;
@@ -253,6 +264,9 @@ int w4a16_pack(int fmt, int N, int K, const void* codes, const void* scales, voi
     return W4A16_ERR_ALIGN;
   DeviceState* d = nullptr;
   if ((r = device_state(&d)) != W4A16_OK) return r;
+  if (fmt == W4A16_FMT_NVFP4_BS)
+    return status_of(w4::launch_pack_bs(N, K, codes, scales, packed_w, packed_scales,
+                                        static_cast<cudaStream_t>(stream)));
   return status_of(w4::launch_pack(fmt, N, K, codes, scales, packed_w, packed_scales,
                                    static_cast<cudaStream_t>(stream)));
 }
@@ -383,12 +397,60 @@ int w4a16_gemm_w4a4(int M, int N, int K, const void* x_bf16, const void* packed_
                             global_scale_w, y_bf16, stream);
 }
 
+// Block-scaled W4A4: the quantiser writes the activation operands in the
+// tensor cores' layout (codes [M][K/2], scale atoms per chunk), then the
+// block-scaled matmul streams both.  Scratch: [amax word, arrival counter,
+// g_eff, pad to 256 B][codes M x K/2][scale atoms chunks x K/64 x 512].
+int w4a16_gemm_w4a4_bs(int M, int N, int K, const void* x_bf16, const void* packed_w,
+                       const void* packed_sf, const float* global_scale_w, void* y_bf16,
+                       void* stream) {
+  int r = check_fmt_shape(W4A16_FMT_NVFP4_BS, N, K, true);
+  if (r != W4A16_OK) return r;
+  if (M < 1 || M > W4A16_MAX_M) return W4A16_ERR_SHAPE;
+  if (!x_bf16 || !packed_w || !packed_sf || !global_scale_w || !y_bf16) return W4A16_ERR_ARG;
+  if (!aligned16(x_bf16) || !aligned16(packed_w) || !aligned16(packed_sf) || !aligned16(y_bf16))
+    return W4A16_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if ((r = device_state(&d)) != W4A16_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const w4::BsPlan pl = w4::plan_bs(M, N, K, d->num_sms);
+  if (pl.S == 0) return W4A16_ERR_SHAPE;
+  const size_t xc_bytes = ((size_t)M * K / 2 + 255) / 256 * 256;
+  const size_t xsf_bytes = (size_t)pl.chunks * (K / 64) * w4::kBsAtomBytes;
+  uint8_t* scratch = nullptr;
+  if ((r = w4a4_scratch(st, 256 + xc_bytes + xsf_bytes, &scratch)) != W4A16_OK) return r;
+  unsigned* amax = reinterpret_cast<unsigned*>(scratch);
+  float* g_eff = reinterpret_cast<float*>(scratch + 8);
+  uint8_t* xc = scratch + 256;
+  uint8_t* xsf = xc + xc_bytes;
+  float* ws = nullptr;
+  const size_t nf = w4::bs_workspace_floats(pl, M);
+  if (nf > 0) {
+    unsigned* cnt = nullptr;
+    void* unused = nullptr;
+    if ((r = workspace(st, 0, nf, 0, &cnt, &ws, &unused)) != W4A16_OK) return r;
+  }
+  cudaError_t e = w4::launch_act_quant_bs(M, K, pl.rows, x_bf16, amax, global_scale_w, xc, xsf,
+                                          nullptr, g_eff, st);
+  if (e != cudaSuccess) return W4A16_ERR_CUDA;
+  return status_of(w4::launch_bs(pl, M, N, K, packed_w, packed_sf, xc, xsf, g_eff, y_bf16, ws,
+                                 d->err, st));
+}
+
 int w4a16_plan(int path, int fmt, int M, int N, int K, int fuse, int num_sms, int* out,
                int out_len) {
   if (fuse != 0 && fuse != 1) return W4A16_ERR_ARG;
-  const int r = check_fmt_shape(fmt, N, K);
+  const int r = check_fmt_shape(fmt, N, K, path == W4A16_PATH_BS);
   if (r != W4A16_OK) return r;
   if (M < 1 || M > W4A16_MAX_M || num_sms < 1 || !out || out_len < 9) return W4A16_ERR_ARG;
+  if (path == W4A16_PATH_BS) {
+    if (fmt != W4A16_FMT_NVFP4_BS || fuse) return W4A16_ERR_ARG;
+    const w4::BsPlan pl = w4::plan_bs(M, N, K, num_sms);
+    const int v[9] = {pl.tiles, pl.chunks, pl.rows, pl.mpad, pl.S, pl.sps, pl.units, pl.grid, pl.smem};
+    for (int i = 0; i < 9; ++i) out[i] = v[i];
+    return pl.S == 0 ? W4A16_ERR_SHAPE : W4A16_PATH_BS;
+  }
+  if (fmt == W4A16_FMT_NVFP4_BS) return W4A16_ERR_ARG;
   if (fuse && (N % 32 != 0)) return W4A16_ERR_SHAPE;
   if (path == W4A16_PATH_AUTO) path = choose_path(fmt, M, N, K);
   if (path == W4A16_PATH_GEMV) {

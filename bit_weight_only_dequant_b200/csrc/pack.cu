@@ -3,6 +3,7 @@
 // version for packing large matrices where they already live.
 #include <string.h>
 
+#include "bs.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -223,6 +224,86 @@ cudaError_t launch_pack(int fmt, int N, int K, const void* codes, const void* sc
     pack_weights_kernel<1><<<bw, 256, 0, st>>>(N, K, (const uint8_t*)codes, (uint8_t*)w);
     pack_scales_kernel<1><<<bs, 256, 0, st>>>(N, K, (const uint8_t*)scales, (uint8_t*)s);
   }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- block-scaled W4A4 layout
+
+int pack_host_bs(int N, int K, const void* codes_v, const void* scales_v, void* w_v, void* s_v) {
+  const uint8_t* c = static_cast<const uint8_t*>(codes_v);
+  const uint8_t* sc = static_cast<const uint8_t*>(scales_v);
+  uint8_t* w = static_cast<uint8_t*>(w_v);
+  uint8_t* s = static_cast<uint8_t*>(s_v);
+  memset(s, 0, (size_t)bs_scale_bytes(N, K));
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < K / 2; ++j) {
+      const uint8_t lo = c[n * K + 2 * j], hi = c[n * K + 2 * j + 1];
+      if (lo > 15 || hi > 15) return -1;
+      w[n * (K / 2) + j] = static_cast<uint8_t>(lo | (hi << 4));
+    }
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t gi = 0; gi < K / kNvfp4Group; ++gi) {
+      const uint8_t b = sc[n * (K / kNvfp4Group) + gi];
+      if ((b & 0x7Fu) == 0x7Fu) return -1;  // E4M3 NaN
+      s[bs_scale_offset(n / kBsTileRows, (int)(n % kBsTileRows), gi, K)] = b;
+    }
+  return 0;
+}
+
+int unpack_host_bs(int N, int K, const void* w_v, const void* s_v, void* codes_v, void* scales_v) {
+  const uint8_t* w = static_cast<const uint8_t*>(w_v);
+  const uint8_t* s = static_cast<const uint8_t*>(s_v);
+  uint8_t* c = static_cast<uint8_t*>(codes_v);
+  uint8_t* sc = static_cast<uint8_t*>(scales_v);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < K / 2; ++j) {
+      const uint8_t b = w[n * (K / 2) + j];
+      c[n * K + 2 * j] = b & 15u;
+      c[n * K + 2 * j + 1] = b >> 4;
+    }
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t gi = 0; gi < K / kNvfp4Group; ++gi)
+      sc[n * (K / kNvfp4Group) + gi] = s[bs_scale_offset(n / kBsTileRows, (int)(n % kBsTileRows), gi, K)];
+  return 0;
+}
+
+namespace {
+
+// One thread per (row, 16-block) of the padded rows: 8 bytes of codes (rows
+// below N) and the block's scale byte (0 past N).
+__global__ void pack_bs_kernel(int N, int K, const uint8_t* __restrict__ codes,
+                               const uint8_t* __restrict__ scales, uint8_t* __restrict__ w,
+                               uint8_t* __restrict__ s) {
+  const int G = K / kNvfp4Group;
+  const long long total = bs_tiles(N) * kBsTileRows * G;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long n = idx / G;
+    const long long gi = idx - n * G;
+    uint8_t sv = 0;
+    if (n < N) {
+      const uint4 v = *reinterpret_cast<const uint4*>(codes + n * K + 16 * gi);
+      const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+      uint32_t out[2] = {0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        out[j >> 3] |= ((in[j >> 2] >> (8 * (j & 3))) & 15u) << (4 * (j & 7));
+      *reinterpret_cast<uint2*>(w + n * (K / 2) + 8 * gi) = make_uint2(out[0], out[1]);
+      sv = scales[n * G + gi];
+    }
+    s[bs_scale_offset(n / kBsTileRows, (int)(n % kBsTileRows), gi, K)] = sv;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_bs(int N, int K, const void* codes, const void* scales, void* w, void* s,
+                           cudaStream_t st) {
+  const long long total = bs_tiles(N) * kBsTileRows * (K / kNvfp4Group);
+  const unsigned blocks = (unsigned)((total + 255) / 256 < 148 * 32 ? (total + 255) / 256 : 148 * 32);
+  pack_bs_kernel<<<blocks, 256, 0, st>>>(N, K, static_cast<const uint8_t*>(codes),
+                                         static_cast<const uint8_t*>(scales),
+                                         static_cast<uint8_t*>(w), static_cast<uint8_t*>(s));
   return cudaGetLastError();
 }
 

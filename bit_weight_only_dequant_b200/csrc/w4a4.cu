@@ -24,6 +24,7 @@
 // library on the block-scaled activation values: at decode and verify row
 // counts W4A4 moves the same weight bytes as W4A16, so the same kernels bound
 // it.
+#include "bs.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -102,12 +103,25 @@ __device__ __forceinline__ float global_scale(unsigned amax_bits) {
   return amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f;   // 6 * 448 = 2688 exactly
 }
 
-// Quantise the 16-block b (row b / (K/16)): codes (one per byte, [M][K]),
-// the E4M3 scale ([M][K/16]) and the block-scaled values e2m1 * e4m3 as BF16
-// ([M][K]), each output optional.
+// Outputs of the quantiser, each optional.  codes: one per byte [M][K];
+// scales: E4M3 [M][K/16]; xq: the block-scaled values e2m1 * e4m3 as BF16
+// [M][K]; xc / xsf: the block-scaled tensor-core operand layouts (codes two
+// per byte [M][K/2], scale atoms per chunk of `rows` rows, layout_bs.h).
+struct QuantOut {
+  uint8_t* codes;
+  uint8_t* scales;
+  __nv_bfloat16* xq;
+  uint8_t* xc;
+  uint8_t* xsf;
+  int rows;
+};
+
+// Quantise the 16-block b (row b / (K/16)).
 __device__ __forceinline__ void quantize_block(const __nv_bfloat16* __restrict__ x, long long b,
-                                               long long nblk, float g, uint8_t* codes,
-                                               uint8_t* scales, __nv_bfloat16* xq) {
+                                               long long nblk, int K, float g, const QuantOut& o) {
+  uint8_t* codes = o.codes;
+  uint8_t* scales = o.scales;
+  __nv_bfloat16* xq = o.xq;
   if (b >= nblk) return;
   const uint4* src = reinterpret_cast<const uint4*>(x) + 2 * b;   // the block's 16 values
   const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
@@ -136,6 +150,19 @@ __device__ __forceinline__ void quantize_block(const __nv_bfloat16* __restrict__
     *reinterpret_cast<uint4*>(codes + 16 * b) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
   if (scales) scales[b] = (uint8_t)s8;
+  if (o.xc) {
+    uint32_t pk[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pk[j >> 3] |= q[j] << (4 * (j & 7));
+    *reinterpret_cast<uint2*>(o.xc + 8 * b) = make_uint2(pk[0], pk[1]);
+  }
+  if (o.xsf) {
+    const long long kblk = K >> 4;
+    const long long row = b / kblk;
+    const long long blk = b - row * kblk;
+    const long long c = row / o.rows;
+    o.xsf[bs_scale_offset(c, (int)(row - c * o.rows), blk, K)] = (uint8_t)s8;
+  }
   if (xq) {
     uint32_t o[8];
 #pragma unroll
@@ -159,9 +186,8 @@ __device__ __forceinline__ void quantize_block(const __nv_bfloat16* __restrict__
 // amax_bits[1] for the next call.
 __global__ void __launch_bounds__(256)
     act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, unsigned* amax_bits,
-                     const float* __restrict__ g_w, uint8_t* __restrict__ codes,
-                     uint8_t* __restrict__ scales, __nv_bfloat16* __restrict__ xq,
-                     float* g_x_out, float* g_eff_out) {
+                     const float* __restrict__ g_w, const QuantOut o, float* g_x_out,
+                     float* g_eff_out) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float g = global_scale(*reinterpret_cast<volatile unsigned*>(amax_bits));
@@ -171,7 +197,7 @@ __global__ void __launch_bounds__(256)
     if (g_x_out) *g_x_out = g;
     if (g_eff_out) *g_eff_out = g_w ? __fmul_rn(__ldg(g_w), g) : g;
   }
-  quantize_block(x, b, nblk, g, codes, scales, xq);
+  quantize_block(x, b, nblk, K, g, o);
   // every thread of this CTA has read amax_bits: the last CTA clears it
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -186,9 +212,10 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-cudaError_t launch_act_quant(int M, int K, const void* x, unsigned* amax_bits, const float* g_w,
-                             void* codes, void* scales, void* xq, float* g_x, float* g_eff,
-                             cudaStream_t st) {
+namespace {
+
+cudaError_t launch_quant(int M, int K, const void* x, unsigned* amax_bits, const float* g_w,
+                         const QuantOut& o, float* g_x, float* g_eff, cudaStream_t st) {
   // amax_bits[0..1] are zero between calls (zeroed once when the scratch is
   // allocated, cleared again by the last quantiser CTA of every call)
   cudaLaunchAttribute attr[1];
@@ -207,9 +234,35 @@ cudaError_t launch_act_quant(int M, int K, const void* x, unsigned* amax_bits, c
   const long long nblk = (long long)M * (K / 16);
   cfg.gridDim = dim3((unsigned)((nblk + 255) / 256), 1, 1);
   return cudaLaunchKernelEx(&cfg, act_quant_kernel, static_cast<const __nv_bfloat16*>(x), M, K,
-                            amax_bits, g_w, static_cast<uint8_t*>(codes),
-                            static_cast<uint8_t*>(scales), static_cast<__nv_bfloat16*>(xq), g_x,
-                            g_eff);
+                            amax_bits, g_w, o, g_x, g_eff);
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(int M, int K, const void* x, unsigned* amax_bits, const float* g_w,
+                             void* codes, void* scales, void* xq, float* g_x, float* g_eff,
+                             cudaStream_t st) {
+  QuantOut o;
+  o.codes = static_cast<uint8_t*>(codes);
+  o.scales = static_cast<uint8_t*>(scales);
+  o.xq = static_cast<__nv_bfloat16*>(xq);
+  o.xc = nullptr;
+  o.xsf = nullptr;
+  o.rows = 1;
+  return launch_quant(M, K, x, amax_bits, g_w, o, g_x, g_eff, st);
+}
+
+cudaError_t launch_act_quant_bs(int M, int K, int rows, const void* x, unsigned* amax_bits,
+                                const float* g_w, void* xc, void* xsf, float* g_x, float* g_eff,
+                                cudaStream_t st) {
+  QuantOut o;
+  o.codes = nullptr;
+  o.scales = nullptr;
+  o.xq = nullptr;
+  o.xc = static_cast<uint8_t*>(xc);
+  o.xsf = static_cast<uint8_t*>(xsf);
+  o.rows = rows;
+  return launch_quant(M, K, x, amax_bits, g_w, o, g_x, g_eff, st);
 }
 
 }  // namespace w4

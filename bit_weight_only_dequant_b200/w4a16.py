@@ -19,12 +19,13 @@ LIB_PATH = os.path.join(HERE, "libw4a16.so")
 FMT_INT4_G128 = 0
 FMT_NVFP4_G16 = 1
 FMT_FP8_E4M3 = 2
-FMTS = {"int4": FMT_INT4_G128, "nvfp4": FMT_NVFP4_G16, "fp8": FMT_FP8_E4M3}
+FMT_NVFP4_BS = 3
+FMTS = {"int4": FMT_INT4_G128, "nvfp4": FMT_NVFP4_G16, "fp8": FMT_FP8_E4M3, "nvfp4_bs": FMT_NVFP4_BS}
 
 OK = 0
 ERR_ARG, ERR_SHAPE, ERR_ALIGN, ERR_DEVICE, ERR_CUDA, ERR_TIMEOUT, ERR_NOMEM = -1, -2, -3, -4, -5, -6, -7
 ERR_SCRATCH = -8
-PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+PATH_AUTO, PATH_GEMV, PATH_TC, PATH_BS = 0, 1, 2, 3
 MAX_M = 8192
 
 _lib = None
@@ -47,6 +48,7 @@ _SIGS = {
     "w4a16_quantize_act_nvfp4": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_w4a4": (_i, [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_gemm_w4a4_ex": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_gemm_w4a4_bs": (_i, [_i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_device_status": (_i, [_vp]),
     "w4a16_selftest_wait_timeout": (_i, [_vp]),
     "w4a16_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _i]),
@@ -206,6 +208,11 @@ def w4a16_version():
 # (allocation and marshalling around the calls above)
 
 
+def w4a16_gemm_w4a4_bs(M, N, K, x, packed_w, packed_sf, global_scale_w, y, stream=None):
+    return lib().w4a16_gemm_w4a4_bs(M, N, K, _ptr(x), _ptr(packed_w), _ptr(packed_sf),
+                                    _ptr(global_scale_w), _ptr(y), _stream(stream))
+
+
 def pack_on_device(fmt: str, N: int, K: int, codes, scales, stream=None):
     """Pack logical device tensors; returns (packed_w, packed_scales) uint8 CUDA tensors."""
     import torch
@@ -262,6 +269,18 @@ def gemm_w4a4(x, packed_w, packed_scales, N: int, global_scale_w, y=None, path=P
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     check(w4a16_gemm_w4a4_ex(path, M, N, K, x, packed_w, packed_scales, global_scale_w, y, stream),
           "w4a16_gemm_w4a4")
+    return y
+
+
+def gemm_w4a4_bs(x, packed_w, packed_sf, N: int, global_scale_w, y=None, stream=None):
+    """W4A4 NVFP4 matmul on the block-scaled tensor cores (weights packed with
+    format "nvfp4_bs"); returns y (BF16 [M][N])."""
+    import torch
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    check(w4a16_gemm_w4a4_bs(M, N, K, x, packed_w, packed_sf, global_scale_w, y, stream),
+          "w4a16_gemm_w4a4_bs")
     return y
 
 

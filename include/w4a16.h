@@ -59,6 +59,7 @@ extern "C" {
 #define W4A16_FMT_INT4_G128 0  /* int4 GPTQ, BF16 scale per 128-group */
 #define W4A16_FMT_NVFP4_G16 1  /* e2m1, E4M3 scale per 16-group, fp32 per-tensor scale */
 #define W4A16_FMT_FP8_E4M3 2   /* E4M3 weights (W8A16), fp32 per-tensor scale, no packed scales */
+#define W4A16_FMT_NVFP4_BS 3   /* NVFP4 weights in the block-scaled tensor-core layout (W4A4 only) */
 
 /* Status codes. */
 #define W4A16_OK 0
@@ -78,6 +79,7 @@ extern "C" {
 #define W4A16_PATH_AUTO 0      /* row-count dispatch */
 #define W4A16_PATH_GEMV 1      /* weight-streaming split-K GEMV (mma.sync fragments), M <= 16 */
 #define W4A16_PATH_TC 2        /* tcgen05 tensor-core path (A in tensor memory), M <= 8192 */
+#define W4A16_PATH_BS 3        /* W4A4 block-scaled tensor-core path (w4a16_plan queries only) */
 #define W4A16_GEMV_MAX_M 16
 
 /*
@@ -240,6 +242,29 @@ int w4a16_gemm_w4a4_ex(int path, int M, int N, int K, const void* x_bf16, const 
                        const void* packed_scales, const float* global_scale_w, void* y_bf16,
                        void* stream);
 
+/*
+ * W4A4 NVFP4 on the block-scaled tensor cores (tcgen05.mma kind::mxf4nvf4
+ * with one E4M3 scale per 16 k on both operands): the same result contract as
+ * w4a16_gemm_w4a4 (the same quantiser, run inside the call, then the exact
+ * W4A4 product within the same bound), with the weights packed in the tensor
+ * cores' own layout, format W4A16_FMT_NVFP4_BS (w4a16_pack / w4a16_pack_host
+ * with that format; sizes from w4a16_packed_weight_bytes / _scale_bytes):
+ *   packed_w: [N][K/2] bytes, byte j of row n = code(k = 2j) | code(2j + 1) << 4;
+ *   packed_sf: E4M3 scales in atoms of 128 rows x 64 k (512 bytes), atom
+ *     (n / 128, kb) at ((n / 128) * (K / 64) + kb) * 512, row r = n % 128 and
+ *     16-block j of kb at byte 16 * (r % 32) + 4 * (r / 32) + j; rows past N
+ *     of the last atom row hold 0.
+ * No tensor-core instruction or thread of this path converts a weight: the
+ * tensor cores read the codes from shared memory and the scales from tensor
+ * memory.  1 <= M <= 8192 (chunks of at most 128 activation rows), N >= 1,
+ * K a multiple of 128; every pointer a 16-byte aligned device pointer.  The
+ * library keeps a scratch per (device, stream) for the quantised activations
+ * (M x K/2 codes and their scale atoms) and, when K is split, fp32 partials.
+ */
+int w4a16_gemm_w4a4_bs(int M, int N, int K, const void* x_bf16, const void* packed_w,
+                       const void* packed_sf, const float* global_scale_w, void* y_bf16,
+                       void* stream);
+
 /* The path W4A16_PATH_AUTO would take for these arguments (>0), or a status. */
 int w4a16_gemm_path(int fmt, int M, int N, int K);
 
@@ -260,8 +285,12 @@ int w4a16_device_status(void* stream);
  *         in flight per CTA, K pieces per band, ring depth, groups per piece,
  *         dynamic shared memory bytes;
  *   TC:   row chunks, rows per chunk, padded rows (MMA N), K splits, 64-blocks
- *         per split, work units, CTAs, dynamic shared memory bytes, 0.
- * Returns the path (W4A16_PATH_GEMV or W4A16_PATH_TC) or a negative status.
+ *         per split, work units, CTAs, dynamic shared memory bytes, 0;
+ *   BS (path W4A16_PATH_BS, fmt W4A16_FMT_NVFP4_BS, the plan of
+ *         w4a16_gemm_w4a4_bs): 128-row tiles, row chunks, rows per chunk,
+ *         padded rows (MMA N), K splits, 256-k stages per split, work units,
+ *         CTAs, dynamic shared memory bytes.
+ * Returns the path (W4A16_PATH_GEMV, _TC or _BS) or a negative status.
  */
 int w4a16_plan(int path, int fmt, int M, int N, int K, int fuse, int num_sms, int* out,
                int out_len);

@@ -41,16 +41,22 @@ def test_packed_sizes():
     assert W.w4a16_packed_scale_bytes(1, 8192, 5120) == 8192 * 320
     assert W.w4a16_packed_weight_bytes(0, 17, 128) == 32 * 64          # rows padded to 16
     assert W.w4a16_packed_weight_bytes(0, 16, 100) == 0                 # K not a multiple of 128
-    assert W.w4a16_packed_weight_bytes(3, 16, 128) == 0                 # bad format
+    assert W.w4a16_packed_weight_bytes(4, 16, 128) == 0                 # bad format
     assert W.w4a16_packed_weight_bytes(2, 8192, 5120) == 8192 * 5120    # FP8: a byte per weight
     assert W.w4a16_packed_scale_bytes(2, 8192, 5120) == 0               # per-tensor scale only
     assert W.w4a16_packed_weight_bytes(2, 17, 128) == 32 * 128
+    # block-scaled W4A4 layout: no row padding for the codes, scale atoms of 128 rows x 64 k
+    assert W.w4a16_packed_weight_bytes(3, 17, 128) == 17 * 64
+    assert W.w4a16_packed_scale_bytes(3, 17, 128) == 1 * 2 * 512
+    assert W.w4a16_packed_scale_bytes(3, 8192, 5120) == 64 * 80 * 512 == 8192 * 320
+    assert W.w4a16_packed_scale_bytes(3, 129, 256) == 2 * 4 * 512
 
 
 @pytest.mark.parametrize("fmt,N,K", [("int4", 16, 128), ("int4", 37, 384), ("nvfp4", 16, 128),
-                                     ("nvfp4", 45, 256), ("fp8", 16, 128), ("fp8", 45, 384)])
+                                     ("nvfp4", 45, 256), ("fp8", 16, 128), ("fp8", 45, 384),
+                                     ("nvfp4_bs", 45, 256), ("nvfp4_bs", 130, 384)])
 def test_host_pack_round_trip(fmt, N, K):
-    p = synth.problem(fmt, 7, 1, N, K)
+    p = synth.problem("nvfp4" if fmt == "nvfp4_bs" else fmt, 7, 1, N, K)
     f = W.FMTS[fmt]
     w = np.zeros(W.w4a16_packed_weight_bytes(f, N, K), np.uint8)
     s = np.zeros(W.w4a16_packed_scale_bytes(f, N, K), np.uint8)
@@ -265,3 +271,43 @@ def test_plans_follow_the_dispatcher():
     assert W.w4a16_plan(W.PATH_AUTO, 0, 64, 34816, 5120)[0] == W.PATH_TC
     assert W.w4a16_plan(W.PATH_GEMV, 0, 17, 16, 128)[0] == W.ERR_SHAPE
     assert W.w4a16_plan(W.PATH_TC, 0, 1, 24, 128, fuse=1)[0] == W.ERR_SHAPE      # 2I not a multiple of 32
+
+
+def test_host_pack_block_scaled_layout():
+    # W4A16_FMT_NVFP4_BS, restated from its description: codes [N][K/2] with
+    # k = 2j in the low nibble of byte j; scales in 512-byte atoms per (128-row
+    # tile, 64-k block), row r = a + 32 b and 16-block j at byte 16 a + 4 b + j
+    N, K = 150, 256
+    rng = np.random.default_rng(11)
+    codes = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    s8 = rng.integers(0, 0x7F, size=(N, K // 16)).astype(np.uint8)
+    w = np.zeros(W.w4a16_packed_weight_bytes(3, N, K), np.uint8)
+    s = np.full(W.w4a16_packed_scale_bytes(3, N, K), 0xAA, np.uint8)
+    assert W.w4a16_pack_host(3, N, K, codes, s8, w, s) == W.OK
+    assert np.array_equal(w, (codes[:, 0::2] | (codes[:, 1::2] << 4)).reshape(-1))
+    expect = np.zeros_like(s)
+    for n in range(N):
+        t, r = divmod(n, 128)
+        for gi in range(K // 16):
+            expect[(t * (K // 64) + gi // 4) * 512 + 16 * (r % 32) + 4 * (r // 32) + gi % 4] = s8[n, gi]
+    assert np.array_equal(s, expect)          # rows past N of the last tile hold 0
+    bad = s8.copy()
+    bad[5, 3] = 0x7F
+    assert W.w4a16_pack_host(3, N, K, codes, bad, w, s) == W.ERR_ARG
+
+
+def test_block_scaled_plan_invariants():
+    out = np.zeros(9, np.int32)
+    for M, N, K in [(1, 8192, 5120), (9, 5120, 6144), (64, 34816, 5120), (64, 5120, 17408),
+                    (1, 1, 256), (200, 300, 1024), (8192, 1000, 512), (129, 256, 128)]:
+        r = W.lib().w4a16_plan(W.PATH_BS, 3, M, N, K, 0, 148, out.ctypes.data, 9)
+        assert r == W.PATH_BS, (M, N, K, r)
+        tiles, chunks, rows, mpad, S, sps, units, grid, smem = (int(v) for v in out)
+        T = -(-K // 256)                                         # the last stage may be half
+        assert tiles == -(-N // 128) and chunks == -(-M // 128) and chunks * rows >= M
+        assert rows <= 128 and mpad % 16 == 0 and rows <= mpad <= 128
+        assert S * sps >= T and (S - 1) * sps < T                  # every split holds a stage
+        assert units == tiles * chunks * S and 1 <= grid <= min(units, 148)
+        assert smem <= 227 * 1024
+    assert W.lib().w4a16_plan(W.PATH_BS, 1, 1, 256, 512, 0, 148, out.ctypes.data, 9) == W.ERR_ARG
+    assert W.lib().w4a16_plan(W.PATH_TC, 3, 1, 256, 512, 0, 148, out.ctypes.data, 9) == W.ERR_ARG

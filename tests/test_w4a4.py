@@ -134,3 +134,82 @@ def test_w4a4_rejects_bad_arguments():
     assert W.w4a16_gemm_w4a4(2, 16, 200, x, 1 << 20, 1 << 20, 1 << 20, 1 << 20) == W.ERR_SHAPE
     assert W.w4a16_gemm_w4a4(2, 16, 256, x, 1 << 20, 1 << 20, None, 1 << 20) == W.ERR_ARG
     assert W.w4a16_quantize_act_nvfp4(2, 250, x, 1 << 20, 1 << 20, 1 << 20) == W.ERR_SHAPE
+
+
+# ---------------------------------------------------------------- block-scaled tensor-core path
+
+def _bs_weights(seed, N, K):
+    pw_ = synth.problem("nvfp4", seed, 1, N, K)
+    codes, scales, _ = to_device_problem(pw_)
+    pw, psf = W.pack_on_device("nvfp4_bs", N, K, codes, scales)
+    return pw_, pw, psf
+
+
+def test_block_scaled_device_packer_matches_host_packer():
+    N, K = 300, 384
+    pw_, pw, psf = _bs_weights(980, N, K)
+    w = np.zeros(W.w4a16_packed_weight_bytes(W.FMT_NVFP4_BS, N, K), np.uint8)
+    s = np.zeros(W.w4a16_packed_scale_bytes(W.FMT_NVFP4_BS, N, K), np.uint8)
+    assert W.w4a16_pack_host(W.FMT_NVFP4_BS, N, K, pw_["codes"], pw_["scales"], w, s) == W.OK
+    assert np.array_equal(pw.cpu().numpy(), w)
+    assert np.array_equal(psf.cpu().numpy(), s)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (3, 1000, 1024), (9, 304, 1152), (16, 160, 3072),
+                                   (64, 272, 640), (200, 96, 384), (2, 24, 17408), (1, 1, 128),
+                                   (130, 130, 256), (64, 129, 384), (128, 512, 2048)])
+def test_w4a4_block_scaled_parity_small(M, N, K):
+    t = torch()
+    x_bits = synth.activations(970 + M, M, K)
+    pw_, pw, psf = _bs_weights(971 + M, N, K)
+    x = t.from_numpy(np.ascontiguousarray(x_bits.view(np.int16))).cuda().view(t.bfloat16)
+    y = W.gemm_w4a4_bs(x, pw, psf, N, gscale_tensor(pw_["g"]))
+    t.cuda.synchronize()
+    W.check(W.w4a16_device_status(), "device status")
+    _assert_w4a4_parity(y.float().cpu().numpy().astype(np.float64), x_bits, pw_,
+                        what=f"W4A4 block-scaled M={M} N={N} K={K}")
+
+
+def test_w4a4_block_scaled_parity_wide_activations():
+    # rows spanning many binades: block scales far below the tensor's largest
+    # (E4M3 subnormals and zeros), all-zero blocks, sparse large elements
+    t = torch()
+    M, N, K = 12, 200, 2048
+    x_bits = synth.adversarial_problem("int4", 985, M, 1, K, "wide")["x"].copy()
+    x_bits[1, 64:96] = 0
+    pw_, pw, psf = _bs_weights(986, N, K)
+    x = t.from_numpy(np.ascontiguousarray(x_bits.view(np.int16))).cuda().view(t.bfloat16)
+    y = W.gemm_w4a4_bs(x, pw, psf, N, gscale_tensor(pw_["g"]))
+    t.cuda.synchronize()
+    W.check(W.w4a16_device_status(), "device status")
+    _assert_w4a4_parity(y.float().cpu().numpy().astype(np.float64), x_bits, pw_, what="wide rows")
+
+
+@pytest.mark.parametrize("name,M", [(n, M) for n in ("qkv", "o", "gate_up", "down") for M in (1, 9, 64)])
+def test_w4a4_block_scaled_full_shapes_sampled(name, M):
+    t = torch()
+    K, N = SHAPES[name]
+    seed = 990
+    x_bits = synth.activations(seed, M, K)
+    p = synth.device_problem("nvfp4", seed + 1, 1, N, K)
+    pw, psf = W.pack_on_device("nvfp4_bs", N, K, p["codes"], p["scales"])
+    del p
+    x = t.from_numpy(np.ascontiguousarray(x_bits.view(np.int16))).cuda().view(t.bfloat16)
+    y = W.gemm_w4a4_bs(x, pw, psf, N, gscale_tensor(synth.NVFP4_GLOBAL_SCALE))
+    t.cuda.synchronize()
+    W.check(W.w4a16_device_status(), "device status")
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 1], np.random.default_rng(M).integers(0, N, 40)]))
+    ph = synth.problem("nvfp4", seed + 1, 1, N, K, rows=rows)
+    _assert_w4a4_parity(y.float().cpu().numpy().astype(np.float64), x_bits, ph, cols=rows,
+                        what=f"W4A4 block-scaled {name} M={M}")
+    del pw, psf, y
+    t.cuda.empty_cache()
+
+
+def test_w4a4_block_scaled_rejects_bad_arguments():
+    t = torch()
+    x = t.zeros((2, 256), dtype=t.bfloat16, device="cuda")
+    assert W.w4a16_gemm_w4a4_bs(2, 16, 200, x, 1 << 20, 1 << 20, 1 << 20, 1 << 20) == W.ERR_SHAPE
+    assert W.w4a16_gemm_w4a4_bs(0, 16, 256, x, 1 << 20, 1 << 20, 1 << 20, 1 << 20) == W.ERR_SHAPE
+    assert W.w4a16_gemm_w4a4_bs(2, 16, 256, x, 1 << 20, 1 << 20, None, 1 << 20) == W.ERR_ARG
+    assert W.w4a16_gemm_w4a4_bs(2, 16, 256, x, (1 << 20) + 8, 1 << 20, 1 << 20, 1 << 20) == W.ERR_ALIGN
