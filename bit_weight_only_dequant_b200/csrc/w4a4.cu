@@ -20,10 +20,10 @@
 // The quantised activation x_hat = e2m1(q) * e4m3(s) * g_x: e2m1 * e4m3 has
 // at most 6 significant bits and lies in [2^-10, 2688], so it is exact in
 // BF16 and FP16; the product with g_x is left to the matmul, whose per-tensor
-// scale becomes g_w * g_x.  The matmul itself is then the NVFP4 path of this
-// library on the block-scaled activation values: at decode and verify row
-// counts W4A4 moves the same weight bytes as W4A16, so the same kernels bound
-// it.
+// scale becomes g_w * g_x.  Two matmuls consume the quantiser's outputs: the
+// block-scaled tensor-core kernel (bs.cu), which takes the codes two per byte
+// and the scales in tensor-memory atoms, and the NVFP4 W4A16 paths of this
+// library, which take the block-scaled values as BF16.
 #include "bs.h"
 #include "common.cuh"
 #include "kernels.h"
