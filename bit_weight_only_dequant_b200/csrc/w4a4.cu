@@ -210,6 +210,45 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Small activation tensors (at most kSmallBlocks 16-blocks): one CTA finds
+// amax|x| with a block reduction and quantises every block itself, so the
+// call is one launch instead of two and touches no amax word.
+constexpr int kSmallThreads = 1024;
+constexpr long long kSmallBlocks = kSmallThreads / 2;
+
+__global__ void __launch_bounds__(kSmallThreads)
+    act_quant_small_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
+                           const float* __restrict__ g_w, const QuantOut o, float* g_x_out,
+                           float* g_eff_out) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ uint32_t red[kSmallThreads / 32];
+  const long long n8 = (long long)M * K / 8, nblk = (long long)M * (K >> 4);
+  const uint4* v = reinterpret_cast<const uint4*>(x);
+  uint32_t mx = 0u;
+  for (long long i = threadIdx.x; i < n8; i += kSmallThreads) {
+    const uint4 c = __ldg(v + i);
+    const uint32_t w[4] = {c.x & 0x7FFF7FFFu, c.y & 0x7FFF7FFFu, c.z & 0x7FFF7FFFu,
+                           c.w & 0x7FFF7FFFu};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mx = max(mx, max(w[j] & 0xFFFFu, w[j] >> 16));
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    mx = __reduce_max_sync(0xffffffffu, red[threadIdx.x]);
+    if (threadIdx.x == 0) red[0] = mx;
+  }
+  __syncthreads();
+  const float g = global_scale(red[0] << 16);
+  if (threadIdx.x == 0) {
+    if (g_x_out) *g_x_out = g;
+    if (g_eff_out) *g_eff_out = g_w ? __fmul_rn(__ldg(g_w), g) : g;
+  }
+  for (long long b = threadIdx.x; b < nblk; b += kSmallThreads) quantize_block(x, b, nblk, K, g, o);
+}
+
 }  // namespace
 
 namespace {
@@ -226,6 +265,12 @@ cudaError_t launch_quant(int M, int K, const void* x, unsigned* amax_bits, const
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if ((long long)M * (K / 16) <= kSmallBlocks) {
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(kSmallThreads, 1, 1);
+    return cudaLaunchKernelEx(&cfg, act_quant_small_kernel, static_cast<const __nv_bfloat16*>(x),
+                              M, K, g_w, o, g_x, g_eff);
+  }
   const long long n8 = (long long)M * K / 8;
   cfg.gridDim = dim3((unsigned)min(1184ll, (n8 + 255) / 256), 1, 1);
   cudaError_t e = cudaLaunchKernelEx(&cfg, act_amax_kernel, static_cast<const __nv_bfloat16*>(x),
