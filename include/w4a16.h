@@ -193,8 +193,7 @@ int w4a16_gemm_gate_up_silu_ex(int path, int fmt, int M, int I, int K, const voi
  *   W4A16_ERR_SCRATCH without launching; M > W4A16_GEMV_MAX_M returns
  *   W4A16_ERR_SHAPE.  Calls neither allocate nor free device memory.
  *   The first call on a device resolves the array's device address and sets
- *   the launch attributes of every kernel variant this entry point uses; make
- *   that first call before any stream capture.
+ *   the launch attributes of every kernel variant this entry point uses.
  *   All calls share the array: calls whose GPU work overlaps (different
  *   streams, or threads sharing a device) race and must be serialised by the
  *   caller.  Each call clears, in stream order, the part that must start at
