@@ -793,7 +793,8 @@ def run_native(args, rank, world, local_rank):
 def run_case(specs: str, launches: int):
     """Launch GEMMs a few times each (for profilers).  specs = one or more
     fmt,M,N,K[,path] separated by ';', run in that order; fmt is int4, nvfp4,
-    fp8 or w4a4 (NVFP4 weights, activations quantised by the library)."""
+    fp8, w4a4 (NVFP4 weights, activations quantised by the library) or w4a4bs
+    (the same on the block-scaled tensor cores)."""
     import torch
     from bit_weight_only_dequant_b200 import w4a16 as W
     torch.cuda.set_device(0)
@@ -802,21 +803,24 @@ def run_case(specs: str, launches: int):
         parts = spec.split(",")
         fmt, M, N, K = parts[0], int(parts[1]), int(parts[2]), int(parts[3])
         path = int(parts[4]) if len(parts) > 4 else W.PATH_AUTO
-        wfmt = "nvfp4" if fmt == "w4a4" else fmt
+        wfmt = {"w4a4": "nvfp4", "w4a4bs": "nvfp4_bs"}.get(fmt, fmt)
         f = W.FMTS[wfmt]
         (pw, ps), = make_weights(wfmt, 3, N, K, 1)
-        x = make_x(wfmt, 3, M, K)
+        x = make_x("nvfp4" if wfmt == "nvfp4_bs" else wfmt, 3, M, K)
         y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         g = torch.tensor([1.0 / 448.0], dtype=torch.float32, device="cuda") if wfmt != "int4" else None
         for _ in range(launches):
             if fmt == "w4a4":
                 W.check(W.w4a16_gemm_w4a4_ex(path, M, N, K, x, pw, ps, g, y), "gemm_w4a4")
+            elif fmt == "w4a4bs":
+                W.check(W.w4a16_gemm_w4a4_bs(M, N, K, x, pw, ps, g, y), "gemm_w4a4_bs")
             else:
                 W.check(W.w4a16_gemm_ex(path, f, M, N, K, x, pw, ps, g, y), "gemm")
         torch.cuda.synchronize()
         W.check(W.w4a16_device_status(), "device status")
         out.append({"case": spec, "launches": launches,
-                    "path": W.w4a16_gemm_path(f, M, N, K) if path == W.PATH_AUTO else path})
+                    "path": W.PATH_BS if fmt == "w4a4bs" else
+                    W.w4a16_gemm_path(f, M, N, K) if path == W.PATH_AUTO else path})
         del pw, ps, x, y
         torch.cuda.empty_cache()
     print(json.dumps(out))
