@@ -157,7 +157,8 @@ def test_block_scaled_device_packer_matches_host_packer():
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 512), (3, 1000, 1024), (9, 304, 1152), (16, 160, 3072),
                                    (64, 272, 640), (200, 96, 384), (2, 24, 17408), (1, 1, 128),
-                                   (130, 130, 256), (64, 129, 384), (128, 512, 2048)])
+                                   (130, 130, 256), (64, 129, 384), (128, 512, 2048),
+                                   (1000, 200, 512)])
 def test_w4a4_block_scaled_parity_small(M, N, K):
     t = torch()
     x_bits = synth.activations(970 + M, M, K)
