@@ -882,8 +882,14 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms, int fuse) {
       for (int d = 2; d <= dmax; ++d) {
         if (d == 7) continue;                  // not instantiated
         const int padded = (piece + d - 1) / d * d;
-        const double cost = (double)rounds * (per_group * padded + 1.0) +
-                            (S > 1 ? 3.0 + 0.5 * S : 0.0) + (d < 4 ? 0.5 * (4 - d) : 0.0);
+        double cost = (double)rounds * (per_group * padded + 1.0) +
+                      (S > 1 ? 3.0 + 0.5 * S : 0.0) + (d < 4 ? 0.5 * (4 - d) : 0.0);
+        // one 8-row tile (M <= 8): + the activation staging, which grows with
+        // M x the K slice (a CTA converts its rows' slice before the first
+        // MMA), so splitting K pays at M = 4..8 where it does not at M = 1
+        // (measured on the O and down projections; at M = 9..16 the fit
+        // without it chooses better)
+        if (pl.mt == 1) cost += (S > 1 ? 1.34 : 0.0) + 0.0185 * M * gslice;
         if (cost < best - 1e-9) {
           best = cost;
           pl.S = S;
