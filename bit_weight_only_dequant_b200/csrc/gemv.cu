@@ -882,8 +882,15 @@ GemvPlan plan_gemv(int fmt, int M, int N, int K, int num_sms, int fuse) {
       for (int d = 2; d <= dmax; ++d) {
         if (d == 7) continue;                  // not instantiated
         const int padded = (piece + d - 1) / d * d;
-        double cost = (double)rounds * (per_group * padded + 1.0) +
-                      (S > 1 ? 3.0 + 0.5 * S : 0.0) + (d < 4 ? 0.5 * (4 - d) : 0.0);
+        // plain layers: padding groups copy nothing, so they cost loop
+        // overhead rather than bytes, and a ring shallower than 4 costs in
+        // proportion to the group's bytes (FP8: measured 8.6 -> 7.8 us on
+        // QKV at M = 1 with 4 stages instead of 2); the fused layer keeps
+        // the fit it was measured with
+        const double pad_cost = fuse ? per_group : 0.5;
+        const double shallow = fuse ? 0.5 : 0.25 * per_group;
+        double cost = (double)rounds * (per_group * piece + pad_cost * (padded - piece) + 1.0) +
+                      (S > 1 ? 3.0 + 0.5 * S : 0.0) + (d < 4 ? shallow * (4 - d) : 0.0);
         // one 8-row tile (M <= 8): + the activation staging, which grows with
         // M x the K slice (a CTA converts its rows' slice before the first
         // MMA), so splitting K pays at M = 4..8 where it does not at M = 1
