@@ -593,13 +593,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Per-row power-of-two rescaling of the activations into FP16 (NVFP4 path):
-// row_mul[m] = 2^e with max|x[m]| * 2^-e in [2^14, 2^15).  One CTA per row,
-// eight BF16 values per 16-byte load; the second pass re-reads the row from
-// cache.  K is a multiple of 128, so rows are 16-byte aligned.
+// Per-row power-of-two rescaling of the activations into FP16 (NVFP4 and
+// FP8 paths): row_mul[m] = 2^e with max|x[m]| * 2^-e in [2^14, 2^15).  One
+// CTA per row, eight BF16 values per 16-byte load; the second pass re-reads
+// the row from cache.  K is a multiple of 128, so rows are 16-byte aligned.
+// Launched with programmatic dependent launch: the tensor-core kernel may
+// start at once, and this kernel reads x (and overwrites the FP16 copy the
+// previous call may still be reading) only after the previous kernel on the
+// stream has finished.
 __global__ void __launch_bounds__(256) prep_x_f16_kernel(const __nv_bfloat16* __restrict__ x,
                                                          __half* __restrict__ xh,
                                                          float* __restrict__ row_mul, int K) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int m = blockIdx.x;
   const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)m * K);
   uint4* out = reinterpret_cast<uint4*>(xh + (size_t)m * K);
@@ -791,12 +797,12 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
     while (cur < pl.smem && !smem_set[dev].compare_exchange_weak(cur, pl.smem)) {
     }
   }
-  // int4: programmatic dependent launch, so on each SM freed by the previous
-  // kernel the CTA starts (tensor memory, barriers, an L2 prefetch of its
-  // first weights) before that kernel has finished; every read of an operand
-  // and every write waits for it (griddepcontrol.wait).
-  // Measured 3-8 % faster back to back.  NVFP4 and FP8 follow their own FP16
-  // rescale kernel and keep an ordinary launch (no gain measured there).
+  // Programmatic dependent launch: on each SM freed by the previous kernel
+  // (for NVFP4 and FP8, the FP16 rescale kernel, itself launched the same
+  // way) the CTA starts (tensor memory, barriers, an L2 prefetch of its first
+  // weights) before that kernel has finished; every read of an operand and
+  // every write waits for it (griddepcontrol.wait).  Measured 3-8 % faster
+  // back to back for int4.
   cudaLaunchConfig_t kcfg = {};
   kcfg.gridDim = dim3((unsigned)pl.grid, 1, 1);
   kcfg.blockDim = dim3(kTcThreads, 1, 1);
@@ -806,7 +812,7 @@ cudaError_t launch_t(const TcPlan& pl, const GemmArgs& a, const void* xsrc, cons
   kattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   kattr[0].val.programmaticStreamSerializationAllowed = 1;
   kcfg.attrs = kattr;
-  kcfg.numAttrs = FMT == 0 ? 1 : 0;
+  kcfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&kcfg, tc_kernel<FMT, MPAD>, map, p);
   if (e != cudaSuccess || pl.S == 1) return e;
 
@@ -922,8 +928,17 @@ cudaError_t launch_tc(const TcPlan& pl, const GemmArgs& a, void* xf16_scratch, c
   if (a.fmt == 0) return launch_fmt<0>(pl, a, a.x, nullptr, st);
   __half* xh = static_cast<__half*>(xf16_scratch);
   float* rm = reinterpret_cast<float*>(static_cast<uint8_t*>(xf16_scratch) + (size_t)a.M * a.K * 2);
-  prep_x_f16_kernel<<<a.M, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.x), xh, rm, a.K);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.M, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prep_x_f16_kernel, static_cast<const __nv_bfloat16*>(a.x),
+                                     xh, rm, a.K);
   if (e != cudaSuccess) return e;
   return a.fmt == 1 ? launch_fmt<1>(pl, a, xh, rm, st) : launch_fmt<kFmtFp8>(pl, a, xh, rm, st);
 }

@@ -477,7 +477,8 @@ def test_device_status_is_clean():
 
 
 # ---------------------------------------------------------------- chained launches
-# Every GEMV launch lets the next kernel on the stream start early
+# Every GEMV and tensor-core launch (and the FP16 rescale of the NVFP4 and
+# FP8 tensor-core paths) lets the next kernel on the stream start early
 # (programmatic dependent launch) and waits for the previous one only before
 # it reads the activations.  A chain whose layers feed each other, issued
 # back to back with no host synchronisation (eagerly and as a CUDA graph),
@@ -497,7 +498,8 @@ def _chain_layers(fmt, dims, seed):
 
 
 @pytest.mark.parametrize("fmt,M,path", [("int4", 1, W.PATH_GEMV), ("int4", 4, W.PATH_GEMV),
-                                        ("int4", 9, W.PATH_AUTO), ("nvfp4", 2, W.PATH_GEMV)])
+                                        ("int4", 9, W.PATH_AUTO), ("nvfp4", 2, W.PATH_GEMV),
+                                        ("nvfp4", 9, W.PATH_TC), ("fp8", 16, W.PATH_TC)])
 @pytest.mark.parametrize("graph", [False, True])
 def test_chained_layers_read_their_inputs_after_they_are_written(fmt, M, path, graph):
     t = torch()
