@@ -30,8 +30,16 @@
 // while Mpad <= 64, so the next unit's MMAs overlap the epilogue -- then the
 // scale buffers.  Every mbarrier wait is bounded; a timeout raises the device
 // error word and the CTA drains its copies and MMAs and frees tensor memory.
-// Launched with programmatic dependent launch: before griddepcontrol.wait the
-// CTA only sets up and prefetches its first weight stages into L2.
+// Launched with programmatic dependent launch right behind the library's own
+// activation quantiser.  While the activations fit one 16-row MMA tile the
+// quantiser lets dependents start only after its own griddepcontrol.wait: by
+// the time this kernel starts every kernel ahead of the quantiser has
+// finished, so the weights and their scales are final and the producer loads
+// them at once (overlapping the quantiser); only the activation codes and
+// scales, which the quantiser writes, wait for griddepcontrol.wait.  With
+// more rows (a longer quantiser, which the early weight stream would slow,
+// measured) the CTA only prefetches its first weight stages into L2 before
+// the wait.
 #include <atomic>
 
 #include "bs.h"
@@ -169,30 +177,52 @@ __global__ void __launch_bounds__(kBsThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer (lane 0)
-    if (lane == 0 && (int)blockIdx.x < p.units) {
-      // before the previous kernel on the stream has finished: an L2 hint
-      // for this CTA's first weight stages only
-      int tile, chunk, split, t_lo, t_hi;
-      bs_unit(p, blockIdx.x, tile, chunk, split, t_lo, t_hi);
-      const int t_end = min(t_hi, t_lo + p.nstages);
-      for (int t = t_lo; t < t_end; ++t)
-        asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                         reinterpret_cast<uint64_t>(&wmap)),
-                     "r"(t * 128), "r"(tile * kBsTileRows)
-                     : "memory");
+    // weights may be loaded before the wait (see above); the quantiser uses
+    // the same condition (rows <= 16) for its late trigger
+    const bool early = p.rows <= 16;
+    if (lane == 0 && !early) {
+      if ((int)blockIdx.x < p.units) {
+        int tile, chunk, split, t_lo, t_hi;
+        bs_unit(p, blockIdx.x, tile, chunk, split, t_lo, t_hi);
+        const int t_end = min(t_hi, t_lo + p.nstages);
+        for (int t = t_lo; t < t_end; ++t)
+          asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                           reinterpret_cast<uint64_t>(&wmap)),
+                       "r"(t * 128), "r"(tile * kBsTileRows)
+                       : "memory");
+      }
+      asm volatile("griddepcontrol.wait;" ::: "memory");
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (lane == 0) {
       int s = 0;                      // stage of load `it`
       uint32_t u = 0, it = 0;         // times the stages have wrapped; loads issued
-      bool ok = true;
+      bool ok = true, xr = !early;    // activation loads may be issued (after the wait)
+      int np = 0;                     // stages whose activation loads are held back
+      int pend_s[kBsMaxStages], pend_t[kBsMaxStages], pend_c[kBsMaxStages];
+      auto x_loads = [&](int slot, int t, int chunk) {
+        uint8_t* st = smem + slot * p.stage_bytes;
+        const uint32_t sf = (uint32_t)min(4, p.KB64 - 4 * t) * kBsAtomBytes;
+        tma_load_2d(st + kBsABytes, &xmap, t * 128, chunk * p.rows, full + slot);
+        bulk_g2s(smem_u32(st + kBsABytes + xbytes + kBsSfBytes),
+                 p.sfb + ((size_t)chunk * p.KB64 + 4 * t) * kBsAtomBytes, sf, full + slot);
+      };
+      // the quantiser's outputs are complete: issue the held-back loads
+      auto x_ready = [&]() {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        for (int i = 0; i < np; ++i) x_loads(pend_s[i], pend_t[i], pend_c[i]);
+        np = 0;
+        xr = true;
+      };
       for (int unit = blockIdx.x; unit < p.units && ok; unit += gridDim.x) {
         int tile, chunk, split, t_lo, t_hi;
         bs_unit(p, unit, tile, chunk, split, t_lo, t_hi);
         for (int t = t_lo; t < t_hi; ++t) {
-          if (u > 0 && !tc_wait(empty + s, (u - 1) & 1, abort_flag, p.err)) {
-            ok = false;
-            break;
+          if (u > 0) {
+            if (!xr) x_ready();         // a stage is reused only after its MMAs, which need x
+            if (!tc_wait(empty + s, (u - 1) & 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
           }
           uint8_t* st = smem + s * p.stage_bytes;
           // scale atoms of this stage (2 in a half stage at the end of K);
@@ -200,11 +230,16 @@ __global__ void __launch_bounds__(kBsThreads, 1)
           const uint32_t sf = (uint32_t)min(4, p.KB64 - 4 * t) * kBsAtomBytes;
           mbar_arrive_expect_tx(full + s, (uint32_t)(kBsABytes + xbytes) + 2 * sf);
           tma_load_2d(st, &wmap, t * 128, tile * kBsTileRows, full + s);
-          tma_load_2d(st + kBsABytes, &xmap, t * 128, chunk * p.rows, full + s);
           bulk_g2s(smem_u32(st + kBsABytes + xbytes),
                    p.sfa + ((size_t)tile * p.KB64 + 4 * t) * kBsAtomBytes, sf, full + s);
-          bulk_g2s(smem_u32(st + kBsABytes + xbytes + kBsSfBytes),
-                   p.sfb + ((size_t)chunk * p.KB64 + 4 * t) * kBsAtomBytes, sf, full + s);
+          if (xr) {
+            x_loads(s, t, chunk);
+          } else {
+            pend_s[np] = s;
+            pend_t[np] = t;
+            pend_c[np] = chunk;
+            ++np;
+          }
           ++it;
           if (++s == p.nstages) {
             s = 0;
@@ -212,6 +247,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
           }
         }
       }
+      if (!xr) x_ready();
       // every issued copy lands before the CTA may exit
       const uint32_t first = it > (uint32_t)p.nstages ? it - (uint32_t)p.nstages : 0u;
       for (uint32_t k = first; k < it; ++k)

@@ -430,6 +430,9 @@ int w4a16_gemm_w4a4_bs(int M, int N, int K, const void* x_bf16, const void* pack
     void* unused = nullptr;
     if ((r = workspace(st, 0, nf, 0, &cnt, &ws, &unused)) != W4A16_OK) return r;
   }
+  // the matmul must be the very next launch after the quantiser: it loads
+  // its weights before its dependent-launch wait, relying on the quantiser
+  // starting dependents only once everything ahead of it has finished
   cudaError_t e = w4::launch_act_quant_bs(M, K, pl.rows, x_bf16, amax, global_scale_w, xc, xsf,
                                           nullptr, g_eff, st);
   if (e != cudaSuccess) return W4A16_ERR_CUDA;

@@ -37,9 +37,14 @@ namespace {
 // entry: the quantiser kernel of the previous call cleared it.  Launched with
 // programmatic dependent launch: x may come from the previous kernel.
 __global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __restrict__ x,
-                                                       long long n8, unsigned* amax_bits) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+                                                       long long n8, unsigned* amax_bits,
+                                                       int late_trigger) {
+  // late_trigger: dependents start only once every kernel ahead of this one
+  // has finished (the block-scaled matmul relies on it to load its weights
+  // early); otherwise at once
+  if (!late_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (late_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint4* v = reinterpret_cast<const uint4*>(x);
   uint32_t mx = 0u;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
@@ -187,9 +192,13 @@ __device__ __forceinline__ void quantize_block(const __nv_bfloat16* __restrict__
 __global__ void __launch_bounds__(256)
     act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, unsigned* amax_bits,
                      const float* __restrict__ g_w, const QuantOut o, float* g_x_out,
-                     float* g_eff_out) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+                     float* g_eff_out, int late_trigger) {
+  // late_trigger: dependents start only once every kernel ahead of this one
+  // has finished (the block-scaled matmul relies on it to load its weights
+  // early); otherwise at once
+  if (!late_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (late_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const float g = global_scale(*reinterpret_cast<volatile unsigned*>(amax_bits));
   const long long nblk = (long long)M * (K >> 4);
   const long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -219,9 +228,13 @@ constexpr long long kSmallBlocks = kSmallThreads / 2;
 __global__ void __launch_bounds__(kSmallThreads)
     act_quant_small_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
                            const float* __restrict__ g_w, const QuantOut o, float* g_x_out,
-                           float* g_eff_out) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+                           float* g_eff_out, int late_trigger) {
+  // late_trigger: dependents start only once every kernel ahead of this one
+  // has finished (the block-scaled matmul relies on it to load its weights
+  // early); otherwise at once
+  if (!late_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (late_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ uint32_t red[kSmallThreads / 32];
   const long long n8 = (long long)M * K / 8, nblk = (long long)M * (K >> 4);
   const uint4* v = reinterpret_cast<const uint4*>(x);
@@ -254,7 +267,8 @@ __global__ void __launch_bounds__(kSmallThreads)
 namespace {
 
 cudaError_t launch_quant(int M, int K, const void* x, unsigned* amax_bits, const float* g_w,
-                         const QuantOut& o, float* g_x, float* g_eff, cudaStream_t st) {
+                         const QuantOut& o, float* g_x, float* g_eff, int late_trigger,
+                         cudaStream_t st) {
   // amax_bits[0..1] are zero between calls (zeroed once when the scratch is
   // allocated, cleared again by the last quantiser CTA of every call)
   cudaLaunchAttribute attr[1];
@@ -269,17 +283,17 @@ cudaError_t launch_quant(int M, int K, const void* x, unsigned* amax_bits, const
     cfg.gridDim = dim3(1, 1, 1);
     cfg.blockDim = dim3(kSmallThreads, 1, 1);
     return cudaLaunchKernelEx(&cfg, act_quant_small_kernel, static_cast<const __nv_bfloat16*>(x),
-                              M, K, g_w, o, g_x, g_eff);
+                              M, K, g_w, o, g_x, g_eff, late_trigger);
   }
   const long long n8 = (long long)M * K / 8;
   cfg.gridDim = dim3((unsigned)min(1184ll, (n8 + 255) / 256), 1, 1);
   cudaError_t e = cudaLaunchKernelEx(&cfg, act_amax_kernel, static_cast<const __nv_bfloat16*>(x),
-                                     n8, amax_bits);
+                                     n8, amax_bits, late_trigger);
   if (e != cudaSuccess) return e;
   const long long nblk = (long long)M * (K / 16);
   cfg.gridDim = dim3((unsigned)((nblk + 255) / 256), 1, 1);
   return cudaLaunchKernelEx(&cfg, act_quant_kernel, static_cast<const __nv_bfloat16*>(x), M, K,
-                            amax_bits, g_w, o, g_x, g_eff);
+                            amax_bits, g_w, o, g_x, g_eff, late_trigger);
 }
 
 }  // namespace
@@ -294,7 +308,7 @@ cudaError_t launch_act_quant(int M, int K, const void* x, unsigned* amax_bits, c
   o.xc = nullptr;
   o.xsf = nullptr;
   o.rows = 1;
-  return launch_quant(M, K, x, amax_bits, g_w, o, g_x, g_eff, st);
+  return launch_quant(M, K, x, amax_bits, g_w, o, g_x, g_eff, 0, st);
 }
 
 cudaError_t launch_act_quant_bs(int M, int K, int rows, const void* x, unsigned* amax_bits,
@@ -307,7 +321,9 @@ cudaError_t launch_act_quant_bs(int M, int K, int rows, const void* x, unsigned*
   o.xc = static_cast<uint8_t*>(xc);
   o.xsf = static_cast<uint8_t*>(xsf);
   o.rows = rows;
-  return launch_quant(M, K, x, amax_bits, g_w, o, g_x, g_eff, st);
+  // the block-scaled matmul loads its weights before its own wait while the
+  // activations fit one 16-row MMA tile (bs.cu): start it only after the wait
+  return launch_quant(M, K, x, amax_bits, g_w, o, g_x, g_eff, rows <= 16 ? 1 : 0, st);
 }
 
 }  // namespace w4

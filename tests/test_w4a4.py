@@ -214,3 +214,26 @@ def test_w4a4_block_scaled_rejects_bad_arguments():
     assert W.w4a16_gemm_w4a4_bs(0, 16, 256, x, 1 << 20, 1 << 20, 1 << 20, 1 << 20) == W.ERR_SHAPE
     assert W.w4a16_gemm_w4a4_bs(2, 16, 256, x, 1 << 20, 1 << 20, None, 1 << 20) == W.ERR_ARG
     assert W.w4a16_gemm_w4a4_bs(2, 16, 256, x, (1 << 20) + 8, 1 << 20, 1 << 20, 1 << 20) == W.ERR_ALIGN
+
+
+def test_w4a4_block_scaled_reads_weights_packed_just_before():
+    # the block-scaled matmul loads its weights before its dependent-launch
+    # wait; weights packed by the kernel right before the call (same stream,
+    # no host synchronisation) must still be read complete
+    t = torch()
+    M, N, K = 4, 1024, 4096
+    x_bits = synth.activations(995, M, K)
+    pw_ = synth.problem("nvfp4", 996, 1, N, K)
+    codes, scales, _ = to_device_problem(pw_)
+    x = t.from_numpy(np.ascontiguousarray(x_bits.view(np.int16))).cuda().view(t.bfloat16)
+    g_w = gscale_tensor(pw_["g"])
+    s = t.cuda.Stream()
+    t.cuda.synchronize()
+    with t.cuda.stream(s):
+        for _ in range(3):
+            pw, psf = W.pack_on_device("nvfp4_bs", N, K, codes, scales, stream=s)
+            y = W.gemm_w4a4_bs(x, pw, psf, N, g_w, stream=s)
+    s.synchronize()
+    W.check(W.w4a16_device_status(s), "device status")
+    _assert_w4a4_parity(y.float().cpu().numpy().astype(np.float64), x_bits, pw_,
+                        what="weights packed just before")
